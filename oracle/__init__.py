@@ -1,0 +1,210 @@
+"""NumPy front end of the double-precision CPU oracle (``muse_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference leg of ``bench.py`` import this package.  The product
+path (``gate_cores_b200``) never imports it and shares no code with it.
+
+Each wrapper takes contiguous NumPy arrays (bf16 as ``uint16`` bit patterns,
+f32 as ``float32``) and returns ``(out, lo, hi, mag)``: the core's output in
+its dtype plus the three double arrays described in ``muse_oracle.h``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "muse_oracle.c")
+_LIB = os.path.join(_HERE, "libmuse_oracle.so")
+
+BF16 = 0
+F32 = 1
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, IEEE rounding, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < max(
+        os.path.getmtime(_SRC), os.path.getmtime(os.path.join(_HERE, "muse_oracle.h"))
+    ):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-Wall", "-Wextra",
+             "-fno-fast-math", "-ffp-contract=off", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            P = ctypes.c_void_p
+            i64, i32, f32, c_int = ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_int
+            lib.muse_oracle_version.restype = c_int
+            lib.muse_oracle_round_bf16.argtypes = [P, P, i64]
+            lib.muse_oracle_round_bf16.restype = None
+            lib.muse_oracle_inv_freq.argtypes = [i32, f32, P]
+            lib.muse_oracle_positions.argtypes = [c_int, i64, i64, P, i32, i64, P]
+            lib.muse_oracle_rms_norm.argtypes = [c_int, P, i64, i64, P, f32, f32, P, P, P, P]
+            lib.muse_oracle_input_scale_norm.argtypes = lib.muse_oracle_rms_norm.argtypes
+            lib.muse_oracle_qk_norm_rope.argtypes = [
+                c_int, P, P, i64, i32, i32, i32, P, f32, f32, c_int, c_int, f32,
+                P, P, P, P, P, P, P, P]
+            lib.muse_oracle_output_norm_gate.argtypes = [
+                c_int, P, P, i64, i32, i32, i32, f32, P, P, P, P]
+            lib.muse_oracle_norm_residual.argtypes = [
+                P, c_int, P, i64, i64, P, f32, P, c_int, f32, P, P, P, P]
+            for name in ("muse_oracle_inv_freq", "muse_oracle_positions", "muse_oracle_rms_norm",
+                         "muse_oracle_input_scale_norm", "muse_oracle_qk_norm_rope",
+                         "muse_oracle_output_norm_gate", "muse_oracle_norm_residual"):
+                getattr(lib, name).restype = c_int
+            _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dt(a: np.ndarray) -> int:
+    if a.dtype == np.uint16:
+        return BF16
+    if a.dtype == np.float32:
+        return F32
+    raise TypeError(f"oracle takes uint16 (bf16 bits) or float32 arrays, got {a.dtype}")
+
+
+def _c(a):
+    return None if a is None else np.ascontiguousarray(a)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what}: invalid argument")
+
+
+def version() -> int:
+    return _load().muse_oracle_version()
+
+
+def round_bf16(v) -> np.ndarray:
+    """Nearest bf16 (ties to even) of each double, as uint16 bit patterns."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty(v.shape, dtype=np.uint16)
+    _load().muse_oracle_round_bf16(_ptr(v), _ptr(out), v.size)
+    return out
+
+
+def inv_freq(head_dim: int, base: float) -> np.ndarray:
+    out = np.empty(head_dim // 2, dtype=np.float32)
+    _check(_load().muse_oracle_inv_freq(head_dim, base, _ptr(out)), "inv_freq")
+    return out
+
+
+def positions(layout: int, batch: int = 0, seqlen: int = 0, cu_seqlens=None,
+              total_tokens: int = 0) -> np.ndarray:
+    """Default positions: BSHD (layout 0) t mod seqlen; THD (layout 1) t - cu_seqlens[d]."""
+    if layout == 0:
+        n = batch * seqlen
+        cu = None
+        ns = 0
+    else:
+        cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+        ns = cu.size - 1
+        n = total_tokens
+    out = np.empty(n, dtype=np.int32)
+    _check(_load().muse_oracle_positions(layout, batch, seqlen, _ptr(cu), ns, total_tokens,
+                                         _ptr(out)), "positions")
+    return out
+
+
+def _checks(shape):
+    return (np.empty(shape, np.float64), np.empty(shape, np.float64), np.empty(shape, np.float64))
+
+
+def rms_norm(x, gain=None, gain_offset=0.0, eps=1e-6):
+    x = _c(x)
+    gain = _c(gain)
+    out = np.empty_like(x)
+    lo, hi, mag = _checks(x.shape)
+    hidden = x.shape[-1]
+    rows = x.size // hidden
+    _check(_load().muse_oracle_rms_norm(_dt(x), _ptr(x), rows, hidden, _ptr(gain), gain_offset,
+                                        eps, _ptr(out), _ptr(lo), _ptr(hi), _ptr(mag)), "rms_norm")
+    return out, lo, hi, mag
+
+
+def input_scale_norm(x, gain=None, gain_offset=0.0, eps=1e-6):
+    x = _c(x)
+    gain = _c(gain)
+    out = np.empty_like(x)
+    lo, hi, mag = _checks(x.shape)
+    hidden = x.shape[-1]
+    rows = x.size // hidden
+    _check(_load().muse_oracle_input_scale_norm(_dt(x), _ptr(x), rows, hidden, _ptr(gain),
+                                                gain_offset, eps, _ptr(out), _ptr(lo), _ptr(hi),
+                                                _ptr(mag)), "input_scale_norm")
+    return out, lo, hi, mag
+
+
+def qk_norm_rope(q, k, pos, eps=1e-6, query_scale=1.0, use_rope=True, upcast_rope=True,
+                 rope_base=10000.0):
+    """q [T, Hq, D], k [T, Hkv, D], pos int32 [T].  Returns (q_res, k_res), each (out, lo, hi, mag)."""
+    q = _c(q)
+    k = _c(k)
+    pos = None if pos is None else np.ascontiguousarray(pos, dtype=np.int32)
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    assert k.shape == (T, hkv, d) and k.dtype == q.dtype
+    qo = np.empty_like(q)
+    ko = np.empty_like(k)
+    ql, qh, qm = _checks(q.shape)
+    kl, kh, km = _checks(k.shape)
+    _check(_load().muse_oracle_qk_norm_rope(
+        _dt(q), _ptr(q), _ptr(k), T, hq, hkv, d, _ptr(pos), eps, query_scale, int(use_rope),
+        int(upcast_rope), rope_base, _ptr(qo), _ptr(ql), _ptr(qh), _ptr(qm), _ptr(ko), _ptr(kl),
+        _ptr(kh), _ptr(km)), "qk_norm_rope")
+    return (qo, ql, qh, qm), (ko, kl, kh, km)
+
+
+def output_norm_gate(o, g, norm_group=None, eps=1e-6):
+    """o, g [T, H, D]; norm_group = D (per head, default) or H*D (whole token)."""
+    o = _c(o)
+    g = _c(g)
+    T, heads, d = o.shape
+    assert g.shape == o.shape and g.dtype == o.dtype
+    ng = d if norm_group is None else norm_group
+    out = np.empty_like(o)
+    lo, hi, mag = _checks(o.shape)
+    _check(_load().muse_oracle_output_norm_gate(_dt(o), _ptr(o), _ptr(g), T, heads, d, ng, eps,
+                                                _ptr(out), _ptr(lo), _ptr(hi), _ptr(mag)),
+           "output_norm_gate")
+    return out, lo, hi, mag
+
+
+def norm_residual(stream, branch, theta, gain=None, gain_offset=0.0, input_scale=False,
+                  norm_eps=1e-6):
+    stream = np.ascontiguousarray(stream, dtype=np.float32)
+    branch = _c(branch)
+    theta = np.ascontiguousarray(theta, dtype=np.float32)
+    gain = _c(gain)
+    assert stream.shape == branch.shape
+    hidden = stream.shape[-1]
+    rows = stream.size // hidden
+    out = np.empty_like(stream)
+    lo, hi, mag = _checks(stream.shape)
+    _check(_load().muse_oracle_norm_residual(
+        _ptr(stream), _dt(branch), _ptr(branch), rows, hidden, _ptr(gain), gain_offset,
+        _ptr(theta), int(input_scale), norm_eps, _ptr(out), _ptr(lo), _ptr(hi), _ptr(mag)),
+        "norm_residual")
+    return out, lo, hi, mag

@@ -1,0 +1,432 @@
+/*
+ * muse_oracle.c - plain double-precision CPU oracle for the five Muse Spark
+ * Open normalisation cores.  TEST INFRASTRUCTURE ONLY (see muse_oracle.h):
+ * only tests, the entry module's smoke check and the benchmark's CPU-baseline
+ * leg load it; the CUDA library never does.
+ *
+ * Every function is the definition written out: loops over rows, heads and
+ * pairs; sums of squares, products, square roots, sines, cosines and
+ * exponentials in double; rounding to bf16 or FP32 exactly where the API
+ * reference page "nemo_automodel.components.models.muse_spark.layers" puts a
+ * dtype boundary.  No blocking, fusion or reordering.
+ *
+ * Build: gcc -O2 -std=c11 -fPIC -shared (no -ffast-math: every rounding here
+ * is IEEE round-to-nearest-even).
+ */
+#include "muse_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define DT_BF16 0
+#define DT_F32 1
+
+int muse_oracle_version(void) { return 1; }
+
+/* ---------------------------------------------------------------- rounding */
+
+/* Nearest bfloat16 value to v, ties to even, returned as a double (every
+ * bfloat16 value is exactly representable in double).  bfloat16 keeps 8
+ * significant bits for normal numbers (exponent >= -126) and a fixed spacing
+ * of 2^-133 below that; the largest finite value is (2 - 2^-7) * 2^127. */
+static double bf16_round(double v) {
+    if (isnan(v) || isinf(v) || v == 0.0) return v;
+    double a = fabs(v);
+    int e;
+    frexp(a, &e);              /* a in [2^(e-1), 2^e) */
+    int q = e - 8;             /* spacing of 8 significant bits */
+    if (q < -133) q = -133;    /* subnormal spacing */
+    double s = ldexp(a, -q);   /* exact scaling */
+    double r = nearbyint(s);   /* default rounding mode: ties to even */
+    double res = ldexp(r, q);
+    if (res >= 0x1p128) res = INFINITY;
+    return copysign(res, v);
+}
+
+static uint16_t bf16_bits(double rounded) {
+    if (isnan(rounded)) return signbit(rounded) ? 0xFFC0u : 0x7FC0u;
+    float f = (float)rounded; /* exact: rounded is a bfloat16 value */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return (uint16_t)(u >> 16);
+}
+
+static double bf16_value(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* Round to the tensor dtype. */
+static double cast_to(int dtype, double v) {
+    return dtype == DT_BF16 ? bf16_round(v) : (double)(float)v;
+}
+
+static double load_elem(int dtype, const void* p, int64_t i) {
+    return dtype == DT_BF16 ? bf16_value(((const uint16_t*)p)[i])
+                            : (double)((const float*)p)[i];
+}
+
+/* Store v (not yet rounded) in the tensor dtype. */
+static void store_elem(int dtype, void* p, int64_t i, double v) {
+    if (dtype == DT_BF16)
+        ((uint16_t*)p)[i] = bf16_bits(bf16_round(v));
+    else
+        ((float*)p)[i] = (float)v;
+}
+
+/* The values an intermediate cast of the real value v may take.  c[0] is the
+ * round-to-nearest-even result.  For bf16, when v lies within
+ * MUSE_ORACLE_AMBIG_REL * |v| of a rounding midpoint, the other neighbour is
+ * returned as c[1] too (an FP32 evaluation of v can land on either side).
+ * FP32 casts keep one value; their evaluation error is continuous and is
+ * covered by the checker's allowance. */
+static int cast_candidates(int dtype, double v, double c[2]) {
+    c[0] = cast_to(dtype, v);
+    if (dtype != DT_BF16) return 1;
+    double d = fabs(v) * MUSE_ORACLE_AMBIG_REL;
+    double lo = bf16_round(v - d), hi = bf16_round(v + d);
+    if (lo == hi) return 1;
+    c[1] = (lo == c[0]) ? hi : lo;
+    return 2;
+}
+
+void muse_oracle_round_bf16(const double* v, uint16_t* bits, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) bits[i] = bf16_bits(bf16_round(v[i]));
+}
+
+/* ------------------------------------------------------------------- RoPE */
+
+int muse_oracle_inv_freq(int32_t head_dim, float base, float* inv_freq) {
+    if (head_dim <= 0 || (head_dim & 1) || !(base > 0.0f) || !inv_freq) return -1;
+    for (int32_t i = 0; i < head_dim / 2; ++i)
+        inv_freq[i] = (float)pow((double)base, -(2.0 * (double)i) / (double)head_dim);
+    return 0;
+}
+
+int muse_oracle_positions(int layout, int64_t batch, int64_t seqlen,
+                          const int32_t* cu_seqlens, int32_t num_seqs,
+                          int64_t total_tokens, int32_t* pos) {
+    if (!pos) return -1;
+    if (layout == 0) {
+        if (batch < 0 || seqlen <= 0) return -1;
+        for (int64_t t = 0; t < batch * seqlen; ++t) pos[t] = (int32_t)(t % seqlen);
+        return 0;
+    }
+    if (layout != 1 || !cu_seqlens || num_seqs < 0) return -1;
+    if (cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != total_tokens) return -1;
+    for (int32_t d = 0; d < num_seqs; ++d) {
+        if (cu_seqlens[d + 1] < cu_seqlens[d]) return -1;
+        for (int64_t t = cu_seqlens[d]; t < cu_seqlens[d + 1]; ++t)
+            pos[t] = (int32_t)(t - cu_seqlens[d]);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------ shared bits */
+
+/* r(x) = 1 / sqrt(mean of squares + eps): "Stabilizer added to the mean
+ * squared activation" (parameter eps of _rms_norm_core). */
+static double inv_rms(double sum_sq, int64_t width, float eps) {
+    return 1.0 / sqrt(sum_sq / (double)width + (double)eps);
+}
+
+/* Effective gain: the zero-centered checkpoint gain plus its offset, summed in
+ * FP32 (MuseSparkRMSNorm: gain_center, effective_weight returns the actual
+ * multiplicative gain). */
+static double eff_gain(const float* gain, float offset, int64_t j) {
+    if (!gain) return 1.0;
+    float w = gain[j] + offset; /* FP32 addition */
+    return (double)w;
+}
+
+static void put_check(double* lo, double* hi, double* mag, int64_t i,
+                      double l, double h, double m) {
+    if (lo) lo[i] = l;
+    if (hi) hi[i] = h;
+    if (mag) mag[i] = m;
+}
+
+static int valid_dtype(int dt) { return dt == DT_BF16 || dt == DT_F32; }
+
+/* ------------------------------------------------------------------ core 1 */
+
+/* _rms_norm_core: normalise in FP32, then apply the effective gain before the
+ * one output cast; the output keeps the input dtype. */
+int muse_oracle_rms_norm(int dtype, const void* x, int64_t rows, int64_t hidden,
+                         const float* gain, float gain_offset, float eps,
+                         void* out, double* lo, double* hi, double* mag) {
+    if (!valid_dtype(dtype) || rows < 0 || hidden <= 0 || (rows && (!x || !out))) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        const int64_t base = r * hidden;
+        double ss = 0.0;
+        for (int64_t j = 0; j < hidden; ++j) {
+            double xj = load_elem(dtype, x, base + j);
+            ss += xj * xj;
+        }
+        const double inv = inv_rms(ss, hidden, eps);
+        for (int64_t j = 0; j < hidden; ++j) {
+            double y = load_elem(dtype, x, base + j) * inv;
+            if (gain) y *= eff_gain(gain, gain_offset, j);
+            store_elem(dtype, out, base + j, y);
+            put_check(lo, hi, mag, base + j, y, y, fabs(y));
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ core 2 */
+
+/* _input_scale_norm_core: apply the effective gain first, then a
+ * parameter-free RMS normalisation whose eps is added to the mean square of
+ * the scaled activation. */
+int muse_oracle_input_scale_norm(int dtype, const void* x, int64_t rows, int64_t hidden,
+                                 const float* gain, float gain_offset, float eps,
+                                 void* out, double* lo, double* hi, double* mag) {
+    if (!valid_dtype(dtype) || rows < 0 || hidden <= 0 || (rows && (!x || !out))) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        const int64_t base = r * hidden;
+        double ss = 0.0;
+        for (int64_t j = 0; j < hidden; ++j) {
+            double z = load_elem(dtype, x, base + j) * eff_gain(gain, gain_offset, j);
+            ss += z * z;
+        }
+        const double inv = inv_rms(ss, hidden, eps);
+        for (int64_t j = 0; j < hidden; ++j) {
+            double z = load_elem(dtype, x, base + j) * eff_gain(gain, gain_offset, j);
+            double y = z * inv;
+            store_elem(dtype, out, base + j, y);
+            put_check(lo, hi, mag, base + j, y, y, fabs(y));
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ core 3 */
+
+#define MAXC 4 /* a value with up to two casts in doubt has at most 4 candidates */
+
+typedef struct {
+    int n;
+    double v[MAXC];
+} cand_set;
+
+static void cand_add(cand_set* s, double v) {
+    for (int i = 0; i < s->n; ++i)
+        if (s->v[i] == v) return;
+    if (s->n < MAXC) s->v[s->n++] = v;
+}
+
+/* One head of core 3: normalise `width` elements of x over the head, cast,
+ * and (query heads) scale and cast again.  Fills the candidate set of each
+ * element; element j's primary value is cs[j].v[0]. */
+static void qk_head_norm(int dtype, const void* x, int64_t base, int32_t d, float eps,
+                         int is_query, float query_scale, cand_set* cs) {
+    double ss = 0.0;
+    for (int32_t j = 0; j < d; ++j) {
+        double xj = load_elem(dtype, x, base + j);
+        ss += xj * xj;
+    }
+    const double inv = inv_rms(ss, d, eps);
+    for (int32_t j = 0; j < d; ++j) {
+        double c[2];
+        int nc = cast_candidates(dtype, load_elem(dtype, x, base + j) * inv, c);
+        cand_set s = {0, {0}};
+        if (!is_query) {
+            for (int i = 0; i < nc; ++i) cand_add(&s, c[i]);
+        } else {
+            /* query_scale: "Multiplier applied after the normalized query's
+             * dtype cast" - the scaled value is cast to the Q dtype again. */
+            for (int i = 0; i < nc; ++i) {
+                double c2[2];
+                int n2 = cast_candidates(dtype, c[i] * (double)query_scale, c2);
+                for (int k = 0; k < n2; ++k) cand_add(&s, c2[k]);
+            }
+        }
+        cs[j] = s;
+    }
+}
+
+static void minmax_upd(double v, double* mn, double* mx) {
+    if (v < *mn) *mn = v;
+    if (v > *mx) *mx = v;
+}
+
+/* Rotate one head's normalised pairs and write outputs + check arrays. */
+static void qk_head_out(int dtype, const cand_set* cs, int32_t d, const float* inv_freq,
+                        int32_t pos, int use_rope, int upcast_rope, void* out,
+                        double* lo, double* hi, double* mag, int64_t base) {
+    if (!use_rope) {
+        for (int32_t j = 0; j < d; ++j) {
+            double mn = INFINITY, mx = -INFINITY;
+            for (int i = 0; i < cs[j].n; ++i) minmax_upd(cs[j].v[i], &mn, &mx);
+            store_elem(dtype, out, base + j, cs[j].v[0]);
+            put_check(lo, hi, mag, base + j, mn, mx, fabs(cs[j].v[0]));
+        }
+        return;
+    }
+    const int fp32_rotation = upcast_rope || dtype == DT_F32;
+    for (int32_t i = 0; i < d / 2; ++i) {
+        const cand_set* A = &cs[2 * i];
+        const cand_set* B = &cs[2 * i + 1];
+        /* Angle in FP32: f32(pos) times the FP32 frequency, one FP32 rounding. */
+        const float phi = (float)pos * inv_freq[i];
+        const double c = cos((double)phi), s = sin((double)phi);
+        double mn0 = INFINITY, mx0 = -INFINITY, mn1 = INFINITY, mx1 = -INFINITY;
+        double m0 = 0.0, m1 = 0.0, y0p = 0.0, y1p = 0.0;
+        if (fp32_rotation) {
+            /* "The original checkpoint computes the rotation in FP32." */
+            for (int ia = 0; ia < A->n; ++ia)
+                for (int ib = 0; ib < B->n; ++ib) {
+                    const double a = A->v[ia], b = B->v[ib];
+                    const double y0 = a * c - b * s;
+                    const double y1 = a * s + b * c;
+                    minmax_upd(y0, &mn0, &mx0);
+                    minmax_upd(y1, &mn1, &mx1);
+                    m0 = fmax(m0, fabs(a * c) + fabs(b * s));
+                    m1 = fmax(m1, fabs(a * s) + fabs(b * c));
+                    if (ia == 0 && ib == 0) { y0p = y0; y1p = y1; }
+                }
+        } else {
+            /* "The HF release rounds both products in the Q/K dtype before
+             * adding them": cos/sin are cast to the Q/K dtype, each product is
+             * rounded to it, and the sum is cast once more.  Every step after
+             * the candidate casts is exact in FP32, so mag stays 0. */
+            double C[2], S[2];
+            const int nC = cast_candidates(dtype, c, C);
+            const int nS = cast_candidates(dtype, s, S);
+            for (int ia = 0; ia < A->n; ++ia)
+                for (int ib = 0; ib < B->n; ++ib)
+                    for (int ic = 0; ic < nC; ++ic)
+                        for (int is = 0; is < nS; ++is) {
+                            const double a = A->v[ia], b = B->v[ib];
+                            const double y0 = cast_to(dtype, a * C[ic]) - cast_to(dtype, b * S[is]);
+                            const double y1 = cast_to(dtype, a * S[is]) + cast_to(dtype, b * C[ic]);
+                            minmax_upd(y0, &mn0, &mx0);
+                            minmax_upd(y1, &mn1, &mx1);
+                            if (ia == 0 && ib == 0 && ic == 0 && is == 0) { y0p = y0; y1p = y1; }
+                        }
+        }
+        store_elem(dtype, out, base + 2 * i, y0p);
+        store_elem(dtype, out, base + 2 * i + 1, y1p);
+        put_check(lo, hi, mag, base + 2 * i, mn0, mx0, m0);
+        put_check(lo, hi, mag, base + 2 * i + 1, mn1, mx1, m1);
+    }
+}
+
+/* _qk_norm_rope_core: per-head FP32 RMS normalisation of Q and K cast back to
+ * their dtype, query_scale after the query's cast, then adjacent-pair RoPE
+ * (pairs (2i, 2i+1), the native checkpoint's convention) in FP32 (legacy) or
+ * in the Q/K dtype (v2).  K is never scaled. */
+int muse_oracle_qk_norm_rope(int dtype, const void* q, const void* k, int64_t tokens,
+                             int32_t hq, int32_t hkv, int32_t head_dim,
+                             const int32_t* pos, float eps, float query_scale,
+                             int use_rope, int upcast_rope, float rope_base,
+                             void* q_out, double* q_lo, double* q_hi, double* q_mag,
+                             void* k_out, double* k_lo, double* k_hi, double* k_mag) {
+    if (!valid_dtype(dtype) || tokens < 0 || hq <= 0 || hkv <= 0 || head_dim <= 0 ||
+        (head_dim & 1))
+        return -1;
+    if (tokens && (!q || !k || !q_out || !k_out || (use_rope && !pos))) return -1;
+    float* inv_freq = (float*)malloc(sizeof(float) * (size_t)(head_dim / 2));
+    cand_set* cs = (cand_set*)malloc(sizeof(cand_set) * (size_t)head_dim);
+    if (!inv_freq || !cs) { free(inv_freq); free(cs); return -1; }
+    if (use_rope && muse_oracle_inv_freq(head_dim, rope_base, inv_freq) != 0) {
+        free(inv_freq); free(cs); return -1;
+    }
+    for (int64_t t = 0; t < tokens; ++t) {
+        const int32_t p = use_rope ? pos[t] : 0;
+        for (int32_t h = 0; h < hq; ++h) {
+            const int64_t base = (t * hq + h) * (int64_t)head_dim;
+            qk_head_norm(dtype, q, base, head_dim, eps, 1, query_scale, cs);
+            qk_head_out(dtype, cs, head_dim, inv_freq, p, use_rope, upcast_rope, q_out,
+                        q_lo, q_hi, q_mag, base);
+        }
+        for (int32_t h = 0; h < hkv; ++h) {
+            const int64_t base = (t * hkv + h) * (int64_t)head_dim;
+            qk_head_norm(dtype, k, base, head_dim, eps, 0, 1.0f, cs);
+            qk_head_out(dtype, cs, head_dim, inv_freq, p, use_rope, upcast_rope, k_out,
+                        k_lo, k_hi, k_mag, base);
+        }
+    }
+    free(inv_freq);
+    free(cs);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ core 4 */
+
+/* _output_norm_gate_core: parameter-free RMS normalisation of the attention
+ * output times the sigmoid of the gate projection, both in FP32, one cast to
+ * the original dtype. */
+int muse_oracle_output_norm_gate(int dtype, const void* o, const void* g, int64_t tokens,
+                                 int32_t heads, int32_t head_dim, int32_t norm_group,
+                                 float eps, void* out, double* lo, double* hi, double* mag) {
+    if (!valid_dtype(dtype) || tokens < 0 || heads <= 0 || head_dim <= 0) return -1;
+    const int64_t width = (int64_t)heads * head_dim;
+    if (norm_group != head_dim && norm_group != width) return -1;
+    if (tokens && (!o || !g || !out)) return -1;
+    const int64_t groups = tokens * width / norm_group;
+    for (int64_t gi = 0; gi < groups; ++gi) {
+        const int64_t base = gi * norm_group;
+        double ss = 0.0;
+        for (int32_t j = 0; j < norm_group; ++j) {
+            double oj = load_elem(dtype, o, base + j);
+            ss += oj * oj;
+        }
+        const double inv = inv_rms(ss, norm_group, eps);
+        for (int32_t j = 0; j < norm_group; ++j) {
+            const double sig = 1.0 / (1.0 + exp(-load_elem(dtype, g, base + j)));
+            const double y = load_elem(dtype, o, base + j) * inv * sig;
+            store_elem(dtype, out, base + j, y);
+            put_check(lo, hi, mag, base + j, y, y, fabs(y));
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ core 5 */
+
+/* _norm_residual_core with the declared learned blend
+ * h' = cos(theta) * h + sin(theta) * nb: the branch is normalised (gain after
+ * the norm, or before it when input_scale is set), cast back to the branch
+ * dtype ("Normalization casts back to this dtype before residual blending"),
+ * then blended into the FP32 stream per channel. */
+int muse_oracle_norm_residual(const float* stream, int branch_dtype, const void* branch,
+                              int64_t rows, int64_t hidden, const float* gain,
+                              float gain_offset, const float* theta, int input_scale,
+                              float norm_eps, float* out, double* lo, double* hi,
+                              double* mag) {
+    if (!valid_dtype(branch_dtype) || rows < 0 || hidden <= 0) return -1;
+    if (rows && (!stream || !branch || !out || !theta)) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        const int64_t base = r * hidden;
+        double ss = 0.0;
+        for (int64_t j = 0; j < hidden; ++j) {
+            double b = load_elem(branch_dtype, branch, base + j);
+            if (input_scale) b *= eff_gain(gain, gain_offset, j);
+            ss += b * b;
+        }
+        const double inv = inv_rms(ss, hidden, norm_eps);
+        for (int64_t j = 0; j < hidden; ++j) {
+            const double b = load_elem(branch_dtype, branch, base + j);
+            const double w = eff_gain(gain, gain_offset, j);
+            const double v = input_scale ? (b * w) * inv : (b * inv) * w;
+            double nb[2];
+            const int n = cast_candidates(branch_dtype, v, nb);
+            const double c = cos((double)theta[j]), s = sin((double)theta[j]);
+            const double h = (double)stream[base + j];
+            double mn = INFINITY, mx = -INFINITY, m = 0.0;
+            for (int i = 0; i < n; ++i) {
+                const double y = c * h + s * nb[i];
+                minmax_upd(y, &mn, &mx);
+                m = fmax(m, fabs(c * h) + fabs(s * nb[i]));
+            }
+            out[base + j] = (float)(c * h + s * nb[0]);
+            put_check(lo, hi, mag, base + j, mn, mx, m);
+        }
+    }
+    return 0;
+}

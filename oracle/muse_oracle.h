@@ -1,0 +1,126 @@
+/*
+ * muse_oracle.h - plain, slow, double-precision CPU oracle for the five fused
+ * per-token normalisation cores of the Muse Spark Open decoder layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check of the entry
+ * module and the benchmark's CPU-baseline leg may load this library.  It
+ * shares no code, header, table or constant with the CUDA library.
+ *
+ * Source of every definition: the NeMo AutoModel API reference page
+ * "nemo_automodel.components.models.muse_spark.layers" (versions 0.4 and
+ * latest), entries _rms_norm_core, _input_scale_norm_core, _qk_norm_rope_core,
+ * _output_norm_gate_core, _norm_residual_core, apply_rotary_embedding,
+ * MuseSparkRotaryEmbedding, MuseSparkRMSNorm and MuseSparkResidual.  Where the
+ * page leaves a step open the reading is stated beside the function.
+ *
+ * Conventions
+ *   - bf16 tensors are passed as uint16_t bit patterns, f32 tensors as float.
+ *   - dtype: 0 = bf16, 1 = f32.
+ *   - All tensors are contiguous and row-major.
+ *   - Every function writes `out` in the output dtype (what the pages' core
+ *     returns) and, when the pointers are not NULL, three double arrays of the
+ *     same element count used by parity checks:
+ *       lo[i], hi[i]  the smallest and largest exact (real-valued) result
+ *                     before the final cast, over every bf16 value that an
+ *                     intermediate cast may legitimately take (see below);
+ *                     lo == hi when no intermediate cast is in doubt;
+ *       mag[i]        the sum of the magnitudes of the terms that form the
+ *                     result before its final cast (|y| for a plain product,
+ *                     |a*c| + |b*s| for a rotation, |cos*h| + |sin*nb| for the
+ *                     residual blend).  A checker scales its FP32 evaluation
+ *                     allowance by it.
+ *   - Intermediate casts to bf16 (the normalised Q/K cast, the query_scale
+ *     cast, the v2 rotation's cos/sin casts, the branch cast before the
+ *     residual blend) are taken to round-to-nearest-even.  An FP32
+ *     evaluation of the same real value differs from it by far less than
+ *     2^-20 relative; when the real value lies within 2^-20 (relative) of a
+ *     bf16 rounding midpoint, both neighbouring bf16 values are admissible
+ *     results of that cast and the oracle carries both forward.
+ *   - Return value: 0 on success, -1 on an invalid argument.
+ */
+#ifndef MUSE_ORACLE_H
+#define MUSE_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Relative distance to a bf16 rounding midpoint below which an intermediate
+ * cast is treated as admitting both neighbours. */
+#define MUSE_ORACLE_AMBIG_REL 0x1p-20
+
+int muse_oracle_version(void);
+
+/* Round each double to the nearest bfloat16 (ties to even) and return its
+ * bit pattern.  NaN maps to a quiet NaN of the same sign. */
+void muse_oracle_round_bf16(const double* v, uint16_t* bits, int64_t n);
+
+/* FP32 RoPE inverse frequencies: inv_freq[i] = f32(base^(-2i/head_dim)),
+ * i = 0 .. head_dim/2 - 1 (MuseSparkRotaryEmbedding: FP32 frequencies,
+ * cos/sin of width head_dim/2). */
+int muse_oracle_inv_freq(int32_t head_dim, float base, float* inv_freq);
+
+/* Positions used when the caller passes none.
+ *   layout 0 (BSHD): tokens = batch*seqlen, pos[t] = t mod seqlen.
+ *   layout 1 (THD):  pos[t] = t - cu_seqlens[d] for the document d whose
+ *                    range [cu_seqlens[d], cu_seqlens[d+1]) holds t.
+ * cu_seqlens (THD only) has num_seqs+1 entries, starts at 0, does not
+ * decrease and ends at total_tokens. */
+int muse_oracle_positions(int layout, int64_t batch, int64_t seqlen,
+                          const int32_t* cu_seqlens, int32_t num_seqs,
+                          int64_t total_tokens, int32_t* pos);
+
+/* Core 1, _rms_norm_core: y = cast((x * r(x)) * w_eff), r(x) = 1/sqrt(mean(x^2)+eps),
+ * w_eff[j] = f32(gain[j] + gain_offset); no gain multiply when gain == NULL. */
+int muse_oracle_rms_norm(int dtype, const void* x, int64_t rows, int64_t hidden,
+                         const float* gain, float gain_offset, float eps,
+                         void* out, double* lo, double* hi, double* mag);
+
+/* Core 2, _input_scale_norm_core: z = x * w_eff, y = cast(z * r(z)). */
+int muse_oracle_input_scale_norm(int dtype, const void* x, int64_t rows, int64_t hidden,
+                                 const float* gain, float gain_offset, float eps,
+                                 void* out, double* lo, double* hi, double* mag);
+
+/* Core 3, _qk_norm_rope_core, on q [tokens, hq, d] and k [tokens, hkv, d]
+ * with explicit positions pos[tokens]:
+ *   n = cast(x * r(x)) per head over d;
+ *   query heads only: n = cast(n * query_scale);
+ *   use_rope: pairs (2i, 2i+1), phi = f32(f32(pos) * inv_freq[i]),
+ *     FP32 rotation (upcast_rope != 0, or dtype f32):
+ *        y0 = a cos(phi) - b sin(phi), y1 = a sin(phi) + b cos(phi), one cast;
+ *     bf16 rotation (upcast_rope == 0, dtype bf16):
+ *        c = bf16(cos phi), s = bf16(sin phi),
+ *        y0 = bf16(bf16(a c) - bf16(b s)), y1 = bf16(bf16(a s) + bf16(b c)).
+ * The *_lo/_hi/_mag arrays may be NULL. */
+int muse_oracle_qk_norm_rope(int dtype, const void* q, const void* k, int64_t tokens,
+                             int32_t hq, int32_t hkv, int32_t head_dim,
+                             const int32_t* pos, float eps, float query_scale,
+                             int use_rope, int upcast_rope, float rope_base,
+                             void* q_out, double* q_lo, double* q_hi, double* q_mag,
+                             void* k_out, double* k_lo, double* k_hi, double* k_mag);
+
+/* Core 4, _output_norm_gate_core, on o and g [tokens, heads, head_dim]:
+ * y = cast(o * r(o) * sigmoid(g)), r over consecutive groups of norm_group
+ * elements (norm_group = head_dim: per head; = heads*head_dim: whole token),
+ * sigmoid(g) = 1/(1+exp(-g)). */
+int muse_oracle_output_norm_gate(int dtype, const void* o, const void* g, int64_t tokens,
+                                 int32_t heads, int32_t head_dim, int32_t norm_group,
+                                 float eps, void* out, double* lo, double* hi, double* mag);
+
+/* Core 5, _norm_residual_core with the declared blend:
+ *   nb = cast_branch(normed(branch)), normed = core 1 form (input_scale == 0)
+ *        or core 2 form (input_scale != 0) with w_eff and norm_eps;
+ *   h' = f32(cos(theta) * h + sin(theta) * nb), per channel theta (FP32). */
+int muse_oracle_norm_residual(const float* stream, int branch_dtype, const void* branch,
+                              int64_t rows, int64_t hidden, const float* gain,
+                              float gain_offset, const float* theta, int input_scale,
+                              float norm_eps, float* out, double* lo, double* hi,
+                              double* mag);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUSE_ORACLE_H */
