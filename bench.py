@@ -1,0 +1,459 @@
+#!/usr/bin/env python
+"""Benchmark of the five fused normalisation cores on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic
+decoder-layer activations: rms_norm, input_scale_norm, qk_norm_rope,
+output_norm_gate and norm_residual, each a single CUDA kernel launched through
+the C ABI.  Default workload: prefill, B=2 x S=4096 tokens, H=4096, 32 Q / 8 KV
+heads of 128.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (weak scaling, no collective on the data path): each rank runs the
+same step on its own batch; launch with torch.distributed.run.  Prints one
+JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gate_cores_b200 import cores, inputs  # noqa: E402
+from gate_cores_b200.inputs import WORKLOADS, num_tokens  # noqa: E402
+
+CORE_ORDER = inputs.CORES
+METRIC = "tokens/s and effective HBM GB/s per fused core vs measured ~8 TB/s peak"
+DOMINANT = "norm_residual"  # largest algorithmic byte count of the five
+KERNEL_NAMES = {c: c + "_kernel" for c in inputs.CORES}
+VARIANT = {"rms_norm": "zero-centered gain (offset 1)", "input_scale_norm": "gain U(0.5,1.5)",
+           "qk_norm_rope": "RoPE in FP32 (legacy), query_scale 1, BSHD-derived positions",
+           "output_norm_gate": "one norm per head", "norm_residual": "gain after the norm"}
+
+
+def algo_bytes(wl, core: str, tokens: int) -> int:
+    """Minimum HBM bytes of one launch: every input read once, every output written once."""
+    H, D = wl.hidden, wl.head_dim
+    per_tok = {"rms_norm": 4 * H, "input_scale_norm": 4 * H,
+               "qk_norm_rope": 4 * (wl.hq + wl.hkv) * D + (4 if wl.positions == "uniform" else 0),
+               "output_norm_gate": 6 * wl.hq * D, "norm_residual": 10 * H}[core]
+    fixed = {"rms_norm": 4 * H, "input_scale_norm": 4 * H, "qk_norm_rope": 0,
+             "output_norm_gate": 0, "norm_residual": 8 * H}[core]
+    return per_tok * tokens + fixed
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ distributed
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def allreduce_max(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the GPU is under load."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, period_ms: int = 20):
+        self.proc = None
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 f"-lms={period_ms}"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r for r in csv.reader(io.StringIO(self.f.read())) if len(r) >= 9]
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ our arm
+
+class Step:
+    """Device-resident inputs and outputs of the five cores for one batch."""
+
+    def __init__(self, wl, seed: int):
+        self.wl = wl
+        self.T = num_tokens(wl, seed)
+        self.host = {c: inputs.make_inputs(wl, c, seed=seed, zero_centered=(c != "input_scale_norm"))
+                     for c in CORE_ORDER}
+        self.dev = {c: {k: (None if v is None else v.cuda()) for k, v in ci.tensors.items()}
+                    for c, ci in self.host.items()}
+        d = self.dev
+        self.out = {
+            "rms_norm": torch.empty_like(d["rms_norm"]["x"]),
+            "input_scale_norm": torch.empty_like(d["input_scale_norm"]["x"]),
+            "qk_q": torch.empty_like(d["qk_norm_rope"]["q"]),
+            "qk_k": torch.empty_like(d["qk_norm_rope"]["k"]),
+            "output_norm_gate": torch.empty_like(d["output_norm_gate"]["o"]),
+            "norm_residual": torch.empty_like(d["norm_residual"]["stream"]),
+        }
+        B, S = wl.batch, wl.seqlen
+        q, k = d["qk_norm_rope"]["q"], d["qk_norm_rope"]["k"]
+        self.thd = wl.layout == "thd"
+        if not self.thd:
+            self.q4 = q.view(B, S, wl.hq, wl.head_dim)
+            self.k4 = k.view(B, S, wl.hkv, wl.head_dim)
+            self.qo4 = self.out["qk_q"].view(B, S, wl.hq, wl.head_dim)
+            self.ko4 = self.out["qk_k"].view(B, S, wl.hkv, wl.head_dim)
+
+    def launch(self, core: str):
+        d, s, o = self.dev[core], self.host[core].scalars, self.out
+        if core == "rms_norm":
+            cores.rms_norm(d["x"], d["gain"], s["gain_offset"], s["eps"], out=o["rms_norm"])
+        elif core == "input_scale_norm":
+            cores.input_scale_norm(d["x"], d["gain"], s["gain_offset"], s["eps"], out=o["input_scale_norm"])
+        elif core == "qk_norm_rope":
+            if self.thd:
+                cores.qk_norm_rope(d["q"], d["k"], d["positions"], d["cu_seqlens"], s["eps"], 1.0, True,
+                                   True, s["rope_base"], q_out=o["qk_q"], k_out=o["qk_k"])
+            else:
+                cores.qk_norm_rope(self.q4, self.k4, d["positions"], None, s["eps"], 1.0, True, True,
+                                   s["rope_base"], q_out=self.qo4, k_out=self.ko4)
+        elif core == "output_norm_gate":
+            cores.output_norm_gate(d["o"], d["g"], None, s["eps"], out=o["output_norm_gate"])
+        elif core == "norm_residual":
+            cores.norm_residual(d["stream"], d["branch"], d["theta"], d["gain"], s["gain_offset"],
+                                False, s["norm_eps"], out=o["norm_residual"])
+
+    def input_tensors(self):
+        for c in CORE_ORDER:
+            for k, v in self.dev[c].items():
+                if v is not None:
+                    yield (c, k), v
+
+    def output_tensors(self):
+        return list(self.out.values())
+
+
+def time_copy_kernel(gib: float = 1.0, reps: int = 10) -> float:
+    n = int(gib * (1 << 30)) // 16 * 16
+    src = torch.empty(n, dtype=torch.uint8, device="cuda")
+    dst = torch.empty_like(src)
+    src.fill_(1)
+    for _ in range(3):
+        cores.stream_copy(src, dst)
+    best = math.inf
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(reps):
+        torch.cuda.synchronize()
+        e0.record()
+        cores.stream_copy(src, dst)
+        e1.record()
+        e1.synchronize()
+        best = min(best, e0.elapsed_time(e1) / 1e3)
+    del src, dst
+    torch.cuda.empty_cache()
+    return 2 * n / best / 1e9
+
+
+def traffic_from_profile(wl_name: str):
+    """dram read+write bytes per launch of the dominant kernel, from the committed
+    ncu summary, when the kernel sources are unchanged since the capture."""
+    import hashlib
+
+    p = os.path.join(ROOT, "profiles", f"{DOMINANT}__{wl_name}.md")
+    if not os.path.exists(p):
+        return None
+    fields = {}
+    for line in open(p):
+        if line.startswith("traffic_bytes_per_launch:") or line.startswith("csrc_sha256:"):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gate_cores_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    if fields.get("csrc_sha256") != h.hexdigest() or "traffic_bytes_per_launch" not in fields:
+        return None
+    return float(fields["traffic_bytes_per_launch"])
+
+
+def cpu_baseline(wl, seconds: float = 12.0, chunk: int = 256):
+    """The oracle as it stands, single-threaded, on the first tokens of the same
+    batch: all five cores per chunk of `chunk` tokens until `seconds` elapse."""
+    import numpy as np
+
+    from tests import harness
+
+    host = {c: harness.make(wl.name, c, harness.DEFAULT_VARIANT[c]) for c in CORE_ORDER}
+    T = num_tokens(wl)
+    done, t0 = 0, time.perf_counter()
+    while done < T and time.perf_counter() - t0 < seconds:
+        rows = np.arange(done, min(T, done + chunk))
+        for c in CORE_ORDER:
+            harness.run_oracle(wl.name, c, host[c], rows)
+        done += len(rows)
+    el = time.perf_counter() - t0
+    return {"value": done / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {done} of {T} tokens of {wl.name}, all five cores, "
+                      f"{el:.1f} s single-threaded double-precision oracle"}
+
+
+def run_ours(args, world, rank, local):
+    wl = WORKLOADS[args.workload]
+    torch.manual_seed(0)
+    st = Step(wl, seed=rank)
+    T = st.T
+    stream = torch.cuda.current_stream()
+    peak, peak_kind = measured_peaks()
+    copy_gbs = time_copy_kernel() if args.copy_ref else None
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    for _ in range(args.warmup):
+        for c in CORE_ORDER:
+            st.launch(c)
+    torch.cuda.synchronize()
+
+    # per-kernel events inside the timed region, on the launching stream
+    ev = {c: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)] for c in CORE_ORDER}
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        for c in CORE_ORDER:
+            ev[c][i][0].record(stream)
+            st.launch(c)
+            ev[c][i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    elapsed = t_start.elapsed_time(t_end) / 1e3
+    elapsed = allreduce_max(elapsed, world)
+    ms_per_step = elapsed / args.steps * 1e3
+    value = world * T * args.steps / elapsed
+
+    per_core = {}
+    for c in CORE_ORDER:
+        us = statistics.mean(a.elapsed_time(b) for a, b in ev[c]) * 1e3
+        us = allreduce_max(us, world)
+        nb = algo_bytes(wl, c, T)
+        per_core[c] = {"us": round(us, 3), "tokens_per_s": round(T / (us * 1e-6), 1),
+                       "gbs": round(nb / (us * 1e-6) / 1e9, 1),
+                       "frac": round(nb / (us * 1e-6) / 1e9 / peak, 4), "algo_bytes": nb,
+                       "kernel": KERNEL_NAMES[c], "variant": VARIANT[c]}
+    dom = per_core[DOMINANT]
+    traffic = traffic_from_profile(wl.name)
+    roofline = {"bound": "hbm", "achieved": dom["gbs"], "peak": peak, "unit": "GB/s",
+                "frac": round(dom["gbs"] / peak, 4), "traffic": traffic,
+                "kernel": KERNEL_NAMES[DOMINANT], "peak_source": peak_kind,
+                "algo_bytes_per_launch": dom["algo_bytes"]}
+
+    e2e = run_e2e(st, args, world) if args.e2e else None
+
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_baseline:
+        cpu = cpu_baseline(wl)
+    barrier(world)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 activations, FP32 residual stream)",
+            "config": {"workload": wl.name, "tokens_per_gpu": T, "batch": wl.batch, "seq_len": wl.seqlen,
+                       "hidden": wl.hidden, "q_heads": wl.hq, "kv_heads": wl.hkv,
+                       "head_dim": wl.head_dim, "parallelism": f"token shards x{world} (no collective)",
+                       "l2": "no flush: each step streams %.2f GB, > 126 MB L2"
+                             % (sum(algo_bytes(wl, c, T) for c in CORE_ORDER) / 1e9)},
+            "per_core": per_core,
+            "roofline": roofline,
+            "copy_kernel_gbs": None if copy_gbs is None else round(copy_gbs, 1),
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "gpu_launches": len(CORE_ORDER) * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(st: Step, args, world):
+    """Same metric through the public API with host buffers: every step copies
+    its inputs from pinned host memory, runs the five cores and reads every
+    output back to pinned host memory."""
+    pinned_in = [(dev, torch.empty(dev.shape, dtype=dev.dtype, pin_memory=True).copy_(dev.cpu()))
+                 for _, dev in st.input_tensors()]
+    pinned_out = [(dev, torch.empty(dev.shape, dtype=dev.dtype, pin_memory=True))
+                  for dev in st.output_tensors()]
+    h2d = sum(h.numel() * h.element_size() for _, h in pinned_in)
+    d2h = sum(h.numel() * h.element_size() for _, h in pinned_out)
+    steps = max(3, min(args.steps, 20))
+
+    def one():
+        for dev, h in pinned_in:
+            dev.copy_(h, non_blocking=True)
+        for c in CORE_ORDER:
+            st.launch(c)
+        for dev, h in pinned_out:
+            h.copy_(dev, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    el = allreduce_max(e0.elapsed_time(e1) / 1e3, world)
+    return {"value": round(world * st.T * steps / el, 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args, world, rank):
+    """The oracle (plain double-precision C, single-threaded) on the host cores:
+    each step is a bounded sample (64 consecutive tokens, rotating through the
+    batch) of the same workload, all five cores."""
+    if rank != 0:
+        return
+    import numpy as np
+
+    from tests import harness
+
+    wl = WORKLOADS[args.workload]
+    host = {c: harness.make(wl.name, c, harness.DEFAULT_VARIANT[c]) for c in CORE_ORDER}
+    T = num_tokens(wl)
+    per_step = 64
+
+    def step(i):
+        lo = (i * per_step) % (T - per_step + 1)
+        rows = np.arange(lo, lo + per_step)
+        for c in CORE_ORDER:
+            harness.run_oracle(wl.name, c, host[c], rows)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    el = time.perf_counter() - t0
+    value = per_step * args.steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, same generator as the GPU arm)",
+        "config": {"workload": wl.name, "tokens_per_step": per_step, "hidden": wl.hidden,
+                   "q_heads": wl.hq, "kv_heads": wl.hkv, "head_dim": wl.head_dim},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{per_step} consecutive tokens per step of {wl.name}, all five cores"},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill_t8192_h4096", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-copy-ref", dest="copy_ref", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            if not torch.cuda.is_available():
+                raise SystemExit("bench.py: no CUDA device (the cores run only on the GPU)")
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

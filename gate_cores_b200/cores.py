@@ -1,0 +1,197 @@
+"""Tensor-level front end: PyTorch CUDA tensors in, PyTorch CUDA tensors out.
+
+Marshalling only - pointers, shapes, strides and the current stream go to the
+C entry points in ``_lib``; every step of the computation runs in the CUDA
+library.  Outputs are fresh tensors unless ``out=`` is given (``out`` may be
+the input itself for an in-place call).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+
+_DT = {torch.bfloat16: _lib.MUSE_DTYPE_BF16, torch.float32: _lib.MUSE_DTYPE_F32}
+
+
+def _dtype(t: torch.Tensor) -> int:
+    try:
+        return _DT[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32") from None
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+
+
+def _rows(x: torch.Tensor):
+    """View x as rows of its last dim: (rows, hidden, row_stride); the last dim must be unit-stride."""
+    if x.dim() < 1 or x.stride(-1) != 1:
+        raise ValueError("last dimension must be contiguous")
+    hidden = x.shape[-1]
+    if x.dim() == 1:
+        return 1, hidden, hidden
+    if x.dim() == 2:
+        return x.shape[0], hidden, x.stride(0)
+    if not x.is_contiguous():
+        raise ValueError("tensors with more than 2 dims must be contiguous")
+    return x.numel() // hidden, hidden, hidden
+
+
+def _out_like(x, out):
+    if out is None:
+        return torch.empty_like(x, memory_format=torch.contiguous_format)
+    if out.shape != x.shape or out.dtype != x.dtype:
+        raise ValueError("out must match the input's shape and dtype")
+    return out
+
+
+def _gain(gain):
+    if gain is None:
+        return None
+    if gain.dtype != torch.float32:
+        raise TypeError("gain must be float32")
+    return gain.contiguous()
+
+
+def rms_norm(x: torch.Tensor, gain: torch.Tensor | None = None, gain_offset: float = 0.0,
+             eps: float = 1e-6, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Core 1 (_rms_norm_core) on the last dim of x."""
+    _cuda(x, gain, out)
+    y = _out_like(x, out)
+    rows, hidden, xs = _rows(x)
+    _, _, ys = _rows(y)
+    g = _gain(gain)
+    _lib.muse_rms_norm(x.data_ptr(), y.data_ptr(), _dtype(x), rows, hidden, xs, ys, _ptr(g),
+                       gain_offset, eps, _stream(stream))
+    return y
+
+
+def input_scale_norm(x: torch.Tensor, gain: torch.Tensor | None = None, gain_offset: float = 0.0,
+                     eps: float = 1e-6, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Core 2 (_input_scale_norm_core) on the last dim of x."""
+    _cuda(x, gain, out)
+    y = _out_like(x, out)
+    rows, hidden, xs = _rows(x)
+    _, _, ys = _rows(y)
+    g = _gain(gain)
+    _lib.muse_input_scale_norm(x.data_ptr(), y.data_ptr(), _dtype(x), rows, hidden, xs, ys,
+                               _ptr(g), gain_offset, eps, _stream(stream))
+    return y
+
+
+def _tok_stride(t: torch.Tensor, heads: int, d: int) -> int:
+    # heads and head_dim of one token must be packed: strides (.., d, 1)
+    if t.stride(-1) != 1 or t.stride(-2) != d or t.shape[-2] != heads:
+        raise ValueError("each token's heads must be contiguous ([.., heads, head_dim])")
+    if t.dim() == 4 and t.stride(0) != t.shape[1] * t.stride(1):
+        raise ValueError("BSHD tensors need a uniform token stride")
+    return t.stride(-3)
+
+
+def qk_norm_rope(q: torch.Tensor, k: torch.Tensor, positions: torch.Tensor | None = None,
+                 cu_seqlens: torch.Tensor | None = None, eps: float = 1e-6,
+                 query_scale: float = 1.0, use_rope: bool = True, upcast_rope: bool = True,
+                 rope_base: float = 10000.0, q_out: torch.Tensor | None = None,
+                 k_out: torch.Tensor | None = None, stream=None):
+    """Core 3 (_qk_norm_rope_core).  q [B,S,Hq,D] (BSHD) or [T,Hq,D] (THD with
+    cu_seqlens [docs+1] int32, or explicit positions [T]); k with Hkv heads.
+    positions: int32, [B,S] or [T]; None derives them from the layout."""
+    _cuda(q, k, positions, cu_seqlens, q_out, k_out)
+    if q.dim() == 4:
+        layout, batch, seqlen, T = _lib.MUSE_LAYOUT_BSHD, q.shape[0], q.shape[1], q.shape[0] * q.shape[1]
+    elif q.dim() == 3:
+        T = q.shape[0]
+        if cu_seqlens is not None:
+            layout, batch, seqlen = _lib.MUSE_LAYOUT_THD, 0, 0
+        else:
+            layout, batch, seqlen = _lib.MUSE_LAYOUT_BSHD, 1, T
+    else:
+        raise ValueError("q must be [B,S,Hq,D] or [T,Hq,D]")
+    hq, d = q.shape[-2], q.shape[-1]
+    hkv = k.shape[-2]
+    if k.shape[:-2] != q.shape[:-2] or k.shape[-1] != d or k.dtype != q.dtype:
+        raise ValueError("k must match q's leading dims, head_dim and dtype")
+    qo = _out_like(q, q_out)
+    ko = _out_like(k, k_out)
+    if positions is not None:
+        if positions.dtype != torch.int32 or positions.numel() != T:
+            raise ValueError("positions must be int32 with one entry per token")
+        positions = positions.contiguous()
+    num_seqs = 0
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32:
+            raise ValueError("cu_seqlens must be int32")
+        cu_seqlens = cu_seqlens.contiguous()
+        num_seqs = cu_seqlens.numel() - 1
+    _lib.muse_qk_norm_rope(
+        q.data_ptr(), k.data_ptr(), qo.data_ptr(), ko.data_ptr(), _dtype(q), layout, batch,
+        seqlen, _ptr(cu_seqlens), num_seqs, T, _ptr(positions), hq, hkv, d,
+        _tok_stride(q, hq, d), _tok_stride(k, hkv, d), _tok_stride(qo, hq, d),
+        _tok_stride(ko, hkv, d), eps, query_scale, use_rope, upcast_rope, rope_base,
+        _stream(stream))
+    return qo, ko
+
+
+def output_norm_gate(o: torch.Tensor, gate: torch.Tensor, norm_group: int | None = None,
+                     eps: float = 1e-6, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Core 4 (_output_norm_gate_core).  o, gate [B,S,H,D] or [T,H,D], contiguous.
+    norm_group None/D: per head; H*D: per token."""
+    _cuda(o, gate, out)
+    if gate.shape != o.shape or gate.dtype != o.dtype:
+        raise ValueError("gate must match o")
+    if not (o.is_contiguous() and gate.is_contiguous()):
+        raise ValueError("o and gate must be contiguous")
+    y = _out_like(o, out)
+    heads, d = o.shape[-2], o.shape[-1]
+    tokens = o.numel() // (heads * d)
+    ng = d if norm_group is None else norm_group
+    _lib.muse_output_norm_gate(o.data_ptr(), gate.data_ptr(), y.data_ptr(), _dtype(o), tokens,
+                               heads, d, ng, eps, _stream(stream))
+    return y
+
+
+def norm_residual(stream_in: torch.Tensor, branch: torch.Tensor, theta: torch.Tensor,
+                  gain: torch.Tensor | None = None, gain_offset: float = 0.0,
+                  input_scale: bool = False, norm_eps: float = 1e-6,
+                  out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Core 5 (_norm_residual_core) with the per-channel cos/sin blend.
+    stream_in FP32 [..., H]; branch [..., H] bf16/f32; theta FP32 [H]."""
+    _cuda(stream_in, branch, theta, gain, out)
+    if stream_in.dtype != torch.float32 or theta.dtype != torch.float32:
+        raise TypeError("stream and theta must be float32")
+    if branch.shape != stream_in.shape:
+        raise ValueError("branch must match the stream's shape")
+    if not (stream_in.is_contiguous() and branch.is_contiguous()):
+        raise ValueError("stream and branch must be contiguous")
+    h_out = _out_like(stream_in, out)
+    hidden = stream_in.shape[-1]
+    rows = stream_in.numel() // hidden
+    g = _gain(gain)
+    _lib.muse_norm_residual(stream_in.data_ptr(), branch.data_ptr(), h_out.data_ptr(),
+                            _dtype(branch), rows, hidden, _ptr(g), gain_offset,
+                            theta.contiguous().data_ptr(), input_scale, norm_eps, _stream(stream))
+    return h_out
+
+
+def stream_copy(src: torch.Tensor, dst: torch.Tensor, stream=None) -> torch.Tensor:
+    """16-byte vector copy of src into dst (same byte size) - the HBM reference kernel."""
+    _cuda(src, dst)
+    nbytes = src.numel() * src.element_size()
+    if dst.numel() * dst.element_size() != nbytes or not (src.is_contiguous() and dst.is_contiguous()):
+        raise ValueError("src and dst must be contiguous and of equal byte size")
+    _lib.muse_stream_copy(src.data_ptr(), dst.data_ptr(), nbytes, _stream(stream))
+    return dst

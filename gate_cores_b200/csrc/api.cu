@@ -1,0 +1,377 @@
+// C ABI of the normalisation cores: argument validation, aliasing checks,
+// launch configuration and status codes.  Everything here runs on the host;
+// no call synchronises or allocates.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include "kernels.h"
+#include "muse_cores.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+muse_status fail(muse_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+muse_status from_cuda(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return MUSE_OK;
+    return fail(MUSE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool valid_dtype(int d) { return d == MUSE_DTYPE_BF16 || d == MUSE_DTYPE_F32; }
+int64_t elem_size(int d) { return d == MUSE_DTYPE_BF16 ? 2 : 4; }
+int vec_elems(int d) { return d == MUSE_DTYPE_BF16 ? 8 : 4; }
+bool aligned(const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+bool finite(float v) { return std::isfinite(v); }
+
+// Bytes touched by a strided tensor: rows intervals [base + r*stride, + width).
+struct Span {
+    int64_t base;
+    int64_t stride;
+    int64_t width;
+    int64_t rows;
+};
+
+Span span(const void* p, int64_t rows, int64_t width_elems, int64_t stride_elems, int64_t es) {
+    return Span{(int64_t)reinterpret_cast<uintptr_t>(p), stride_elems * es, width_elems * es, rows};
+}
+
+bool same_span(const Span& a, const Span& b) {
+    return a.base == b.base && a.stride == b.stride && a.width == b.width && a.rows == b.rows;
+}
+
+int64_t floor_div(int64_t a, int64_t b) {  // b > 0
+    int64_t q = a / b;
+    if ((a % b != 0) && (a < 0)) --q;
+    return q;
+}
+
+// True when any byte of a lies in b.  Exact for equal strides (or a single
+// row on either side); conservative (bounding ranges) otherwise.
+bool overlap(Span a, Span b) {
+    if (a.rows <= 0 || b.rows <= 0 || a.width <= 0 || b.width <= 0) return false;
+    const int64_t a_end = a.base + (a.rows - 1) * a.stride + a.width;
+    const int64_t b_end = b.base + (b.rows - 1) * b.stride + b.width;
+    if (a_end <= b.base || b_end <= a.base) return false;
+    if (a.rows == 1) a.stride = b.stride;
+    if (b.rows == 1) b.stride = a.stride;
+    if (a.stride != b.stride || a.stride <= 0) return true;
+    // Rows ra of a and rb of b meet iff, with k = rb - ra and d = b.base - a.base,
+    // -b.width < d + k * stride < a.width.
+    const int64_t S = a.stride, d = b.base - a.base;
+    int64_t kmin = floor_div(-b.width - d, S) + 1;
+    int64_t kmax = -floor_div(-(a.width - d), S) - 1;  // ceil((a.width - d) / S) - 1
+    if (kmin < -(a.rows - 1)) kmin = -(a.rows - 1);
+    if (kmax > b.rows - 1) kmax = b.rows - 1;
+    return kmin <= kmax;
+}
+
+// An output may coincide exactly with one input; any other overlap with any
+// tensor of the call is an error.
+bool bad_alias(const Span& out, const Span& other, bool may_coincide) {
+    if (may_coincide && same_span(out, other)) return false;
+    return overlap(out, other);
+}
+
+muse_status row_entry(muse::RowOp op, const void* x, void* y, muse_dtype dtype, int64_t rows,
+                      int64_t hidden, int64_t xs, int64_t ys, const float* gain,
+                      float gain_offset, float eps, cudaStream_t stream, const char* name) {
+    if (!valid_dtype(dtype)) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, (int)dtype);
+    if (rows < 0 || hidden <= 0)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: rows=%lld hidden=%lld", name, (long long)rows, (long long)hidden);
+    if (!finite(eps) || eps < 0.0f || !finite(gain_offset))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: eps must be finite and >= 0, gain_offset finite", name);
+    if (xs < hidden || ys < hidden)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: row strides must be >= hidden", name);
+    if (rows == 0) return MUSE_OK;
+    if (!x || !y) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null x or y", name);
+    const int64_t es = elem_size(dtype);
+    if (!aligned(x, 16) || !aligned(y, 16) || (hidden * es) % 16 || (xs * es) % 16 || (ys * es) % 16)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: pointers, row widths and strides must be 16-byte multiples", name);
+    if (gain && !aligned(gain, 16)) return fail(MUSE_ERR_UNSUPPORTED, "%s: gain not 16-byte aligned", name);
+    if (hidden * es > MUSE_MAX_ROW_BYTES)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: row of %lld bytes exceeds %d", name, (long long)(hidden * es), MUSE_MAX_ROW_BYTES);
+    const Span sx = span(x, rows, hidden, xs, es), sy = span(y, rows, hidden, ys, es);
+    if (bad_alias(sy, sx, true) || (gain && bad_alias(sy, span(gain, 1, hidden, hidden, 4), false)))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: output partially overlaps an input", name);
+    muse::RowArgs a{};
+    a.x = x;
+    a.y = y;
+    a.gain = gain;
+    a.rows = rows;
+    a.x_stride = xs;
+    a.y_stride = ys;
+    a.width = (int32_t)hidden;
+    a.gain_offset = gain_offset;
+    a.eps = eps;
+    return from_cuda(muse::launch_row(dtype, op, a, stream), name);
+}
+
+}  // namespace
+
+namespace muse {
+
+int sm_count() {
+    static std::mutex mu;
+    static std::map<int, int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(dev);
+    if (it != cache.end()) return it->second;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+    return n;
+}
+
+int blocks_per_sm(const void* kernel, int threads) {
+    static std::mutex mu;
+    static std::map<std::tuple<const void*, int, int>, int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+    const auto key = std::make_tuple(kernel, threads, dev);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = cache.find(key);
+        if (it != cache.end()) return it->second;
+    }
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n < 1) n = 1;
+    std::lock_guard<std::mutex> lock(mu);
+    cache[key] = n;
+    return n;
+}
+
+}  // namespace muse
+
+extern "C" {
+
+int muse_version(void) { return MUSE_VERSION; }
+
+const char* muse_status_string(muse_status s) {
+    switch (s) {
+        case MUSE_OK: return "MUSE_OK";
+        case MUSE_ERR_INVALID_ARGUMENT: return "MUSE_ERR_INVALID_ARGUMENT";
+        case MUSE_ERR_UNSUPPORTED: return "MUSE_ERR_UNSUPPORTED";
+        case MUSE_ERR_CUDA: return "MUSE_ERR_CUDA";
+    }
+    return "MUSE_ERR_UNKNOWN";
+}
+
+const char* muse_last_error(void) { return g_err; }
+
+muse_status muse_rms_norm(const void* x, void* y, muse_dtype dtype, int64_t rows, int64_t hidden,
+                          int64_t x_row_stride, int64_t y_row_stride, const float* gain,
+                          float gain_offset, float eps, cudaStream_t stream) {
+    return row_entry(muse::RowOp::kRms, x, y, dtype, rows, hidden, x_row_stride, y_row_stride,
+                     gain, gain_offset, eps, stream, "muse_rms_norm");
+}
+
+muse_status muse_input_scale_norm(const void* x, void* y, muse_dtype dtype, int64_t rows,
+                                  int64_t hidden, int64_t x_row_stride, int64_t y_row_stride,
+                                  const float* gain, float gain_offset, float eps,
+                                  cudaStream_t stream) {
+    return row_entry(muse::RowOp::kInputScale, x, y, dtype, rows, hidden, x_row_stride,
+                     y_row_stride, gain, gain_offset, eps, stream, "muse_input_scale_norm");
+}
+
+muse_status muse_qk_norm_rope(const void* q, const void* k, void* q_out, void* k_out,
+                              muse_dtype dtype, muse_layout layout, int64_t batch,
+                              int64_t seqlen, const int32_t* cu_seqlens, int32_t num_seqs,
+                              int64_t total_tokens, const int32_t* positions, int32_t hq,
+                              int32_t hkv, int32_t head_dim, int64_t q_tok_stride,
+                              int64_t k_tok_stride, int64_t q_out_tok_stride,
+                              int64_t k_out_tok_stride, float eps, float query_scale,
+                              int use_rope, int upcast_rope, float rope_base,
+                              cudaStream_t stream) {
+    const char* name = "muse_qk_norm_rope";
+    if (!valid_dtype(dtype)) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, (int)dtype);
+    if (layout != MUSE_LAYOUT_BSHD && layout != MUSE_LAYOUT_THD)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown layout %d", name, (int)layout);
+    int64_t tokens = 0;
+    if (layout == MUSE_LAYOUT_BSHD) {
+        if (batch < 0 || seqlen < 0 || (batch > 0 && seqlen == 0))
+            return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: batch=%lld seqlen=%lld", name, (long long)batch, (long long)seqlen);
+        tokens = batch * seqlen;
+    } else {
+        if (total_tokens < 0 || num_seqs < 0)
+            return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: total_tokens=%lld num_seqs=%d", name, (long long)total_tokens, num_seqs);
+        tokens = total_tokens;
+    }
+    if (hq <= 0 || hkv <= 0 || hq % hkv != 0)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: hq=%d must be a positive multiple of hkv=%d", name, hq, hkv);
+    if (head_dim <= 0 || (head_dim & 1))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: head_dim=%d must be positive and even", name, head_dim);
+    if (!finite(eps) || eps < 0.0f || !finite(query_scale))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: eps must be finite and >= 0, query_scale finite", name);
+    if (use_rope && !(finite(rope_base) && rope_base > 0.0f))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: rope_base must be finite and > 0", name);
+    const int64_t qw = (int64_t)hq * head_dim, kw = (int64_t)hkv * head_dim;
+    if (q_tok_stride < qw || q_out_tok_stride < qw || k_tok_stride < kw || k_out_tok_stride < kw)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: token strides must cover all heads", name);
+    const bool derive = use_rope && !positions;
+    if (tokens > 0 && derive && layout == MUSE_LAYOUT_THD && (!cu_seqlens || num_seqs < 1))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: THD without positions needs cu_seqlens and num_seqs >= 1", name);
+    if (tokens == 0) return MUSE_OK;
+    if (!q || !k || !q_out || !k_out) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null q/k/q_out/k_out", name);
+    const int64_t es = elem_size(dtype);
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(q_out, 16) || !aligned(k_out, 16) ||
+        (head_dim * es) % 16 || (q_tok_stride * es) % 16 || (k_tok_stride * es) % 16 ||
+        (q_out_tok_stride * es) % 16 || (k_out_tok_stride * es) % 16)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: pointers, head_dim and strides must be 16-byte multiples", name);
+    if (head_dim / vec_elems(dtype) > 32 || head_dim / 2 > muse::kMaxHalfDim)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: head_dim=%d exceeds 512 bytes per head", name, head_dim);
+    if ((positions && !aligned(positions, 4)) || (cu_seqlens && !aligned(cu_seqlens, 4)))
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: positions / cu_seqlens not 4-byte aligned", name);
+    const Span sq = span(q, tokens, qw, q_tok_stride, es), sk = span(k, tokens, kw, k_tok_stride, es);
+    const Span sqo = span(q_out, tokens, qw, q_out_tok_stride, es);
+    const Span sko = span(k_out, tokens, kw, k_out_tok_stride, es);
+    bool bad = bad_alias(sqo, sq, true) || bad_alias(sqo, sk, false) || bad_alias(sqo, sko, false) ||
+               bad_alias(sko, sk, true) || bad_alias(sko, sq, false);
+    if (use_rope && positions) {
+        const Span sp = span(positions, 1, tokens, tokens, 4);
+        bad = bad || bad_alias(sqo, sp, false) || bad_alias(sko, sp, false);
+    }
+    if (derive && layout == MUSE_LAYOUT_THD) {
+        const Span sc = span(cu_seqlens, 1, (int64_t)num_seqs + 1, (int64_t)num_seqs + 1, 4);
+        bad = bad || bad_alias(sqo, sc, false) || bad_alias(sko, sc, false);
+    }
+    if (bad) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: output partially overlaps an input", name);
+
+    muse::QkArgs a{};
+    a.q = q;
+    a.k = k;
+    a.q_out = q_out;
+    a.k_out = k_out;
+    a.positions = positions;
+    a.cu_seqlens = cu_seqlens;
+    a.tokens = tokens;
+    a.seqlen = layout == MUSE_LAYOUT_BSHD ? seqlen : 1;
+    a.q_stride = q_tok_stride;
+    a.k_stride = k_tok_stride;
+    a.q_out_stride = q_out_tok_stride;
+    a.k_out_stride = k_out_tok_stride;
+    a.num_seqs = num_seqs;
+    a.hq = hq;
+    a.hkv = hkv;
+    a.head_dim = head_dim;
+    a.tile_tokens = 1;
+    a.pos_mode = positions ? 0 : (layout == MUSE_LAYOUT_BSHD ? 1 : 2);
+    a.eps = eps;
+    a.query_scale = query_scale;
+    // FP32 rotary frequencies: base^(-2i/D) evaluated in double, rounded once.
+    if (use_rope)
+        for (int i = 0; i < head_dim / 2; ++i)
+            a.inv_freq[i] = (float)std::pow((double)rope_base, -(2.0 * i) / (double)head_dim);
+    return from_cuda(muse::launch_qk(dtype, use_rope, upcast_rope, a, stream), name);
+}
+
+muse_status muse_output_norm_gate(const void* o, const void* gate, void* y, muse_dtype dtype,
+                                  int64_t tokens, int32_t heads, int32_t head_dim,
+                                  int32_t norm_group, float eps, cudaStream_t stream) {
+    const char* name = "muse_output_norm_gate";
+    if (!valid_dtype(dtype)) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, (int)dtype);
+    if (tokens < 0 || heads <= 0 || head_dim <= 0)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: tokens=%lld heads=%d head_dim=%d", name, (long long)tokens, heads, head_dim);
+    const int64_t width = (int64_t)heads * head_dim;
+    if (norm_group != head_dim && norm_group != width)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: norm_group=%d must be head_dim or heads*head_dim", name, norm_group);
+    if (!finite(eps) || eps < 0.0f) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: eps must be finite and >= 0", name);
+    if (tokens == 0) return MUSE_OK;
+    if (!o || !gate || !y) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null o/gate/y", name);
+    const int64_t es = elem_size(dtype);
+    if (!aligned(o, 16) || !aligned(gate, 16) || !aligned(y, 16) || (head_dim * es) % 16)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: pointers and head_dim must be 16-byte multiples", name);
+    const bool per_head = norm_group == head_dim && head_dim / vec_elems(dtype) <= 32;
+    if (!per_head && norm_group * es > MUSE_MAX_ROW_BYTES)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: norm group of %lld bytes exceeds %d", name, (long long)(norm_group * es), MUSE_MAX_ROW_BYTES);
+    const Span so = span(o, tokens, width, width, es), sg = span(gate, tokens, width, width, es);
+    const Span sy = span(y, tokens, width, width, es);
+    if (bad_alias(sy, so, true) || bad_alias(sy, sg, true))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: output partially overlaps an input", name);
+    if (per_head) {
+        muse::HeadGateArgs a{};
+        a.o = o;
+        a.gate = gate;
+        a.y = y;
+        a.rows = tokens * heads;
+        a.width = head_dim;
+        a.eps = eps;
+        return from_cuda(muse::launch_head_gate(dtype, a, stream), name);
+    }
+    muse::RowArgs a{};
+    a.x = o;
+    a.gate = gate;
+    a.y = y;
+    a.rows = tokens * (width / norm_group);
+    a.x_stride = a.y_stride = a.gate_stride = norm_group;
+    a.width = norm_group;
+    a.eps = eps;
+    return from_cuda(muse::launch_row(dtype, muse::RowOp::kNormGate, a, stream), name);
+}
+
+muse_status muse_norm_residual(const float* stream_in, const void* branch, float* stream_out,
+                               muse_dtype branch_dtype, int64_t rows, int64_t hidden,
+                               const float* gain, float gain_offset, const float* theta,
+                               int input_scale, float norm_eps, cudaStream_t stream) {
+    const char* name = "muse_norm_residual";
+    if (!valid_dtype(branch_dtype)) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, (int)branch_dtype);
+    if (rows < 0 || hidden <= 0)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: rows=%lld hidden=%lld", name, (long long)rows, (long long)hidden);
+    if (!finite(norm_eps) || norm_eps < 0.0f || !finite(gain_offset))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: norm_eps must be finite and >= 0, gain_offset finite", name);
+    if (rows == 0) return MUSE_OK;
+    if (!stream_in || !branch || !stream_out || !theta)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null stream_in/branch/stream_out/theta", name);
+    const int64_t es = elem_size(branch_dtype);
+    if (!aligned(stream_in, 16) || !aligned(stream_out, 16) || !aligned(branch, 16) || (hidden * es) % 16)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: pointers and row widths must be 16-byte multiples", name);
+    if (!aligned(theta, 16) || (gain && !aligned(gain, 16)))
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: theta / gain not 16-byte aligned", name);
+    if (hidden * es > MUSE_MAX_ROW_BYTES)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: branch row of %lld bytes exceeds %d", name, (long long)(hidden * es), MUSE_MAX_ROW_BYTES);
+    const Span sin_ = span(stream_in, rows, hidden, hidden, 4), sout = span(stream_out, rows, hidden, hidden, 4);
+    const Span sb = span(branch, rows, hidden, hidden, es), st = span(theta, 1, hidden, hidden, 4);
+    bool bad = bad_alias(sout, sin_, true) || bad_alias(sout, sb, false) || bad_alias(sout, st, false);
+    if (gain) bad = bad || bad_alias(sout, span(gain, 1, hidden, hidden, 4), false);
+    if (bad) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: output partially overlaps an input", name);
+    muse::RowArgs a{};
+    a.x = branch;
+    a.stream_in = stream_in;
+    a.stream_out = stream_out;
+    a.gain = gain;
+    a.theta = theta;
+    a.rows = rows;
+    a.x_stride = hidden;
+    a.s_in_stride = a.s_out_stride = hidden;
+    a.width = (int32_t)hidden;
+    a.gain_offset = gain_offset;
+    a.eps = norm_eps;
+    const muse::RowOp op = input_scale ? muse::RowOp::kResidualIS : muse::RowOp::kResidual;
+    return from_cuda(muse::launch_row(branch_dtype, op, a, stream), name);
+}
+
+muse_status muse_stream_copy(const void* src, void* dst, int64_t bytes, cudaStream_t stream) {
+    const char* name = "muse_stream_copy";
+    if (bytes < 0) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: bytes=%lld", name, (long long)bytes);
+    if (bytes == 0) return MUSE_OK;
+    if (!src || !dst) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null pointer", name);
+    if (bytes % 16 || !aligned(src, 16) || !aligned(dst, 16))
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: pointers and size must be 16-byte multiples", name);
+    if (overlap(span(src, 1, bytes, bytes, 1), span(dst, 1, bytes, bytes, 1)))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: ranges overlap", name);
+    return from_cuda(muse::launch_copy(src, dst, bytes, stream), name);
+}
+
+}  // extern "C"

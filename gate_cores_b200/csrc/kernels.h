@@ -1,0 +1,77 @@
+// Internal launch interface between the C ABI (api.cu) and the kernel files.
+// Host-side only; arguments arrive here already validated.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace muse {
+
+enum class RowOp : int {
+    kRms = 0,          // core 1: y = cast((x r) w)
+    kInputScale = 1,   // core 2: z = x w, y = cast(z r(z))
+    kNormGate = 2,     // core 4, one norm per token row: y = cast(o r sigmoid(g))
+    kResidual = 3,     // core 5, gain after the norm
+    kResidualIS = 4,   // core 5, gain before the norm
+};
+
+// One row = one token's `width` elements.  Strides in elements.
+struct RowArgs {
+    const void* x;          // x (cores 1, 2), o (core 4), branch (core 5)
+    void* y;                // output rows (cores 1, 2, 4)
+    const void* gate;       // core 4
+    const float* stream_in; // core 5
+    float* stream_out;      // core 5
+    const float* gain;      // may be null
+    const float* theta;     // core 5
+    int64_t rows;
+    int64_t x_stride, y_stride, gate_stride, s_in_stride, s_out_stride;
+    int32_t width;
+    int32_t rows_per_cta;   // set by the launcher
+    float gain_offset;
+    float eps;
+};
+
+// Many short rows (one attention head each), contiguous: core 4 per head.
+struct HeadGateArgs {
+    const void* o;
+    const void* gate;
+    void* y;
+    int64_t rows;     // tokens * heads
+    int32_t width;    // head_dim
+    float eps;
+};
+
+constexpr int kMaxHalfDim = 128;  // head_dim <= 256
+constexpr int kMaxTileTokens = 16;  // 2 x 2 x 16 x 128 floats = 32 KB of cos/sin table
+
+struct QkArgs {
+    const void* q;
+    const void* k;
+    void* q_out;
+    void* k_out;
+    const int32_t* positions;   // explicit positions or null
+    const int32_t* cu_seqlens;  // THD document boundaries (positions == null)
+    int64_t tokens;
+    int64_t seqlen;             // BSHD: positions derive as t mod seqlen
+    int64_t q_stride, k_stride, q_out_stride, k_out_stride;  // elements per token
+    int32_t num_seqs;
+    int32_t hq, hkv, head_dim;
+    int32_t tile_tokens;        // tokens per CTA tile (<= kMaxTileTokens)
+    int32_t pos_mode;           // 0 explicit, 1 BSHD derived, 2 THD derived
+    float eps;
+    float query_scale;
+    float inv_freq[kMaxHalfDim];
+};
+
+// Returns cudaSuccess or the launch error.
+cudaError_t launch_row(int dtype, RowOp op, const RowArgs& a, cudaStream_t s);
+cudaError_t launch_head_gate(int dtype, const HeadGateArgs& a, cudaStream_t s);
+cudaError_t launch_qk(int dtype, int use_rope, int upcast_rope, const QkArgs& a, cudaStream_t s);
+cudaError_t launch_copy(const void* src, void* dst, int64_t bytes, cudaStream_t s);
+
+// Device facts for grid sizing (cached per device).
+int sm_count();
+int blocks_per_sm(const void* kernel, int threads);
+
+}  // namespace muse

@@ -1,0 +1,174 @@
+/*
+ * muse_cores.h - C ABI of the B200 (sm_100a) fused per-token normalisation
+ * cores of the Muse Spark Open decoder layer.
+ *
+ * The five cores restate the pure functions documented on the NeMo AutoModel
+ * API reference page "nemo_automodel.components.models.muse_spark.layers":
+ * _rms_norm_core, _input_scale_norm_core, _qk_norm_rope_core,
+ * _output_norm_gate_core and _norm_residual_core.  Each entry point launches
+ * one CUDA kernel that makes one pass over HBM.
+ *
+ * Common contract
+ *   - Every pointer to tensor data is a DEVICE pointer owned by the caller;
+ *     the library allocates no memory and keeps no per-call state.  The
+ *     only process-wide state is a cache of SM counts and occupancy figures.
+ *   - Every call is asynchronous on `stream` (NULL = the legacy default
+ *     stream of the current device) and never synchronises.  Results are
+ *     valid once work queued on `stream` after the call has completed.
+ *   - Tensors are row-major.  A "row stride" counts ELEMENTS between the
+ *     first elements of consecutive rows (tokens) and must be >= the row width.
+ *   - dtype is the activation dtype; every output keeps the dtype of the
+ *     tensor it replaces (the residual stream stays FP32).  Gains
+ *     and blend angles are FP32; every reduction and every product runs in
+ *     FP32.
+ *   - Aliasing: an output may be the very same memory as its input (same
+ *     pointer, same stride: in-place); any other overlap between an output and
+ *     any tensor of the call returns MUSE_ERR_INVALID_ARGUMENT.
+ *   - rows/tokens == 0 returns MUSE_OK without a launch.
+ *   - Limits (MUSE_ERR_UNSUPPORTED): every tensor pointer (gains and blend
+ *     angles included) and every row stride in bytes must be a multiple of
+ *     16 bytes, and every row width (and head_dim) a multiple of 8 elements
+ *     for bf16 or 4 for f32 (16 bytes).  positions and cu_seqlens need 4-byte
+ *     alignment.  Row widths up to MUSE_MAX_ROW_BYTES bytes; head_dim up to
+ *     512 bytes (256 bf16 or 128 f32 elements).
+ *   - Errors: a status is returned before anything is launched when an
+ *     argument is invalid; MUSE_ERR_CUDA reports a failed launch (the CUDA
+ *     error is cleared).  muse_last_error() gives a one-line description of
+ *     the last failing call on the calling thread.
+ */
+#ifndef MUSE_CORES_H
+#define MUSE_CORES_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MUSE_VERSION 1
+/* Widest row a single CTA normalises: 32768 bf16 or 16384 f32 elements. */
+#define MUSE_MAX_ROW_BYTES 65536
+
+typedef enum muse_status {
+    MUSE_OK = 0,
+    MUSE_ERR_INVALID_ARGUMENT = 1,
+    MUSE_ERR_UNSUPPORTED = 2,
+    MUSE_ERR_CUDA = 3
+} muse_status;
+
+typedef enum muse_dtype { MUSE_DTYPE_BF16 = 0, MUSE_DTYPE_F32 = 1 } muse_dtype;
+
+typedef enum muse_layout { MUSE_LAYOUT_BSHD = 0, MUSE_LAYOUT_THD = 1 } muse_layout;
+
+int muse_version(void);
+const char* muse_status_string(muse_status s);
+/* Description of the last non-OK status returned on this thread ("" if none). */
+const char* muse_last_error(void);
+
+/*
+ * Core 1 - _rms_norm_core (FP32 normalisation, then the effective gain, then
+ * the single cast to the output dtype; MuseSparkRMSNorm, zero-centered gain).
+ *   y[r, j] = cast( (x[r, j] * inv_rms(x[r, :])) * w_eff[j] ),
+ *   inv_rms(v) = 1 / sqrt(mean_j(v_j^2) + eps),
+ *   w_eff[j] = f32(gain[j] + gain_offset)   (gain_offset 1.0 for the
+ *   zero-centered checkpoint gain, 0 otherwise); gain == NULL: no multiply.
+ * x [rows, hidden] with row stride x_row_stride, y [rows, hidden] with row
+ * stride y_row_stride, both `dtype`; gain [hidden] FP32 or NULL.
+ */
+muse_status muse_rms_norm(const void* x, void* y, muse_dtype dtype, int64_t rows,
+                          int64_t hidden, int64_t x_row_stride, int64_t y_row_stride,
+                          const float* gain, float gain_offset, float eps,
+                          cudaStream_t stream);
+
+/*
+ * Core 2 - _input_scale_norm_core (the effective gain scales the row first;
+ * the FP32 norm and its eps then act on the SCALED activation).
+ *   z[r, j] = x[r, j] * w_eff[j]  (FP32),  y[r, j] = cast( z[r, j] * inv_rms(z[r, :]) ).
+ * Arguments as muse_rms_norm.
+ */
+muse_status muse_input_scale_norm(const void* x, void* y, muse_dtype dtype, int64_t rows,
+                                  int64_t hidden, int64_t x_row_stride, int64_t y_row_stride,
+                                  const float* gain, float gain_offset, float eps,
+                                  cudaStream_t stream);
+
+/*
+ * Core 3 - _qk_norm_rope_core (per-head Q/K normalisation and rotation that
+ * keeps every cast of the checkpoint in place), with the rotary frequencies of
+ * MuseSparkRotaryEmbedding and the adjacent-pair rotation of
+ * apply_rotary_embedding computed in the kernel from positions.
+ * Per token t and per head (hq query heads, hkv key heads), over head_dim D:
+ *   n = cast( x * inv_rms(x) );  query heads only: n = cast( n * query_scale );
+ *   use_rope: for pair i = 0 .. D/2-1 with (a, b) = (n[2i], n[2i+1]),
+ *     phi = f32( f32(pos_t) * inv_freq[i] ),  inv_freq[i] = f32(rope_base^(-2i/D));
+ *     upcast_rope != 0 (original checkpoint, FP32 rotation):
+ *       y[2i] = cast(a cos(phi) - b sin(phi)), y[2i+1] = cast(a sin(phi) + b cos(phi));
+ *     upcast_rope == 0 (HF release, rotation in the Q/K dtype):
+ *       c = cast(cos phi), s = cast(sin phi),
+ *       y[2i] = cast(cast(a c) - cast(b s)), y[2i+1] = cast(cast(a s) + cast(b c)).
+ * q [T, hq, D] with token stride q_tok_stride, k [T, hkv, D] with
+ * k_tok_stride (views into a fused QKV projection are fine); outputs with
+ * their own token strides; heads of one token are contiguous.
+ * Tokens: BSHD: T = batch * seqlen; THD: T = total_tokens.
+ * positions: int32 [T] device array, or NULL to derive them:
+ *   BSHD: pos_t = t mod seqlen;  THD: pos_t = t - cu_seqlens[d] for the
+ *   document d with cu_seqlens[d] <= t < cu_seqlens[d+1].
+ * cu_seqlens: int32 [num_seqs+1] device array (THD with positions == NULL
+ * only; otherwise ignored).  It must start at 0, not decrease and end at
+ * total_tokens; the library cannot check device contents without a
+ * synchronisation, so other contents give unspecified positions (never an
+ * out-of-bounds access).  Under context parallelism pass positions.
+ * Requires hq % hkv == 0 (GQA), D even, D <= 256.
+ */
+muse_status muse_qk_norm_rope(const void* q, const void* k, void* q_out, void* k_out,
+                              muse_dtype dtype, muse_layout layout, int64_t batch,
+                              int64_t seqlen, const int32_t* cu_seqlens, int32_t num_seqs,
+                              int64_t total_tokens, const int32_t* positions, int32_t hq,
+                              int32_t hkv, int32_t head_dim, int64_t q_tok_stride,
+                              int64_t k_tok_stride, int64_t q_out_tok_stride,
+                              int64_t k_out_tok_stride, float eps, float query_scale,
+                              int use_rope, int upcast_rope, float rope_base,
+                              cudaStream_t stream);
+
+/*
+ * Core 4 - _output_norm_gate_core (norm without gain of the attention output,
+ * times the sigmoid of the gate projection; both in FP32, one cast).
+ *   y = cast( o * inv_rms(o over its group) * sigmoid(g) ),  sigmoid(g) = 1/(1+exp(-g)).
+ * o, gate, y: [tokens, heads, head_dim] contiguous, `dtype`.
+ * norm_group = head_dim: one norm per head (the head-split layout the page
+ * passes); norm_group = heads*head_dim: one norm per token.
+ */
+muse_status muse_output_norm_gate(const void* o, const void* gate, void* y, muse_dtype dtype,
+                                  int64_t tokens, int32_t heads, int32_t head_dim,
+                                  int32_t norm_group, float eps, cudaStream_t stream);
+
+/*
+ * Core 5 - _norm_residual_core (branch norm, cast back to the branch dtype,
+ * then blended into the FP32 stream) with the learned blend of
+ * MuseSparkResidual read as a per-channel rotation by theta:
+ *   nb[r, j] = cast_branch( normed(branch[r, :])[j] ),  normed = core 1's form
+ *     (input_scale == 0: gain after the norm) or core 2's form (input_scale != 0),
+ *     with w_eff = f32(gain + gain_offset) (gain may be NULL) and norm_eps;
+ *   stream_out[r, j] = cos(theta[j]) * stream_in[r, j] + sin(theta[j]) * nb[r, j]   (FP32).
+ * stream_in, stream_out: FP32 [rows, hidden] contiguous (stream_out ==
+ * stream_in is allowed); branch: [rows, hidden] contiguous, branch_dtype;
+ * gain, theta: FP32 [hidden].
+ */
+muse_status muse_norm_residual(const float* stream_in, const void* branch, float* stream_out,
+                               muse_dtype branch_dtype, int64_t rows, int64_t hidden,
+                               const float* gain, float gain_offset, const float* theta,
+                               int input_scale, float norm_eps, cudaStream_t stream);
+
+/*
+ * Bandwidth reference (not a core): copy `bytes` bytes from src to dst with
+ * 16-byte vector loads and stores over a persistent grid.  It measures the
+ * HBM roofline on the same device the cores run on.  bytes % 16 == 0; both
+ * pointers 16-byte aligned; the ranges must not overlap.
+ */
+muse_status muse_stream_copy(const void* src, void* dst, int64_t bytes, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUSE_CORES_H */

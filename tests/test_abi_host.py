@@ -1,0 +1,139 @@
+"""Host-side checks of the C ABI library, no GPU needed: the library loads,
+exports every entry point include/muse_cores.h declares, and rejects invalid
+arguments before anything is launched.  The pointers below are never
+dereferenced: each call fails validation on the host first."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gate_cores_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "muse_cores.h")
+INV, UNS = _lib.MUSE_ERR_INVALID_ARGUMENT, _lib.MUSE_ERR_UNSUPPORTED
+BF16, F32 = _lib.MUSE_DTYPE_BF16, _lib.MUSE_DTYPE_F32
+A = 0x7F0000000000  # a 256-byte aligned fake device address (never touched)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(muse_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(names) == set(_lib.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+        assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
+
+
+def test_version_and_status_strings(lib):
+    assert _lib.muse_version() == 1
+    assert _lib.muse_status_string(0) == "MUSE_OK"
+    assert _lib.muse_status_string(2) == "MUSE_ERR_UNSUPPORTED"
+
+
+def rms(lib, x=A, y=A + (1 << 24), dt=BF16, rows=4, hidden=256, xs=None, ys=None, gain=None,
+        off=0.0, eps=1e-6):
+    xs = hidden if xs is None else xs
+    ys = hidden if ys is None else ys
+    return lib.muse_rms_norm(x, y, dt, rows, hidden, xs, ys, gain, off, eps, None)
+
+
+def test_row_validation(lib):
+    assert rms(lib, rows=0) == 0  # empty: OK without a launch
+    assert rms(lib, dt=7) == INV
+    assert rms(lib, rows=-1) == INV
+    assert rms(lib, hidden=0) == INV
+    assert rms(lib, x=None) == INV
+    assert rms(lib, xs=100) == INV                      # stride < hidden
+    assert rms(lib, eps=float("nan")) == INV
+    assert rms(lib, eps=-1.0) == INV
+    assert rms(lib, x=A + 8) == UNS                     # misaligned pointer
+    assert rms(lib, hidden=260) == UNS                  # not a 16-byte row
+    assert rms(lib, hidden=256, xs=260) == UNS          # stride not 16-byte
+    assert rms(lib, hidden=65536) == UNS                # wider than one CTA row
+    assert rms(lib, gain=A + 2) == UNS
+    assert rms(lib, gain=A + 8) == UNS                  # gains load as 16-byte vectors
+    assert b"muse_rms_norm" in lib.muse_last_error()
+
+
+def test_row_partial_overlap_rejected(lib):
+    # y starts half a row into x: overlapping but not the same tensor
+    assert rms(lib, x=A, y=A + 256) == INV
+    # y overlaps the gain vector
+    assert rms(lib, x=A, y=A + (1 << 20), gain=A + (1 << 20) + 64) == INV
+    # input-scale variant shares the checks
+    assert lib.muse_input_scale_norm(A, A + 256, BF16, 4, 256, 256, 256, None, 0.0, 1e-6, None) == INV
+
+
+def qk(lib, q=A, k=A + (1 << 26), qo=A + (2 << 26), ko=A + (3 << 26), dt=BF16, layout=0, batch=2,
+       seqlen=8, cu=None, ns=0, total=0, pos=None, hq=4, hkv=2, d=64, qs=None, ks=None, qos=None,
+       kos=None, eps=1e-6, scale=1.0, rope=1, upcast=1, base=1e4):
+    qs = hq * d if qs is None else qs
+    ks = hkv * d if ks is None else ks
+    qos = hq * d if qos is None else qos
+    kos = hkv * d if kos is None else kos
+    return lib.muse_qk_norm_rope(q, k, qo, ko, dt, layout, batch, seqlen, cu, ns, total, pos, hq,
+                                 hkv, d, qs, ks, qos, kos, eps, scale, rope, upcast, base, None)
+
+
+def test_qk_validation(lib):
+    assert qk(lib, batch=0) == 0
+    assert qk(lib, layout=5) == INV
+    assert qk(lib, hq=6, hkv=4) == INV                  # GQA needs hq % hkv == 0
+    assert qk(lib, d=63) == INV                         # odd head_dim
+    assert qk(lib, base=0.0) == INV
+    assert qk(lib, base=float("inf")) == INV
+    assert qk(lib, qs=100) == INV                       # stride below the heads' width
+    assert qk(lib, layout=1, total=16, cu=None) == INV  # THD with derived positions needs cu_seqlens
+    assert qk(lib, layout=1, total=16, cu=A + (5 << 26), ns=0) == INV
+    assert qk(lib, layout=1, total=-1) == INV
+    assert qk(lib, d=36) == UNS                         # 72-byte heads: not 16-byte multiples
+    assert qk(lib, d=512) == UNS                        # above 512 bytes per head
+    assert qk(lib, dt=F32, d=256) == UNS
+    assert qk(lib, q=A + 4) == UNS
+    assert qk(lib, pos=A + (5 << 26) + 2) == UNS
+
+
+def test_qk_aliasing_rules(lib):
+    # q_out half a head into q: partial overlap
+    assert qk(lib, qo=A + 64) == INV
+    # k_out overlapping q
+    assert qk(lib, ko=A + 128) == INV
+    # outputs overlapping the positions array
+    assert qk(lib, pos=A + (2 << 26) + 64) == INV
+    # fused QKV with q_out and k_out landing on each other's columns
+    W = (4 + 2 * 2) * 64
+    assert qk(lib, q=A, k=A + 4 * 64 * 2, qo=A + 4 * 64 * 2, ko=A, qs=W, ks=W, qos=W, kos=W) == INV
+
+
+def test_gate_and_residual_validation(lib):
+    g = lib.muse_output_norm_gate
+    assert g(A, A + (1 << 24), A + (2 << 24), BF16, 4, 4, 64, 32, 1e-6, None) == INV  # norm_group
+    assert g(A, A + (1 << 24), A + (2 << 24), BF16, 0, 4, 64, 64, 1e-6, None) == 0
+    assert g(A, A + (1 << 24), A + 64, BF16, 4, 4, 64, 64, 1e-6, None) == INV
+    assert g(A, A + (1 << 24), A + (2 << 24), BF16, 4, 4, 60, 60, 1e-6, None) == UNS
+    r = lib.muse_norm_residual
+    assert r(A, A + (1 << 24), A + (2 << 24), BF16, 0, 256, None, 0.0, A + (3 << 24), 0, 1e-6, None) == 0
+    assert r(A, A + (1 << 24), A + (2 << 24), BF16, 4, 256, None, 0.0, None, 0, 1e-6, None) == INV
+    assert r(A, A + (1 << 24), A + 512, BF16, 4, 256, None, 0.0, A + (3 << 24), 0, 1e-6, None) == INV
+    # stream_out overlapping the branch
+    assert r(A, A + (1 << 24), A + (1 << 24) + 1024, BF16, 4, 256, None, 0.0, A + (3 << 24), 0,
+             1e-6, None) == INV
+    assert r(A, A + (1 << 24), A + (2 << 24), BF16, 4, 252, None, 0.0, A + (3 << 24), 0, 1e-6,
+             None) == UNS
+    c = lib.muse_stream_copy
+    assert c(A, A + 4096, 0, None) == 0
+    assert c(A, A + 4096, 8192, None) == INV            # overlapping ranges
+    assert c(A, A + (1 << 20), 100, None) == UNS

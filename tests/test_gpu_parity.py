@@ -1,0 +1,90 @@
+"""GPU parity: every core, every variant, through the C ABI, against the oracle.
+
+Small workloads (the tiny decoder-layer pass and ragged shapes that leave idle
+lanes, idle threads and odd tails) are compared element by element over the
+whole output.  The full-size workloads run in the same launch configuration
+as the benchmark and are compared on sampled tokens (first, last, middle and
+seeded random ones), which the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gate_cores_b200 import inputs
+from gate_cores_b200.inputs import Workload
+
+from . import harness
+from .parity import check
+
+pytestmark = pytest.mark.gpu
+
+RAGGED = [
+    Workload("ragged_t37_h264", hidden=264, hq=6, hkv=2, head_dim=80, rope_base=1.0e4,
+             batch=1, seqlen=37),
+    Workload("ragged_b3s5_h40", hidden=40, hq=3, hkv=1, head_dim=16, rope_base=1.0e4,
+             batch=3, seqlen=5),
+    Workload("ragged_thd_h512", hidden=512, hq=8, hkv=4, head_dim=64, rope_base=5.0e5,
+             layout="thd", positions="restart", num_seqs=7, seq_len_range=(0, 40)),
+    Workload("ragged_t1_h4096", hidden=4096, hq=32, hkv=8, head_dim=128, rope_base=5.0e5,
+             batch=1, seqlen=1),
+    Workload("ragged_t300_h8192", hidden=8192, hq=64, hkv=8, head_dim=256, rope_base=5.0e5,
+             batch=3, seqlen=100, outlier_frac=0.01),
+]
+
+SMALL = [inputs.WORKLOADS["tiny_t64_h256"]] + RAGGED
+CASES = [(core, var) for core in inputs.CORES for var in harness.VARIANTS[core]]
+
+
+def _compare(wl, core, ci, rows=None, tag=""):
+    outs = harness.run_gpu(wl, core, ci)
+    torch.cuda.synchronize()
+    refs = harness.run_oracle(wl, core, ci, rows)
+    stats = []
+    for o, r in zip(outs, refs):
+        g = harness.to_host(o, rows)
+        stats.append(check(g, r, f"{wl.name}/{core}/{tag}"))
+    return stats
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+@pytest.mark.parametrize("core,variant", CASES, ids=lambda x: str(x))
+def test_small_full_outputs(cuda_ok, wl, core, variant):
+    if core == "qk_norm_rope" and variant == "f32" and wl.head_dim // 4 > 32:
+        pytest.skip("f32 heads above 512 bytes are outside the documented limit")
+    ci = harness.make(wl, core, variant)
+    _compare(wl, core, ci, None, variant)
+
+
+FULL = ["prefill_t8192_h4096", "decode_t128_h4096", "thd16_h5120", "large_t32768_h8192"]
+FULL_CASES = [(c, harness.DEFAULT_VARIANT[c]) for c in inputs.CORES] + [
+    ("qk_norm_rope", "v2"), ("norm_residual", "gain_before"), ("output_norm_gate", "per_token"),
+    ("rms_norm", "f32_io")]
+
+
+@pytest.mark.parametrize("name", FULL)
+@pytest.mark.parametrize("core,variant", FULL_CASES, ids=lambda x: str(x))
+def test_full_size_sampled(cuda_ok, name, core, variant):
+    wl = inputs.WORKLOADS[name]
+    ci = harness.make(name, core, variant)
+    T = inputs.num_tokens(wl)
+    rows = harness.sample_rows(T, 40, seed=hash(core) & 0xFFFF)
+    _compare(wl, core, ci, rows, variant)
+
+
+def test_positions_explicit_equal_derived_bitwise(cuda_ok):
+    for name in ("prefill_t8192_h4096", "thd16_h5120"):
+        wl = inputs.WORKLOADS[name]
+        a = harness.run_gpu(wl, "qk_norm_rope", harness.make(name, "qk_norm_rope", "upcast"))
+        b = harness.run_gpu(wl, "qk_norm_rope", harness.make(name, "qk_norm_rope", "explicit_pos"))
+        for x, y in zip(a, b):
+            assert torch.equal(x.view(torch.int16), y.view(torch.int16))
+
+
+def test_ambiguity_is_rare(cuda_ok):
+    # the dual-candidate rule must stay a corner case, not a loophole
+    wl = inputs.WORKLOADS["prefill_t8192_h4096"]
+    for core in ("qk_norm_rope", "norm_residual"):
+        ci = harness.make(wl.name, core, harness.DEFAULT_VARIANT[core])
+        rows = harness.sample_rows(inputs.num_tokens(wl), 64)
+        for st in _compare(wl, core, ci, rows, "ambig"):
+            assert st["ambiguous"] <= max(10, 2e-3 * st["n"]), st
