@@ -127,8 +127,8 @@ int muse_oracle_positions(int layout, int64_t batch, int64_t seqlen,
 
 /* ------------------------------------------------------------ shared bits */
 
-/* r(x) = 1 / sqrt(mean of squares + eps): "Stabilizer added to the mean
- * squared activation" (parameter eps of _rms_norm_core). */
+/* r(x) = 1 / sqrt(mean of squares + eps): eps sits inside the square root,
+ * added to the mean square (parameter eps of _rms_norm_core). */
 static double inv_rms(double sum_sq, int64_t width, float eps) {
     return 1.0 / sqrt(sum_sq / (double)width + (double)eps);
 }
@@ -237,8 +237,8 @@ static void qk_head_norm(int dtype, const void* x, int64_t base, int32_t d, floa
         if (!is_query) {
             for (int i = 0; i < nc; ++i) cand_add(&s, c[i]);
         } else {
-            /* query_scale: "Multiplier applied after the normalized query's
-             * dtype cast" - the scaled value is cast to the Q dtype again. */
+            /* query_scale multiplies the query after its cast to the Q dtype;
+             * the scaled value is cast to the Q dtype again. */
             for (int i = 0; i < nc; ++i) {
                 double c2[2];
                 int n2 = cast_candidates(dtype, c[i] * (double)query_scale, c2);
@@ -277,7 +277,7 @@ static void qk_head_out(int dtype, const cand_set* cs, int32_t d, const float* i
         double mn0 = INFINITY, mx0 = -INFINITY, mn1 = INFINITY, mx1 = -INFINITY;
         double m0 = 0.0, m1 = 0.0, y0p = 0.0, y1p = 0.0;
         if (fp32_rotation) {
-            /* "The original checkpoint computes the rotation in FP32." */
+            /* Legacy (original checkpoint) rotation: FP32 arithmetic. */
             for (int ia = 0; ia < A->n; ++ia)
                 for (int ib = 0; ib < B->n; ++ib) {
                     const double a = A->v[ia], b = B->v[ib];
@@ -290,10 +290,10 @@ static void qk_head_out(int dtype, const cand_set* cs, int32_t d, const float* i
                     if (ia == 0 && ib == 0) { y0p = y0; y1p = y1; }
                 }
         } else {
-            /* "The HF release rounds both products in the Q/K dtype before
-             * adding them": cos/sin are cast to the Q/K dtype, each product is
-             * rounded to it, and the sum is cast once more.  Every step after
-             * the candidate casts is exact in FP32, so mag stays 0. */
+            /* v2 (HF release) rotation in the Q/K dtype: cos/sin are cast to
+             * it, each of the two products is rounded to it before the
+             * addition, and the sum is cast once more.  Every step after the
+             * candidate casts is exact in FP32, so mag stays 0. */
             double C[2], S[2];
             const int nC = cast_candidates(dtype, c, C);
             const int nS = cast_candidates(dtype, s, S);
@@ -392,7 +392,7 @@ int muse_oracle_output_norm_gate(int dtype, const void* o, const void* g, int64_
 /* _norm_residual_core with the declared learned blend
  * h' = cos(theta) * h + sin(theta) * nb: the branch is normalised (gain after
  * the norm, or before it when input_scale is set), cast back to the branch
- * dtype ("Normalization casts back to this dtype before residual blending"),
+ * dtype before the blend (the branch cast is left unchanged by the fusion),
  * then blended into the FP32 stream per channel. */
 int muse_oracle_norm_residual(const float* stream, int branch_dtype, const void* branch,
                               int64_t rows, int64_t hidden, const float* gain,
