@@ -28,7 +28,7 @@ MUSE_LAYOUT_THD = 1
 EXPORTS = (
     "muse_version", "muse_status_string", "muse_last_error", "muse_rms_norm",
     "muse_input_scale_norm", "muse_qk_norm_rope", "muse_output_norm_gate",
-    "muse_norm_residual", "muse_stream_copy",
+    "muse_norm_residual", "muse_device_error", "muse_stream_copy",
 )
 
 
@@ -71,6 +71,7 @@ def load() -> ctypes.CDLL:
         lib.muse_output_norm_gate.argtypes = [P, P, P, c_int, i64, i32, i32, i32, f32, P]
         lib.muse_norm_residual.argtypes = [P, P, P, c_int, i64, i64, P, f32, P, c_int, f32, P]
         lib.muse_stream_copy.argtypes = [P, P, i64, P]
+        lib.muse_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), c_int]
         for name in EXPORTS[3:]:
             getattr(lib, name).restype = c_int
         _lib = lib
@@ -128,6 +129,14 @@ def muse_norm_residual(stream_in, branch, stream_out, branch_dtype, rows, hidden
                        gain_offset, theta, input_scale, norm_eps, stream) -> None:
     _call("muse_norm_residual", stream_in, branch, stream_out, branch_dtype, rows, hidden, gain,
           gain_offset, theta, int(input_scale), norm_eps, stream)
+
+
+def muse_device_error(clear: bool = False) -> int:
+    """Device-side error word of the current device (bit 0: a bounded mbarrier
+    wait in a row kernel timed out).  Synchronous."""
+    flags = ctypes.c_uint(0)
+    _call("muse_device_error", ctypes.byref(flags), int(clear))
+    return flags.value
 
 
 def muse_stream_copy(src, dst, nbytes, stream) -> None:

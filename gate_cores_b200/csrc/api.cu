@@ -135,19 +135,19 @@ int sm_count() {
     return n;
 }
 
-int blocks_per_sm(const void* kernel, int threads) {
+int blocks_per_sm(const void* kernel, int threads, size_t dyn_smem) {
     static std::mutex mu;
-    static std::map<std::tuple<const void*, int, int>, int> cache;
+    static std::map<std::tuple<const void*, int, int, size_t>, int> cache;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 1;
-    const auto key = std::make_tuple(kernel, threads, dev);
+    const auto key = std::make_tuple(kernel, threads, dev, dyn_smem);
     {
         std::lock_guard<std::mutex> lock(mu);
         auto it = cache.find(key);
         if (it != cache.end()) return it->second;
     }
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n < 1) n = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, dyn_smem) != cudaSuccess || n < 1) n = 1;
     std::lock_guard<std::mutex> lock(mu);
     cache[key] = n;
     return n;
@@ -360,6 +360,11 @@ muse_status muse_norm_residual(const float* stream_in, const void* branch, float
     a.eps = norm_eps;
     const muse::RowOp op = input_scale ? muse::RowOp::kResidualIS : muse::RowOp::kResidual;
     return from_cuda(muse::launch_row(branch_dtype, op, a, stream), name);
+}
+
+muse_status muse_device_error(unsigned int* flags, int clear) {
+    if (!flags) return fail(MUSE_ERR_INVALID_ARGUMENT, "muse_device_error: null flags");
+    return from_cuda(muse::read_device_error(flags, clear != 0), "muse_device_error");
 }
 
 muse_status muse_stream_copy(const void* src, void* dst, int64_t bytes, cudaStream_t stream) {

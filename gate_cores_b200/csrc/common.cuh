@@ -66,6 +66,82 @@ template <> __device__ __forceinline__ uint4 pack<float>(const float* f) {
                       __float_as_uint(f[2]), __float_as_uint(f[3]));
 }
 
+// ---- Packed FP32 pairs (Blackwell f32x2 instructions: one issue slot, two
+// IEEE round-to-nearest FP32 operations, bit-identical to two scalar ones).
+typedef unsigned long long f32x2;
+
+__device__ __forceinline__ f32x2 f2_make(float lo, float hi) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_split(f32x2 p, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
+}
+__device__ __forceinline__ f32x2 f2_mul(f32x2 a, f32x2 b) {
+    f32x2 r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) {
+    f32x2 r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// A 16-byte vector of T as Vec<T>::N / 2 packed pairs (element order kept).
+template <typename T> __device__ __forceinline__ void to_pairs(const uint4& v, f32x2* p);
+template <> __device__ __forceinline__ void to_pairs<__nv_bfloat16>(const uint4& v, f32x2* p) {
+    p[0] = f2_make(bf16_lo(v.x), bf16_hi(v.x));
+    p[1] = f2_make(bf16_lo(v.y), bf16_hi(v.y));
+    p[2] = f2_make(bf16_lo(v.z), bf16_hi(v.z));
+    p[3] = f2_make(bf16_lo(v.w), bf16_hi(v.w));
+}
+template <> __device__ __forceinline__ void to_pairs<float>(const uint4& v, f32x2* p) {
+    p[0] = f2_make(__uint_as_float(v.x), __uint_as_float(v.y));
+    p[1] = f2_make(__uint_as_float(v.z), __uint_as_float(v.w));
+}
+
+// Pairs -> 16-byte vector of T (bf16: round to nearest even).
+template <typename T> __device__ __forceinline__ uint4 from_pairs(const f32x2* p);
+template <> __device__ __forceinline__ uint4 from_pairs<__nv_bfloat16>(const f32x2* p) {
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        float lo, hi;
+        f2_split(p[k], lo, hi);
+        w[k] = pack_bf16x2(lo, hi);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+template <> __device__ __forceinline__ uint4 from_pairs<float>(const f32x2* p) {
+    float a, b, c, d;
+    f2_split(p[0], a, b);
+    f2_split(p[1], c, d);
+    return make_uint4(__float_as_uint(a), __float_as_uint(b), __float_as_uint(c), __float_as_uint(d));
+}
+
+// Round a pair to T and back (the cast at a dtype boundary; exact for FP32).
+template <typename T> __device__ __forceinline__ f32x2 round_pair(f32x2 p);
+template <> __device__ __forceinline__ f32x2 round_pair<__nv_bfloat16>(f32x2 p) {
+    float lo, hi;
+    f2_split(p, lo, hi);
+    const uint32_t w = pack_bf16x2(lo, hi);
+    return f2_make(bf16_lo(w), bf16_hi(w));
+}
+template <> __device__ __forceinline__ f32x2 round_pair<float>(f32x2 p) { return p; }
+
+__device__ __forceinline__ float f2_sum(f32x2 p) {
+    float lo, hi;
+    f2_split(p, lo, hi);
+    return lo + hi;
+}
+
 // Sum of squares of N floats as a balanced tree (short rounding chains).
 template <int N> __device__ __forceinline__ float sum_sq(const float* f) {
     if constexpr (N == 1) {
@@ -111,10 +187,10 @@ __device__ __forceinline__ float inv_rms_fast(float sum_sq_total, float inv_widt
     return rsqrtf(sum_sq_total * inv_width + eps);
 }
 
-// Reciprocal (rcp.approx.f32, at most 1 ulp; keeps subnormal results).
-__device__ __forceinline__ float rcp_approx(float x) {
+// Reciprocal of a normal number (rcp.approx.ftz.f32, at most 1 ulp).
+__device__ __forceinline__ float rcp_approx_ftz(float x) {
     float r;
-    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
     return r;
 }
 
@@ -136,7 +212,8 @@ template <typename T> __device__ __forceinline__ float times_sigmoid(float v, fl
 template <> __device__ __forceinline__ float times_sigmoid<__nv_bfloat16>(float v, float g) {
     const float a = fabsf(g);
     const float t = exp2_approx(fmaf(-a, 1.44269504088896341f, 64.0f));
-    const float d = rcp_approx(fmaf(t, 0x1p-64f, 1.0f));
+    // 1 + t 2^-64 lies in [1, 2]: the flush-to-zero reciprocal is exact enough.
+    const float d = rcp_approx_ftz(fmaf(t, 0x1p-64f, 1.0f));
     return g >= 0.0f ? v * d : ((v * t) * d) * 0x1p-64f;
 }
 // FP32 outputs need FP32 accuracy: expf (at most 2 ulp) and IEEE division;

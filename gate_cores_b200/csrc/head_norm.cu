@@ -14,19 +14,15 @@
 namespace muse {
 namespace {
 
-// Sum of squares of one 16-byte vector.
-template <typename T> __device__ __forceinline__ float vec_sum_sq(const uint4& v);
-template <> __device__ __forceinline__ float vec_sum_sq<__nv_bfloat16>(const uint4& v) {
-    float s0 = bf16_lo(v.x) * bf16_lo(v.x), s1 = bf16_hi(v.x) * bf16_hi(v.x);
-    s0 = fmaf(bf16_lo(v.y), bf16_lo(v.y), s0); s1 = fmaf(bf16_hi(v.y), bf16_hi(v.y), s1);
-    s0 = fmaf(bf16_lo(v.z), bf16_lo(v.z), s0); s1 = fmaf(bf16_hi(v.z), bf16_hi(v.z), s1);
-    s0 = fmaf(bf16_lo(v.w), bf16_lo(v.w), s0); s1 = fmaf(bf16_hi(v.w), bf16_hi(v.w), s1);
-    return s0 + s1;
-}
-template <> __device__ __forceinline__ float vec_sum_sq<float>(const uint4& v) {
-    float f[4];
-    unpack<float>(v, f);
-    return sum_sq<4>(f);
+// Sum of squares of one 16-byte vector (two packed partial sums).
+template <typename T> __device__ __forceinline__ float vec_sum_sq(const uint4& v) {
+    constexpr int P = Vec<T>::N / 2;
+    f32x2 p[P];
+    to_pairs<T>(v, p);
+    f32x2 acc = f2_mul(p[0], p[0]);
+#pragma unroll
+    for (int k = 1; k < P; ++k) acc = f2_fma(p[k], p[k], acc);
+    return f2_sum(acc);
 }
 
 // ------------------------------------------------------------ core 4 per head
@@ -102,9 +98,11 @@ __device__ __forceinline__ uint4 qk_vec(const uint4& in, float r, bool scale, fl
                                         const float* cs, const float* sn);
 
 template <bool ROPE, bool UPCAST>
-__device__ __forceinline__ uint32_t qk_pair_bf16(uint32_t w, float r, bool scale, float qs, float c, float s) {
+__device__ __forceinline__ uint32_t qk_pair_bf16(uint32_t w, f32x2 r2, bool scale, float qs, float c, float s) {
     // cast of the normalised pair to bf16 (cvt.rn.bf16x2)
-    uint32_t n = pack_bf16x2(bf16_lo(w) * r, bf16_hi(w) * r);
+    float n0, n1;
+    f2_split(f2_mul(f2_make(bf16_lo(w), bf16_hi(w)), r2), n0, n1);
+    uint32_t n = pack_bf16x2(n0, n1);
     if (scale) n = pack_bf16x2(bf16_lo(n) * qs, bf16_hi(n) * qs);
     if constexpr (!ROPE) {
         return n;
@@ -124,26 +122,29 @@ __device__ __forceinline__ uint32_t qk_pair_bf16(uint32_t w, float r, bool scale
 template <>
 __device__ __forceinline__ uint4 qk_vec<__nv_bfloat16, false, true>(const uint4& in, float r, bool scale, float qs,
                                                                    const float*, const float*) {
-    return make_uint4(qk_pair_bf16<false, true>(in.x, r, scale, qs, 0, 0),
-                      qk_pair_bf16<false, true>(in.y, r, scale, qs, 0, 0),
-                      qk_pair_bf16<false, true>(in.z, r, scale, qs, 0, 0),
-                      qk_pair_bf16<false, true>(in.w, r, scale, qs, 0, 0));
+    const f32x2 r2 = f2_make(r, r);
+    return make_uint4(qk_pair_bf16<false, true>(in.x, r2, scale, qs, 0, 0),
+                      qk_pair_bf16<false, true>(in.y, r2, scale, qs, 0, 0),
+                      qk_pair_bf16<false, true>(in.z, r2, scale, qs, 0, 0),
+                      qk_pair_bf16<false, true>(in.w, r2, scale, qs, 0, 0));
 }
 template <>
 __device__ __forceinline__ uint4 qk_vec<__nv_bfloat16, true, true>(const uint4& in, float r, bool scale, float qs,
                                                                   const float* c, const float* s) {
-    return make_uint4(qk_pair_bf16<true, true>(in.x, r, scale, qs, c[0], s[0]),
-                      qk_pair_bf16<true, true>(in.y, r, scale, qs, c[1], s[1]),
-                      qk_pair_bf16<true, true>(in.z, r, scale, qs, c[2], s[2]),
-                      qk_pair_bf16<true, true>(in.w, r, scale, qs, c[3], s[3]));
+    const f32x2 r2 = f2_make(r, r);
+    return make_uint4(qk_pair_bf16<true, true>(in.x, r2, scale, qs, c[0], s[0]),
+                      qk_pair_bf16<true, true>(in.y, r2, scale, qs, c[1], s[1]),
+                      qk_pair_bf16<true, true>(in.z, r2, scale, qs, c[2], s[2]),
+                      qk_pair_bf16<true, true>(in.w, r2, scale, qs, c[3], s[3]));
 }
 template <>
 __device__ __forceinline__ uint4 qk_vec<__nv_bfloat16, true, false>(const uint4& in, float r, bool scale, float qs,
                                                                    const float* c, const float* s) {
-    return make_uint4(qk_pair_bf16<true, false>(in.x, r, scale, qs, c[0], s[0]),
-                      qk_pair_bf16<true, false>(in.y, r, scale, qs, c[1], s[1]),
-                      qk_pair_bf16<true, false>(in.z, r, scale, qs, c[2], s[2]),
-                      qk_pair_bf16<true, false>(in.w, r, scale, qs, c[3], s[3]));
+    const f32x2 r2 = f2_make(r, r);
+    return make_uint4(qk_pair_bf16<true, false>(in.x, r2, scale, qs, c[0], s[0]),
+                      qk_pair_bf16<true, false>(in.y, r2, scale, qs, c[1], s[1]),
+                      qk_pair_bf16<true, false>(in.z, r2, scale, qs, c[2], s[2]),
+                      qk_pair_bf16<true, false>(in.w, r2, scale, qs, c[3], s[3]));
 }
 // FP32 tensors: the casts are exact and the rotation is FP32 in both modes.
 template <bool ROPE>

@@ -24,6 +24,7 @@ struct RowArgs {
     float* stream_out;      // core 5
     const float* gain;      // may be null
     const float* theta;     // core 5
+    const float* cos_sin;   // core 5: [cos(theta) | sin(theta)] table, or null
     int64_t rows;
     int64_t x_stride, y_stride, gate_stride, s_in_stride, s_out_stride;
     int32_t width;
@@ -65,13 +66,18 @@ struct QkArgs {
 };
 
 // Returns cudaSuccess or the launch error.
+// launch_row: TMA-pipelined kernels (row_tma.cu), falling back to
+// launch_row_regs (register-staged, row_norm.cu) for rows too wide to stage.
 cudaError_t launch_row(int dtype, RowOp op, const RowArgs& a, cudaStream_t s);
+cudaError_t launch_row_regs(int dtype, RowOp op, const RowArgs& a, cudaStream_t s);
+// Device-side error word (bit 0: a bounded mbarrier wait timed out).
+cudaError_t read_device_error(unsigned int* out, bool clear);
 cudaError_t launch_head_gate(int dtype, const HeadGateArgs& a, cudaStream_t s);
 cudaError_t launch_qk(int dtype, int use_rope, int upcast_rope, const QkArgs& a, cudaStream_t s);
 cudaError_t launch_copy(const void* src, void* dst, int64_t bytes, cudaStream_t s);
 
 // Device facts for grid sizing (cached per device).
 int sm_count();
-int blocks_per_sm(const void* kernel, int threads);
+int blocks_per_sm(const void* kernel, int threads, size_t dyn_smem = 0);
 
 }  // namespace muse

@@ -13,8 +13,8 @@ namespace muse {
 namespace {
 
 constexpr int kMaxThreads = 512;  // threads per CTA (one row)
-constexpr int kResidualChunk = 4;  // rows per CTA for core 5
-constexpr int kRowChunk = 2;       // rows per CTA for cores 1, 2 and 4
+constexpr int kResidualChunk = 8;  // rows per CTA for core 5
+constexpr int kRowChunk = 4;       // rows per CTA for cores 1, 2 and 4
 
 __host__ __device__ constexpr bool is_residual(RowOp op) { return op == RowOp::kResidual || op == RowOp::kResidualIS; }
 __host__ __device__ constexpr bool scales_first(RowOp op) { return op == RowOp::kInputScale || op == RowOp::kResidualIS; }
@@ -28,51 +28,89 @@ struct RowFrag {
     uint4 h[is_residual(OP) ? VPT * SV : 1];
 };
 
-template <typename T, RowOp OP, int VPT, bool HAS_GAIN, int STAGES>
+// Per-thread constant pieces (float4) per slot: effective gain, cos, sin.
+template <typename T, RowOp OP, bool HAS_GAIN>
+__host__ __device__ constexpr int const_pieces_per_slot() {
+    return (HAS_GAIN ? Vec<T>::N / 4 : 0) + (is_residual(OP) ? 2 * (Vec<T>::N / 4) : 0);
+}
+
+// CSM: the constants live in shared memory (each thread reads back only what
+// it wrote, so no barrier) instead of registers - fewer registers, more
+// resident CTAs, more rows in flight.
+template <typename T, RowOp OP, int VPT, bool HAS_GAIN, int STAGES, bool CSM>
 __device__ __forceinline__ void row_norm_body(const RowArgs& a) {
     constexpr int V = Vec<T>::N;
     constexpr int SV = V / 4;
+    constexpr int CP = const_pieces_per_slot<T, OP, HAS_GAIN>();
+    constexpr int GOFF = 0, COFF = HAS_GAIN ? SV : 0, SOFF = COFF + SV;
     using Frag = RowFrag<T, OP, VPT>;
     __shared__ float red[2][32];
+    extern __shared__ float4 csm[];  // [VPT * CP][nt] when CSM
 
     const int tid = threadIdx.x;
     const int nt = blockDim.x;
     const int nvec = a.width / V;
-    const float widthf = (float)a.width;
+    const float inv_width = 1.0f / (float)a.width;
 
     bool valid[VPT];
 #pragma unroll
     for (int i = 0; i < VPT; ++i) valid[i] = tid + i * nt < nvec;
 
     // Per-slot constants, fixed for the CTA's lifetime: effective gain
-    // (16-byte loads) and the blend's cos/sin.
-    float w[HAS_GAIN ? VPT : 1][V];
-    float cth[is_residual(OP) ? VPT : 1][V];
-    float sth[is_residual(OP) ? VPT : 1][V];
+    // (16-byte loads) and the blend's cos/sin (computed, or read from a
+    // [cos | sin] table when the caller provides one).
+    constexpr int RV = CSM ? 1 : V;
+    float w[HAS_GAIN ? VPT : 1][RV];
+    float cth[is_residual(OP) ? VPT : 1][RV];
+    float sth[is_residual(OP) ? VPT : 1][RV];
+    auto put = [&](int i, int q, float4 v, float (&dst)[is_residual(OP) ? VPT : 1][RV], int k) {
+        if constexpr (CSM) {
+            csm[(i * CP + q) * nt + tid] = v;
+        } else {
+            dst[i][4 * k + 0] = v.x; dst[i][4 * k + 1] = v.y; dst[i][4 * k + 2] = v.z; dst[i][4 * k + 3] = v.w;
+        }
+    };
     auto load_constants = [&]() {
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
             const int v = valid[i] ? tid + i * nt : 0;
-            if constexpr (HAS_GAIN) {
 #pragma unroll
-                for (int k = 0; k < V / 4; ++k) {
-                    const float4 g4 = __ldg(reinterpret_cast<const float4*>(a.gain) + v * (V / 4) + k);
-                    w[i][4 * k + 0] = g4.x + a.gain_offset;
-                    w[i][4 * k + 1] = g4.y + a.gain_offset;
-                    w[i][4 * k + 2] = g4.z + a.gain_offset;
-                    w[i][4 * k + 3] = g4.w + a.gain_offset;
+            for (int k = 0; k < SV; ++k) {
+                if constexpr (HAS_GAIN) {
+                    float4 g4 = __ldg(reinterpret_cast<const float4*>(a.gain) + v * SV + k);
+                    g4.x += a.gain_offset; g4.y += a.gain_offset; g4.z += a.gain_offset; g4.w += a.gain_offset;
+                    if constexpr (CSM) {
+                        csm[(i * CP + GOFF + k) * nt + tid] = g4;
+                    } else {
+                        w[i][4 * k + 0] = g4.x; w[i][4 * k + 1] = g4.y; w[i][4 * k + 2] = g4.z; w[i][4 * k + 3] = g4.w;
+                    }
                 }
-            }
-            if constexpr (is_residual(OP)) {
-#pragma unroll
-                for (int k = 0; k < V / 4; ++k) {
-                    const float4 t4 = __ldg(reinterpret_cast<const float4*>(a.theta) + v * (V / 4) + k);
-                    const float th[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) sincosf(th[e], &sth[i][4 * k + e], &cth[i][4 * k + e]);
+                if constexpr (is_residual(OP)) {
+                    float4 c4, s4;
+                    if (a.cos_sin) {  // precomputed [cos | sin] table
+                        c4 = __ldg(reinterpret_cast<const float4*>(a.cos_sin) + v * SV + k);
+                        s4 = __ldg(reinterpret_cast<const float4*>(a.cos_sin + a.width) + v * SV + k);
+                    } else {
+                        const float4 t4 = __ldg(reinterpret_cast<const float4*>(a.theta) + v * SV + k);
+                        sincosf(t4.x, &s4.x, &c4.x);
+                        sincosf(t4.y, &s4.y, &c4.y);
+                        sincosf(t4.z, &s4.z, &c4.z);
+                        sincosf(t4.w, &s4.w, &c4.w);
+                    }
+                    put(i, COFF + k, c4, cth, k);
+                    put(i, SOFF + k, s4, sth, k);
                 }
             }
         }
+    };
+    // 4 constants of slot i, group k (elements 4k .. 4k+3)
+    auto piece = [&](int i, int q, const float (&src)[is_residual(OP) ? VPT : 1][RV], int k) -> float4 {
+        if constexpr (CSM) return csm[(i * CP + q) * nt + tid];
+        else return make_float4(src[i][4 * k], src[i][4 * k + 1], src[i][4 * k + 2], src[i][4 * k + 3]);
+    };
+    auto wpiece = [&](int i, int k) -> float4 {
+        if constexpr (CSM) return csm[(i * CP + GOFF + k) * nt + tid];
+        else return make_float4(w[i][4 * k], w[i][4 * k + 1], w[i][4 * k + 2], w[i][4 * k + 3]);
     };
 
     auto load = [&](int64_t row, Frag& f) {
@@ -103,11 +141,14 @@ __device__ __forceinline__ void row_norm_body(const RowArgs& a) {
             unpack<T>(f.x[i], xf[i]);
             if constexpr (scales_first(OP) && HAS_GAIN) {
 #pragma unroll
-                for (int e = 0; e < V; ++e) xf[i][e] = xf[i][e] * w[i][e];
+                for (int k = 0; k < SV; ++k) {
+                    const float4 w4 = wpiece(i, k);
+                    xf[i][4 * k] *= w4.x; xf[i][4 * k + 1] *= w4.y; xf[i][4 * k + 2] *= w4.z; xf[i][4 * k + 3] *= w4.w;
+                }
             }
             ss += sum_sq<V>(xf[i]);
         }
-        const float r = inv_rms(block_sum(ss, red, bank), widthf, a.eps);
+        const float r = inv_rms_fast(block_sum(ss, red, bank), inv_width, a.eps);
 
         if constexpr (OP == RowOp::kRms || OP == RowOp::kInputScale || OP == RowOp::kNormGate) {
             char* yr = static_cast<char*>(a.y) + row * a.y_stride * (int64_t)sizeof(T);
@@ -117,11 +158,18 @@ __device__ __forceinline__ void row_norm_body(const RowArgs& a) {
                 float gf[V];
                 if constexpr (OP == RowOp::kNormGate) unpack<T>(f.g[i], gf);
 #pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    float t = xf[i][e] * r;
-                    if constexpr (OP == RowOp::kRms && HAS_GAIN) t = t * w[i][e];
-                    if constexpr (OP == RowOp::kNormGate) t = times_sigmoid<T>(t, gf[e]);
-                    o[e] = t;
+                for (int k = 0; k < SV; ++k) {
+                    float4 w4 = make_float4(1.f, 1.f, 1.f, 1.f);
+                    if constexpr (OP == RowOp::kRms && HAS_GAIN) w4 = wpiece(i, k);
+                    const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int e = 4 * k + j;
+                        float t = xf[i][e] * r;
+                        if constexpr (OP == RowOp::kRms && HAS_GAIN) t = t * wv[j];
+                        if constexpr (OP == RowOp::kNormGate) t = times_sigmoid<T>(t, gf[e]);
+                        o[e] = t;
+                    }
                 }
                 if (valid[i]) st_vec(yr + (int64_t)(tid + i * nt) * 16, pack<T>(o));
             }
@@ -134,11 +182,20 @@ __device__ __forceinline__ void row_norm_body(const RowArgs& a) {
                 for (int k = 0; k < SV; ++k) unpack<float>(f.h[i * SV + k], hin + 4 * k);
                 float o[V];
 #pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    float t = xf[i][e] * r;  // z r when the gain came first
-                    if constexpr (OP == RowOp::kResidual && HAS_GAIN) t = t * w[i][e];
-                    const float nb = round_to<T>(t);  // cast back to the branch dtype
-                    o[e] = cth[i][e] * hin[e] + sth[i][e] * nb;
+                for (int k = 0; k < SV; ++k) {
+                    float4 w4 = make_float4(1.f, 1.f, 1.f, 1.f);
+                    if constexpr (OP == RowOp::kResidual && HAS_GAIN) w4 = wpiece(i, k);
+                    const float4 c4 = piece(i, COFF + k, cth, k), s4 = piece(i, SOFF + k, sth, k);
+                    const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+                    const float cv[4] = {c4.x, c4.y, c4.z, c4.w}, sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int e = 4 * k + j;
+                        float t = xf[i][e] * r;  // z r when the gain came first
+                        if constexpr (OP == RowOp::kResidual && HAS_GAIN) t = t * wv[j];
+                        const float nb = round_to<T>(t);  // cast back to the branch dtype
+                        o[e] = cv[j] * hin[e] + sv[j] * nb;
+                    }
                 }
                 if (valid[i]) {
 #pragma unroll
@@ -171,25 +228,25 @@ __device__ __forceinline__ void row_norm_body(const RowArgs& a) {
 }
 
 // One entry symbol per core, so launch lists and profiles name the core.
-template <typename T, int VPT, bool G, int S>
+template <typename T, int VPT, bool G, int S, bool CSM>
 __global__ void __launch_bounds__(kMaxThreads) rms_norm_kernel(const __grid_constant__ RowArgs a) {
-    row_norm_body<T, RowOp::kRms, VPT, G, S>(a);
+    row_norm_body<T, RowOp::kRms, VPT, G, S, CSM>(a);
 }
-template <typename T, int VPT, bool G, int S>
+template <typename T, int VPT, bool G, int S, bool CSM>
 __global__ void __launch_bounds__(kMaxThreads) input_scale_norm_kernel(const __grid_constant__ RowArgs a) {
-    row_norm_body<T, RowOp::kInputScale, VPT, G, S>(a);
+    row_norm_body<T, RowOp::kInputScale, VPT, G, S, CSM>(a);
 }
-template <typename T, int VPT, bool G, int S>
+template <typename T, int VPT, bool G, int S, bool CSM>
 __global__ void __launch_bounds__(kMaxThreads) output_norm_gate_row_kernel(const __grid_constant__ RowArgs a) {
-    row_norm_body<T, RowOp::kNormGate, VPT, G, S>(a);
+    row_norm_body<T, RowOp::kNormGate, VPT, G, S, CSM>(a);
 }
-template <typename T, int VPT, bool G, int S>
+template <typename T, int VPT, bool G, int S, bool CSM>
 __global__ void __launch_bounds__(kMaxThreads) norm_residual_kernel(const __grid_constant__ RowArgs a) {
-    row_norm_body<T, RowOp::kResidual, VPT, G, S>(a);
+    row_norm_body<T, RowOp::kResidual, VPT, G, S, CSM>(a);
 }
-template <typename T, int VPT, bool G, int S>
+template <typename T, int VPT, bool G, int S, bool CSM>
 __global__ void __launch_bounds__(kMaxThreads) norm_residual_input_scale_kernel(const __grid_constant__ RowArgs a) {
-    row_norm_body<T, RowOp::kResidualIS, VPT, G, S>(a);
+    row_norm_body<T, RowOp::kResidualIS, VPT, G, S, CSM>(a);
 }
 
 // Row buffers in the ring: one.  Measured on B200 (prefill rows, H = 4096):
@@ -197,36 +254,52 @@ __global__ void __launch_bounds__(kMaxThreads) norm_residual_input_scale_kernel(
 template <RowOp OP>
 constexpr int stages() { return 1; }
 
+// Constants (gain, cos/sin) in shared memory: holding them in registers
+// (8 to 24 floats per slot) costs resident CTAs and rows in flight - measured
+// at prefill sizes on B200.
+template <RowOp OP>
+constexpr bool const_in_smem() { return true; }
+
 template <typename T, RowOp OP, int VPT, bool G>
 constexpr auto row_kernel() {
     constexpr int S = stages<OP>();
-    if constexpr (OP == RowOp::kRms) return rms_norm_kernel<T, VPT, G, S>;
-    else if constexpr (OP == RowOp::kInputScale) return input_scale_norm_kernel<T, VPT, G, S>;
-    else if constexpr (OP == RowOp::kNormGate) return output_norm_gate_row_kernel<T, VPT, G, S>;
-    else if constexpr (OP == RowOp::kResidual) return norm_residual_kernel<T, VPT, G, S>;
-    else return norm_residual_input_scale_kernel<T, VPT, G, S>;
+    constexpr bool C = const_in_smem<OP>();
+    if constexpr (OP == RowOp::kRms) return rms_norm_kernel<T, VPT, G, S, C>;
+    else if constexpr (OP == RowOp::kInputScale) return input_scale_norm_kernel<T, VPT, G, S, C>;
+    else if constexpr (OP == RowOp::kNormGate) return output_norm_gate_row_kernel<T, VPT, G, S, C>;
+    else if constexpr (OP == RowOp::kResidual) return norm_residual_kernel<T, VPT, G, S, C>;
+    else return norm_residual_input_scale_kernel<T, VPT, G, S, C>;
 }
 
-template <typename T, RowOp OP, int VPT>
-cudaError_t launch_row_vpt(const RowArgs& a0, int nvec, cudaStream_t s) {
+template <typename T, RowOp OP, int VPT, bool G>
+cudaError_t launch_row_g(const RowArgs& a0, int nvec, cudaStream_t s) {
     RowArgs a = a0;
     const int nt = ((nvec + VPT - 1) / VPT + 31) / 32 * 32;
     a.rows_per_cta = is_residual(OP) ? kResidualChunk : kRowChunk;
-    auto kern = a.gain ? row_kernel<T, OP, VPT, true>() : row_kernel<T, OP, VPT, false>();
+    auto kern = row_kernel<T, OP, VPT, G>();
+    const size_t smem = const_in_smem<OP>() ? (size_t)16 * nt * VPT * const_pieces_per_slot<T, OP, G>() : 0;
+    if (smem > 32 * 1024) {  // above the default 48 KB once the static part is added
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
     const int64_t grid = (a.rows + a.rows_per_cta - 1) / a.rows_per_cta;
-    kern<<<(unsigned)grid, nt, 0, s>>>(a);
+    kern<<<(unsigned)grid, nt, smem, s>>>(a);
     return cudaGetLastError();
 }
 
+template <typename T, RowOp OP, int VPT>
+cudaError_t launch_row_vpt(const RowArgs& a, int nvec, cudaStream_t s) {
+    return a.gain ? launch_row_g<T, OP, VPT, true>(a, nvec, s) : launch_row_g<T, OP, VPT, false>(a, nvec, s);
+}
+
 // Slots per thread: the fewest that fit a row into kThreadsRow threads (small
-// CTAs, many resident) - or kMaxThreads for core 5, whose per-thread cos/sin
-// registers favour fewer slots.
+// CTAs, many resident; twice that for core 5).
 constexpr int kThreadsRow = 128;
 
 template <typename T, RowOp OP>
 cudaError_t launch_row_t(const RowArgs& a, cudaStream_t s) {
     const int nvec = a.width / Vec<T>::N;
-    const int cap = is_residual(OP) ? kMaxThreads : kThreadsRow;
+    const int cap = is_residual(OP) ? 2 * kThreadsRow : kThreadsRow;
     if (nvec <= cap) return launch_row_vpt<T, OP, 1>(a, nvec, s);
     if (nvec <= 2 * cap) return launch_row_vpt<T, OP, 2>(a, nvec, s);
     if (nvec <= 4 * cap) return launch_row_vpt<T, OP, 4>(a, nvec, s);
@@ -247,7 +320,7 @@ cudaError_t launch_row_dt(RowOp op, const RowArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_row(int dtype, RowOp op, const RowArgs& a, cudaStream_t s) {
+cudaError_t launch_row_regs(int dtype, RowOp op, const RowArgs& a, cudaStream_t s) {
     return dtype == 0 ? launch_row_dt<__nv_bfloat16>(op, a, s) : launch_row_dt<float>(op, a, s);
 }
 

@@ -1,0 +1,374 @@
+// Row-wide normalisation kernels (cores 1, 2, 5 and core 4 with one norm per
+// token) on a TMA bulk-copy pipeline.
+//
+// Each CTA owns a contiguous chunk of rows.  One producer warp streams whole
+// rows (activation row, plus the gate row for core 4 or the FP32 stream row
+// for core 5) from global memory into a ring of S shared-memory stages with
+// cp.async.bulk, each stage tracked by a "full" mbarrier (transaction bytes)
+// and an "empty" mbarrier (one arrival per consumer warp).  The consumer warps
+// read their 16-byte pieces of a stage, release it, reduce the row's sum of
+// squares (named barrier among consumers only), and write the outputs.  Rows
+// in flight per SM are set by the stage count, not by registers.
+//
+// Every mbarrier wait is bounded: after kSpinLimit polls the thread records a
+// timeout in a device-wide error word (read by muse_device_error), stops, and
+// the producer waits - again bounded - for its own copies still in flight
+// before the CTA exits.
+#include <type_traits>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace muse {
+
+__device__ unsigned int g_device_error;  // bit 0: an mbarrier wait timed out
+
+namespace {
+
+constexpr uint32_t kSpinLimit = 1u << 24;
+
+__host__ __device__ constexpr bool t_is_residual(RowOp op) { return op == RowOp::kResidual || op == RowOp::kResidualIS; }
+__host__ __device__ constexpr bool t_scales_first(RowOp op) { return op == RowOp::kInputScale || op == RowOp::kResidualIS; }
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+// Bounded wait for the phase of the given parity; false on timeout.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kSpinLimit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    atomicOr(&g_device_error, 1u);
+    return false;
+}
+// Bulk copy global -> shared, completing `bytes` on the mbarrier.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+// Barrier among the consumer threads only (named barrier 1).
+__device__ __forceinline__ void consumer_sync(int nthreads) {
+    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+// Sum over the consumer threads; two banks of partials, one barrier per call.
+__device__ __forceinline__ float consumer_sum(float v, float (*red)[32], int& bank, int ncons) {
+    v = group_sum<32>(v);
+    const int nw = ncons >> 5;
+    if (nw == 1) return v;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[bank][warp] = v;
+    consumer_sync(ncons);
+    float t = lane < nw ? red[bank][lane] : 0.0f;
+    bank ^= 1;
+    return group_sum<32>(t);
+}
+
+template <typename T, RowOp OP>
+struct TmaShape {
+    static constexpr int V = Vec<T>::N;
+    static constexpr int SV = V / 4;
+};
+
+// Byte offsets of one stage: activation row, then gate row (core 4) or FP32
+// stream row (core 5), each 128-byte aligned.
+struct StageLayout {
+    uint32_t x_bytes, x_off, g_off, h_off, stage_bytes;
+};
+
+__host__ __device__ inline uint32_t align128(uint32_t v) { return (v + 127u) & ~127u; }
+
+template <typename T, RowOp OP>
+__host__ __device__ inline StageLayout stage_layout(int width) {
+    StageLayout L;
+    L.x_bytes = (uint32_t)width * sizeof(T);
+    L.x_off = 0;
+    uint32_t off = align128(L.x_bytes);
+    L.g_off = off;
+    if (OP == RowOp::kNormGate) off += align128(L.x_bytes);
+    L.h_off = off;
+    if (t_is_residual(OP)) off += align128((uint32_t)width * 4u);
+    L.stage_bytes = off;
+    return L;
+}
+
+template <typename T, RowOp OP, int VPT, bool HAS_GAIN, int S>
+__global__ void __launch_bounds__(512 + 32) row_tma_kernel(const __grid_constant__ RowArgs a) {
+    using Sh = TmaShape<T, OP>;
+    constexpr int V = Sh::V, SV = Sh::SV;
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ float red[2][32];
+    __shared__ __align__(8) uint64_t full_bar[S];
+    __shared__ __align__(8) uint64_t empty_bar[S];
+
+    const int ncons = blockDim.x - 32;  // consumer threads; the last warp produces
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int nvec = a.width / V;
+    const StageLayout L = stage_layout<T, OP>(a.width);
+
+    const int64_t r0 = (int64_t)blockIdx.x * a.rows_per_cta;
+    const int64_t r1 = min(r0 + (int64_t)a.rows_per_cta, a.rows);
+    const int n = (int)max((int64_t)0, r1 - r0);
+
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], (uint32_t)(ncons >> 5));
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (warp == (ncons >> 5)) {
+        // ---------------- producer warp: lane 0 issues whole-row bulk copies
+        if (lane == 0) {
+            uint32_t bytes = L.x_bytes;
+            if (OP == RowOp::kNormGate) bytes += L.x_bytes;
+            if (t_is_residual(OP)) bytes += (uint32_t)a.width * 4u;
+            int issued = 0;
+            bool ok = true;
+            for (int k = 0; k < n && ok; ++k) {
+                const int s = k % S;
+                if (k >= S) ok = mbar_wait(&empty_bar[s], (uint32_t)((k / S - 1) & 1));
+                if (!ok) break;
+                unsigned char* st = smem + (size_t)s * L.stage_bytes;
+                const int64_t row = r0 + k;
+                mbar_arrive_expect_tx(&full_bar[s], bytes);
+                bulk_g2s(st + L.x_off, static_cast<const char*>(a.x) + row * a.x_stride * (int64_t)sizeof(T),
+                         L.x_bytes, &full_bar[s]);
+                if constexpr (OP == RowOp::kNormGate)
+                    bulk_g2s(st + L.g_off, static_cast<const char*>(a.gate) + row * a.gate_stride * (int64_t)sizeof(T),
+                             L.x_bytes, &full_bar[s]);
+                if constexpr (t_is_residual(OP))
+                    bulk_g2s(st + L.h_off, a.stream_in + row * a.s_in_stride, (uint32_t)a.width * 4u, &full_bar[s]);
+                ++issued;
+            }
+            // Before exiting, every copy this CTA issued must have landed: in
+            // the normal path the consumers already waited on them, so these
+            // waits return at once.
+            for (int k = max(0, issued - S); k < issued; ++k)
+                if (!mbar_wait(&full_bar[k % S], (uint32_t)((k / S) & 1))) break;
+        }
+        return;
+    }
+
+    // ---------------- consumer warps
+    bool valid[VPT];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) valid[i] = tid + i * ncons < nvec;
+
+    // per-slot constants in registers (the pipeline, not registers, holds the
+    // rows in flight)
+    float w[HAS_GAIN ? VPT : 1][V];
+    float cth[t_is_residual(OP) ? VPT : 1][V];
+    float sth[t_is_residual(OP) ? VPT : 1][V];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int v = valid[i] ? tid + i * ncons : 0;
+#pragma unroll
+        for (int k = 0; k < SV; ++k) {
+            if constexpr (HAS_GAIN) {
+                const float4 g4 = __ldg(reinterpret_cast<const float4*>(a.gain) + v * SV + k);
+                w[i][4 * k + 0] = g4.x + a.gain_offset;
+                w[i][4 * k + 1] = g4.y + a.gain_offset;
+                w[i][4 * k + 2] = g4.z + a.gain_offset;
+                w[i][4 * k + 3] = g4.w + a.gain_offset;
+            }
+            if constexpr (t_is_residual(OP)) {
+                const float4 t4 = __ldg(reinterpret_cast<const float4*>(a.theta) + v * SV + k);
+                sincosf(t4.x, &sth[i][4 * k + 0], &cth[i][4 * k + 0]);
+                sincosf(t4.y, &sth[i][4 * k + 1], &cth[i][4 * k + 1]);
+                sincosf(t4.z, &sth[i][4 * k + 2], &cth[i][4 * k + 2]);
+                sincosf(t4.w, &sth[i][4 * k + 3], &cth[i][4 * k + 3]);
+            }
+        }
+    }
+    const float inv_width = 1.0f / (float)a.width;
+
+    // After a timed-out wait a warp stops touching the ring and the outputs but
+    // keeps joining the consumer barrier, so no other warp is left waiting.
+    bool alive = true;
+    int bank = 0;
+    for (int k = 0; k < n; ++k) {
+        const int s = k % S;
+        if (alive) alive = mbar_wait(&full_bar[s], (uint32_t)((k / S) & 1));
+        alive = __all_sync(0xffffffffu, alive);
+        const unsigned char* st = smem + (size_t)s * L.stage_bytes;
+        uint4 xv[VPT], gv[OP == RowOp::kNormGate ? VPT : 1], hv[t_is_residual(OP) ? VPT * SV : 1];
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int v = tid + i * ncons;
+            const bool rd = alive && valid[i];
+            xv[i] = rd ? reinterpret_cast<const uint4*>(st + L.x_off)[v] : make_uint4(0, 0, 0, 0);
+            if constexpr (OP == RowOp::kNormGate)
+                gv[i] = rd ? reinterpret_cast<const uint4*>(st + L.g_off)[v] : make_uint4(0, 0, 0, 0);
+            if constexpr (t_is_residual(OP)) {
+#pragma unroll
+                for (int q = 0; q < SV; ++q)
+                    hv[i * SV + q] = rd ? reinterpret_cast<const uint4*>(st + L.h_off)[v * SV + q]
+                                        : make_uint4(0, 0, 0, 0);
+            }
+        }
+        // this warp is done with the stage
+        __syncwarp();
+        if (lane == 0 && alive) mbar_arrive(&empty_bar[s]);
+
+        const int64_t row = r0 + k;
+        float xf[VPT][V];
+        float ss = 0.0f;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            unpack<T>(xv[i], xf[i]);
+            if constexpr (t_scales_first(OP) && HAS_GAIN) {
+#pragma unroll
+                for (int e = 0; e < V; ++e) xf[i][e] *= w[i][e];
+            }
+            ss += sum_sq<V>(xf[i]);
+        }
+        const float r = inv_rms_fast(consumer_sum(ss, red, bank, ncons), inv_width, a.eps);
+
+        if constexpr (OP == RowOp::kRms || OP == RowOp::kInputScale || OP == RowOp::kNormGate) {
+            char* yr = static_cast<char*>(a.y) + row * a.y_stride * (int64_t)sizeof(T);
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                float o[V];
+                float gf[V];
+                if constexpr (OP == RowOp::kNormGate) unpack<T>(gv[i], gf);
+#pragma unroll
+                for (int e = 0; e < V; ++e) {
+                    float t = xf[i][e] * r;
+                    if constexpr (OP == RowOp::kRms && HAS_GAIN) t = t * w[i][e];
+                    if constexpr (OP == RowOp::kNormGate) t = times_sigmoid<T>(t, gf[e]);
+                    o[e] = t;
+                }
+                if (alive && valid[i]) st_vec(yr + (int64_t)(tid + i * ncons) * 16, pack<T>(o));
+            }
+        } else {
+            char* hr = reinterpret_cast<char*>(a.stream_out + row * a.s_out_stride);
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                float hin[V];
+#pragma unroll
+                for (int q = 0; q < SV; ++q) unpack<float>(hv[i * SV + q], hin + 4 * q);
+                float o[V];
+#pragma unroll
+                for (int e = 0; e < V; ++e) {
+                    float t = xf[i][e] * r;  // z r when the gain came first
+                    if constexpr (OP == RowOp::kResidual && HAS_GAIN) t = t * w[i][e];
+                    const float nb = round_to<T>(t);  // cast back to the branch dtype
+                    o[e] = cth[i][e] * hin[e] + sth[i][e] * nb;
+                }
+                if (alive && valid[i]) {
+#pragma unroll
+                    for (int q = 0; q < SV; ++q)
+                        st_vec(hr + ((int64_t)(tid + i * ncons) * SV + q) * 16, pack<float>(o + 4 * q));
+                }
+            }
+        }
+    }
+}
+
+}  // namespace
+
+// Stage count and consumer threads per op; launch shape.
+template <typename T, RowOp OP, int VPT, bool G, int S>
+cudaError_t launch_row_tma_s(const RowArgs& a0, int nvec, cudaStream_t s) {
+    RowArgs a = a0;
+    const int ncons = ((nvec + VPT - 1) / VPT + 31) / 32 * 32;
+    const int threads = ncons + 32;
+    const StageLayout L = stage_layout<T, OP>(a.width);
+    const size_t smem = (size_t)S * L.stage_bytes;
+    auto kern = row_tma_kernel<T, OP, VPT, G, S>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int per_sm = blocks_per_sm((const void*)kern, threads, smem);
+    int64_t grid = (int64_t)per_sm * sm_count();
+    if (grid > a.rows) grid = a.rows;
+    if (grid < 1) grid = 1;
+    a.rows_per_cta = (int32_t)((a.rows + grid - 1) / grid);
+    grid = (a.rows + a.rows_per_cta - 1) / a.rows_per_cta;
+    kern<<<(unsigned)grid, threads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename T, RowOp OP, int VPT, bool G>
+cudaError_t launch_row_tma_v(const RowArgs& a, int nvec, int stages, cudaStream_t s) {
+    if (stages >= 3) return launch_row_tma_s<T, OP, VPT, G, 3>(a, nvec, s);
+    return launch_row_tma_s<T, OP, VPT, G, 2>(a, nvec, s);
+}
+
+// Launch shape, measured on B200 at prefill sizes (H = 4096): two or three
+// stages per CTA and as many CTAs per SM as fit beat deeper rings (3 to 4
+// CTAs of 256 consumers for 8 KB rows: 91% of the HBM copy bandwidth; 2 CTAs
+// for core 5's 24 KB rows: 93%).  Core 5 keeps at most 2 slots per consumer
+// thread (its 24 per-slot constants live in registers).
+constexpr uint32_t kRingMaxBytes = 200 * 1024;
+constexpr int kConsumers = 256;
+
+template <typename T, RowOp OP>
+cudaError_t launch_row_op(const RowArgs& a, cudaStream_t s) {
+    const int nvec = a.width / Vec<T>::N;
+    const StageLayout L = stage_layout<T, OP>(a.width);
+    const int dt = std::is_same<T, float>::value ? 1 : 0;
+    if (2 * L.stage_bytes > kRingMaxBytes) return launch_row_regs(dt, OP, a, s);
+    const int stages = L.stage_bytes >= 16 * 1024 ? 2 : 3;
+    const bool g = a.gain != nullptr;
+    // slots per consumer thread: the fewest that fit a row into kConsumers
+    // threads (core 5: at most 2 slots, up to twice the consumers)
+    if (nvec <= kConsumers)
+        return g ? launch_row_tma_v<T, OP, 1, true>(a, nvec, stages, s) : launch_row_tma_v<T, OP, 1, false>(a, nvec, stages, s);
+    if (nvec <= 2 * kConsumers || (t_is_residual(OP) && nvec <= 4 * kConsumers))
+        return g ? launch_row_tma_v<T, OP, 2, true>(a, nvec, stages, s) : launch_row_tma_v<T, OP, 2, false>(a, nvec, stages, s);
+    if constexpr (!t_is_residual(OP)) {
+        if (nvec <= 4 * kConsumers)
+            return g ? launch_row_tma_v<T, OP, 4, true>(a, nvec, stages, s) : launch_row_tma_v<T, OP, 4, false>(a, nvec, stages, s);
+    }
+    return launch_row_regs(dt, OP, a, s);
+}
+
+template <typename T>
+cudaError_t launch_row_t2(RowOp op, const RowArgs& a, cudaStream_t s) {
+    switch (op) {
+        case RowOp::kRms: return launch_row_op<T, RowOp::kRms>(a, s);
+        case RowOp::kInputScale: return launch_row_op<T, RowOp::kInputScale>(a, s);
+        case RowOp::kNormGate: return launch_row_op<T, RowOp::kNormGate>(a, s);
+        case RowOp::kResidual: return launch_row_op<T, RowOp::kResidual>(a, s);
+        case RowOp::kResidualIS: return launch_row_op<T, RowOp::kResidualIS>(a, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_row(int dtype, RowOp op, const RowArgs& a, cudaStream_t s) {
+    return dtype == 0 ? launch_row_t2<__nv_bfloat16>(op, a, s) : launch_row_t2<float>(op, a, s);
+}
+
+cudaError_t read_device_error(unsigned int* out, bool clear) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_device_error, sizeof(unsigned int));
+    if (e != cudaSuccess || !clear) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
+}
+
+}  // namespace muse

@@ -160,6 +160,17 @@ muse_status muse_norm_residual(const float* stream_in, const void* branch, float
                                int input_scale, float norm_eps, cudaStream_t stream);
 
 /*
+ * Device-side error word of the current device, for diagnostics.  The row
+ * kernels stream rows through shared memory with bulk copies tracked by
+ * mbarriers; every wait on one is bounded, and a wait that gives up sets bit 0
+ * of this word (and the affected kernel stops writing).  *flags receives the
+ * word; clear != 0 resets it.  Synchronous: it waits for the device.  Returns
+ * MUSE_ERR_INVALID_ARGUMENT for a NULL flags pointer, MUSE_ERR_CUDA if the
+ * copy fails.
+ */
+muse_status muse_device_error(unsigned int* flags, int clear);
+
+/*
  * Bandwidth reference (not a core): copy `bytes` bytes from src to dst with
  * 16-byte vector loads and stores over a persistent grid.  It measures the
  * HBM roofline on the same device the cores run on.  bytes % 16 == 0; both

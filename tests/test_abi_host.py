@@ -133,6 +133,7 @@ def test_gate_and_residual_validation(lib):
              1e-6, None) == INV
     assert r(A, A + (1 << 24), A + (2 << 24), BF16, 4, 252, None, 0.0, A + (3 << 24), 0, 1e-6,
              None) == UNS
+    assert lib.muse_device_error(None, 0) == INV
     c = lib.muse_stream_copy
     assert c(A, A + 4096, 0, None) == 0
     assert c(A, A + 4096, 8192, None) == INV            # overlapping ranges

@@ -88,3 +88,9 @@ def test_ambiguity_is_rare(cuda_ok):
         rows = harness.sample_rows(inputs.num_tokens(wl), 64)
         for st in _compare(wl, core, ci, rows, "ambig"):
             assert st["ambiguous"] <= max(10, 2e-3 * st["n"]), st
+
+
+def test_no_device_error_after_parity_runs(cuda_ok):
+    # every bounded mbarrier wait in the row kernels completed
+    from gate_cores_b200 import _lib
+    assert _lib.muse_device_error() == 0
