@@ -229,23 +229,23 @@ __device__ __forceinline__ void row_norm_body(const RowArgs& a) {
 
 // One entry symbol per core, so launch lists and profiles name the core.
 template <typename T, int VPT, bool G, int S, bool CSM>
-__global__ void __launch_bounds__(kMaxThreads) rms_norm_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(kMaxThreads) rms_norm_regs_kernel(const __grid_constant__ RowArgs a) {
     row_norm_body<T, RowOp::kRms, VPT, G, S, CSM>(a);
 }
 template <typename T, int VPT, bool G, int S, bool CSM>
-__global__ void __launch_bounds__(kMaxThreads) input_scale_norm_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(kMaxThreads) input_scale_norm_regs_kernel(const __grid_constant__ RowArgs a) {
     row_norm_body<T, RowOp::kInputScale, VPT, G, S, CSM>(a);
 }
 template <typename T, int VPT, bool G, int S, bool CSM>
-__global__ void __launch_bounds__(kMaxThreads) output_norm_gate_row_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(kMaxThreads) output_norm_gate_row_regs_kernel(const __grid_constant__ RowArgs a) {
     row_norm_body<T, RowOp::kNormGate, VPT, G, S, CSM>(a);
 }
 template <typename T, int VPT, bool G, int S, bool CSM>
-__global__ void __launch_bounds__(kMaxThreads) norm_residual_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(kMaxThreads) norm_residual_regs_kernel(const __grid_constant__ RowArgs a) {
     row_norm_body<T, RowOp::kResidual, VPT, G, S, CSM>(a);
 }
 template <typename T, int VPT, bool G, int S, bool CSM>
-__global__ void __launch_bounds__(kMaxThreads) norm_residual_input_scale_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(kMaxThreads) norm_residual_input_scale_regs_kernel(const __grid_constant__ RowArgs a) {
     row_norm_body<T, RowOp::kResidualIS, VPT, G, S, CSM>(a);
 }
 
@@ -264,11 +264,11 @@ template <typename T, RowOp OP, int VPT, bool G>
 constexpr auto row_kernel() {
     constexpr int S = stages<OP>();
     constexpr bool C = const_in_smem<OP>();
-    if constexpr (OP == RowOp::kRms) return rms_norm_kernel<T, VPT, G, S, C>;
-    else if constexpr (OP == RowOp::kInputScale) return input_scale_norm_kernel<T, VPT, G, S, C>;
-    else if constexpr (OP == RowOp::kNormGate) return output_norm_gate_row_kernel<T, VPT, G, S, C>;
-    else if constexpr (OP == RowOp::kResidual) return norm_residual_kernel<T, VPT, G, S, C>;
-    else return norm_residual_input_scale_kernel<T, VPT, G, S, C>;
+    if constexpr (OP == RowOp::kRms) return rms_norm_regs_kernel<T, VPT, G, S, C>;
+    else if constexpr (OP == RowOp::kInputScale) return input_scale_norm_regs_kernel<T, VPT, G, S, C>;
+    else if constexpr (OP == RowOp::kNormGate) return output_norm_gate_row_regs_kernel<T, VPT, G, S, C>;
+    else if constexpr (OP == RowOp::kResidual) return norm_residual_regs_kernel<T, VPT, G, S, C>;
+    else return norm_residual_input_scale_regs_kernel<T, VPT, G, S, C>;
 }
 
 template <typename T, RowOp OP, int VPT, bool G>
