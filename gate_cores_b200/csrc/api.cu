@@ -266,7 +266,7 @@ muse_status muse_qk_norm_rope(const void* q, const void* k, void* q_out, void* k
     a.hq = hq;
     a.hkv = hkv;
     a.head_dim = head_dim;
-    a.tile_tokens = 1;
+    a.split = 1;
     a.pos_mode = positions ? 0 : (layout == MUSE_LAYOUT_BSHD ? 1 : 2);
     a.eps = eps;
     a.query_scale = query_scale;

@@ -91,191 +91,153 @@ __device__ __forceinline__ int32_t token_position(const QkArgs& a, int64_t t) {
     return (int32_t)(t - __ldg(a.cu_seqlens + lo));
 }
 
-// Normalised, cast, optionally scaled and rotated 16-byte vector of one head.
-// cs/sn: cos/sin of this vector's Vec<T>::N / 2 pairs.
-template <typename T, bool ROPE, bool UPCAST>
-__device__ __forceinline__ uint4 qk_vec(const uint4& in, float r, bool scale, float qs,
-                                        const float* cs, const float* sn);
-
-template <bool ROPE, bool UPCAST>
-__device__ __forceinline__ uint32_t qk_pair_bf16(uint32_t w, f32x2 r2, bool scale, float qs, float c, float s) {
-    // cast of the normalised pair to bf16 (cvt.rn.bf16x2)
-    float n0, n1;
-    f2_split(f2_mul(f2_make(bf16_lo(w), bf16_hi(w)), r2), n0, n1);
-    uint32_t n = pack_bf16x2(n0, n1);
-    if (scale) n = pack_bf16x2(bf16_lo(n) * qs, bf16_hi(n) * qs);
-    if constexpr (!ROPE) {
-        return n;
+// Rotation of one normalised, cast pair (a, b) by (c, s).
+//   legacy / FP32 tensors: FP32 rotation (the caller casts once afterwards);
+//   v2 (bf16): each product rounded to bf16, then the sum, rounded by the caller.
+template <typename T, bool UPCAST>
+__device__ __forceinline__ f32x2 rope_pair(f32x2 n, float c, float s) {
+    float a, b;
+    f2_split(n, a, b);
+    if constexpr (UPCAST) {
+        return f2_make(a * c - b * s, a * s + b * c);
     } else {
-        const float x0 = bf16_lo(n), x1 = bf16_hi(n);
-        if constexpr (UPCAST) {
-            return pack_bf16x2(x0 * c - x1 * s, x0 * s + x1 * c);
-        } else {
-            // v2: each product rounded to bf16 before the sum, the sum cast again
-            const uint32_t p = pack_bf16x2(x0 * c, x1 * s);
-            const uint32_t q = pack_bf16x2(x0 * s, x1 * c);
-            return pack_bf16x2(bf16_lo(p) - bf16_hi(p), bf16_lo(q) + bf16_hi(q));
-        }
+        const uint32_t p = pack_bf16x2(a * c, b * s);
+        const uint32_t q = pack_bf16x2(a * s, b * c);
+        return f2_make(bf16_lo(p) - bf16_hi(p), bf16_lo(q) + bf16_hi(q));
     }
 }
 
-template <>
-__device__ __forceinline__ uint4 qk_vec<__nv_bfloat16, false, true>(const uint4& in, float r, bool scale, float qs,
-                                                                   const float*, const float*) {
-    const f32x2 r2 = f2_make(r, r);
-    return make_uint4(qk_pair_bf16<false, true>(in.x, r2, scale, qs, 0, 0),
-                      qk_pair_bf16<false, true>(in.y, r2, scale, qs, 0, 0),
-                      qk_pair_bf16<false, true>(in.z, r2, scale, qs, 0, 0),
-                      qk_pair_bf16<false, true>(in.w, r2, scale, qs, 0, 0));
-}
-template <>
-__device__ __forceinline__ uint4 qk_vec<__nv_bfloat16, true, true>(const uint4& in, float r, bool scale, float qs,
-                                                                  const float* c, const float* s) {
-    const f32x2 r2 = f2_make(r, r);
-    return make_uint4(qk_pair_bf16<true, true>(in.x, r2, scale, qs, c[0], s[0]),
-                      qk_pair_bf16<true, true>(in.y, r2, scale, qs, c[1], s[1]),
-                      qk_pair_bf16<true, true>(in.z, r2, scale, qs, c[2], s[2]),
-                      qk_pair_bf16<true, true>(in.w, r2, scale, qs, c[3], s[3]));
-}
-template <>
-__device__ __forceinline__ uint4 qk_vec<__nv_bfloat16, true, false>(const uint4& in, float r, bool scale, float qs,
-                                                                   const float* c, const float* s) {
-    const f32x2 r2 = f2_make(r, r);
-    return make_uint4(qk_pair_bf16<true, false>(in.x, r2, scale, qs, c[0], s[0]),
-                      qk_pair_bf16<true, false>(in.y, r2, scale, qs, c[1], s[1]),
-                      qk_pair_bf16<true, false>(in.z, r2, scale, qs, c[2], s[2]),
-                      qk_pair_bf16<true, false>(in.w, r2, scale, qs, c[3], s[3]));
-}
-// FP32 tensors: the casts are exact and the rotation is FP32 in both modes.
-template <bool ROPE>
-__device__ __forceinline__ uint4 qk_vec_f32(const uint4& in, float r, bool scale, float qs,
-                                            const float* c, const float* s) {
-    float f[4];
-    unpack<float>(in, f);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        f[e] = f[e] * r;
-        if (scale) f[e] = f[e] * qs;
-    }
-    if constexpr (ROPE) {
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const float x0 = f[2 * j], x1 = f[2 * j + 1];
-            f[2 * j] = x0 * c[j] - x1 * s[j];
-            f[2 * j + 1] = x0 * s[j] + x1 * c[j];
-        }
-    }
-    return pack<float>(f);
-}
-template <>
-__device__ __forceinline__ uint4 qk_vec<float, false, true>(const uint4& in, float r, bool scale, float qs,
-                                                           const float* c, const float* s) {
-    return qk_vec_f32<false>(in, r, scale, qs, c, s);
-}
-template <>
-__device__ __forceinline__ uint4 qk_vec<float, true, true>(const uint4& in, float r, bool scale, float qs,
-                                                          const float* c, const float* s) {
-    return qk_vec_f32<true>(in, r, scale, qs, c, s);
-}
-
-// One CTA per tile of tile_tokens consecutive tokens.  The CTA first fills a
-// shared table with cos/sin of every (token, pair) angle - one sincosf per pair
-// per token - then its warps walk the tile's (token, head step) units, CH
-// units at a time with all their loads in flight.  Head steps cover query
-// heads first, then key heads.
-template <typename T, int L, int VPL, bool ROPE, bool UPCAST, int CH>
+// One CTA per tile of tokens; each warp owns one token (or, with split > 1,
+// one of `split` ranges of that token's head steps).  The CTA first fills a
+// shared table with cos/sin of every (token, pair) angle of the tile - one
+// sincosf per pair per token - and each lane then keeps the cos/sin of its own
+// VPL vectors in registers: a lane covers the same element positions of every
+// head, so the values serve all heads of the token.  The token's query heads
+// and then its key heads are walked in steps of RW heads, BATCH steps at a
+// time with all their loads in flight; element arithmetic runs on packed FP32
+// pairs and each pair is unpacked once.
+template <typename T, int L, int VPL, bool ROPE, bool UPCAST, int BATCH>
 __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant__ QkArgs a) {
     constexpr int V = Vec<T>::N;
-    constexpr int P = V / 2;  // rotation pairs per vector
+    constexpr int P = V / 2;  // pairs per vector
     constexpr int RW = 32 / L;
-    extern __shared__ float table[];  // [cos | sin][tile_tokens][head_dim / 2]
+    extern __shared__ float table[];  // [cos | sin][tile tokens][head_dim / 2]
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int nwarps = blockDim.x >> 5;
+    const int split = a.split;
+    const int tt = nwarps / split;  // tokens per tile
     const int sub = lane % L;
     const int slot = lane / L;
     const int nvec = a.head_dim / V;
-    const float inv_width = 1.0f / (float)a.head_dim;
     const int half = a.head_dim / 2;
-    const int tt = a.tile_tokens;
-    const int nh = a.hq + a.hkv;
-    const int nsteps = (nh + RW - 1) / RW;
-    const bool scale_q = a.query_scale != 1.0f;
+    const float inv_width = 1.0f / (float)a.head_dim;
     const int64_t t0 = (int64_t)blockIdx.x * tt;
     const int ntok = (int)min((int64_t)tt, a.tokens - t0);
     float* cs = table;
     float* sn = table + tt * half;
 
     if constexpr (ROPE) {
-        for (int i = threadIdx.x; i < ntok * half; i += blockDim.x) {
-            const int k = i / half;
+        for (int k = warp; k < ntok; k += nwarps) {
             const float pos = (float)token_position(a, t0 + k);
-            const float phi = pos * a.inv_freq[i - k * half];  // one FP32 rounding
-            float sv, cv;
-            sincosf(phi, &sv, &cv);
-            if constexpr (!UPCAST) {
-                cv = round_to<T>(cv);
-                sv = round_to<T>(sv);
+            for (int p = lane; p < half; p += 32) {
+                const float phi = pos * a.inv_freq[p];  // one FP32 rounding
+                float sv, cv;
+                sincosf(phi, &sv, &cv);
+                if constexpr (!UPCAST) {
+                    cv = round_to<T>(cv);
+                    sv = round_to<T>(sv);
+                }
+                cs[k * half + p] = cv;
+                sn[k * half + p] = sv;
             }
-            cs[i] = cv;
-            sn[i] = sv;
         }
         __syncthreads();
     }
-    const int units = ntok * nsteps;
-    for (int u0 = warp * CH; u0 < units; u0 += nwarps * CH) {
-        uint4 xv[CH][VPL];
-        int tok[CH], head[CH];
-        bool ok[CH][VPL];
+    const int tok = warp / split;
+    if (tok >= ntok) return;
+    const int part = warp - tok * split;
+    const int64_t t = t0 + tok;
+
+    // this lane's vectors of a head: sub, sub + L, ...
+    bool vok[VPL];
+    uint32_t voff[VPL];
+    float cv[VPL][P], sv[VPL][P];
 #pragma unroll
-        for (int c = 0; c < CH; ++c) {
-            const int u = u0 + c;
-            tok[c] = u / nsteps;
-            head[c] = (u - tok[c] * nsteps) * RW + slot;
-            const bool hv = u < units && head[c] < nh;
-            const int64_t t = t0 + tok[c];
-            const char* src = head[c] < a.hq
-                ? static_cast<const char*>(a.q) + (t * a.q_stride + (int64_t)head[c] * a.head_dim) * (int64_t)sizeof(T)
-                : static_cast<const char*>(a.k) + (t * a.k_stride + (int64_t)(head[c] - a.hq) * a.head_dim) * (int64_t)sizeof(T);
+    for (int k = 0; k < VPL; ++k) {
+        const int vi = sub + k * L;
+        vok[k] = vi < nvec;
+        voff[k] = (uint32_t)vi * 16u;
+        if constexpr (ROPE) {
+            const int tb = tok * half + (vok[k] ? vi * P : 0);
 #pragma unroll
-            for (int k = 0; k < VPL; ++k) {
-                const int vi = sub + k * L;
-                ok[c][k] = hv && vi < nvec;
-                xv[c][k] = ok[c][k] ? ld_stream(src + (int64_t)vi * 16) : make_uint4(0, 0, 0, 0);
+            for (int j = 0; j < P; ++j) {
+                cv[k][j] = cs[tb + j];
+                sv[k][j] = sn[tb + j];
             }
         }
+    }
+    const uint32_t head_bytes = (uint32_t)a.head_dim * sizeof(T);
+    const f32x2 qs2 = f2_make(a.query_scale, a.query_scale);
+    const int nst_q = (a.hq + RW - 1) / RW;
+    const int nst = nst_q + (a.hkv + RW - 1) / RW;
+    const int spw = (nst + split - 1) / split;
+    const int g_begin = part * spw, g_end = min(nst, g_begin + spw);
+
+    // segment 0: query heads, segment 1: key heads
+#pragma unroll 1
+    for (int seg = 0; seg < 2; ++seg) {
+        const int s_lo = max(g_begin, seg == 0 ? 0 : nst_q) - (seg == 0 ? 0 : nst_q);
+        const int s_hi = min(g_end, seg == 0 ? nst_q : nst) - (seg == 0 ? 0 : nst_q);
+        if (s_lo >= s_hi) continue;
+        const int count = seg == 0 ? a.hq : a.hkv;
+        const bool scale = seg == 0 && a.query_scale != 1.0f;
+        const char* src = seg == 0 ? static_cast<const char*>(a.q) + t * a.q_stride * (int64_t)sizeof(T)
+                                   : static_cast<const char*>(a.k) + t * a.k_stride * (int64_t)sizeof(T);
+        char* dst = seg == 0 ? static_cast<char*>(a.q_out) + t * a.q_out_stride * (int64_t)sizeof(T)
+                             : static_cast<char*>(a.k_out) + t * a.k_out_stride * (int64_t)sizeof(T);
+        for (int st0 = s_lo; st0 < s_hi; st0 += BATCH) {
+            uint4 xv[BATCH][VPL];
+            bool hv[BATCH];
 #pragma unroll
-        for (int c = 0; c < CH; ++c) {
-            float ss = 0.0f;
+            for (int b = 0; b < BATCH; ++b) {
+                const int head = (st0 + b) * RW + slot;
+                hv[b] = st0 + b < s_hi && head < count;
+                const char* hs = src + (uint32_t)head * head_bytes;
 #pragma unroll
-            for (int k = 0; k < VPL; ++k) ss += vec_sum_sq<T>(xv[c][k]);
-            const float r = inv_rms_fast(group_sum<L>(ss), inv_width, a.eps);
-            const bool is_q = head[c] < a.hq;
-            const int64_t t = t0 + tok[c];
-            char* dst = is_q
-                ? static_cast<char*>(a.q_out) + (t * a.q_out_stride + (int64_t)head[c] * a.head_dim) * (int64_t)sizeof(T)
-                : static_cast<char*>(a.k_out) + (t * a.k_out_stride + (int64_t)(head[c] - a.hq) * a.head_dim) * (int64_t)sizeof(T);
+                for (int k = 0; k < VPL; ++k)
+                    xv[b][k] = (hv[b] && vok[k]) ? ld_stream(hs + voff[k]) : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
-            for (int k = 0; k < VPL; ++k) {
-                const int vi = sub + k * L;
-                // this vector's cos/sin (table row 0 for idle lanes and units)
-                const int tb = ok[c][k] ? tok[c] * half + vi * P : 0;
-                float cv[P], sv[P];
-                if constexpr (ROPE) {
+            for (int b = 0; b < BATCH; ++b) {
+                f32x2 x[VPL][P];
+                f32x2 acc = f2_make(0.0f, 0.0f);
 #pragma unroll
-                    for (int j = 0; j < P; ++j) {
-                        cv[j] = cs[tb + j];
-                        sv[j] = sn[tb + j];
-                    }
+                for (int k = 0; k < VPL; ++k) {
+                    to_pairs<T>(xv[b][k], x[k]);
+#pragma unroll
+                    for (int q = 0; q < P; ++q) acc = f2_fma(x[k][q], x[k][q], acc);
                 }
-                const uint4 y = qk_vec<T, ROPE, UPCAST>(xv[c][k], r, is_q && scale_q, a.query_scale, cv, sv);
-                if (ok[c][k]) st_vec(dst + (int64_t)vi * 16, y);
+                const float r = inv_rms_fast(group_sum<L>(f2_sum(acc)), inv_width, a.eps);
+                const f32x2 r2 = f2_make(r, r);
+                const int head = (st0 + b) * RW + slot;
+                char* hd = dst + (uint32_t)head * head_bytes;
+#pragma unroll
+                for (int k = 0; k < VPL; ++k) {
+                    f32x2 y[P];
+#pragma unroll
+                    for (int q = 0; q < P; ++q) {
+                        f32x2 n = round_pair<T>(f2_mul(x[k][q], r2));     // cast to the Q/K dtype
+                        if (scale) n = round_pair<T>(f2_mul(n, qs2));     // query_scale, cast again
+                        if constexpr (ROPE) n = rope_pair<T, UPCAST>(n, cv[k][q], sv[k][q]);
+                        y[q] = n;
+                    }
+                    if (hv[b] && vok[k]) st_vec(hd + voff[k], from_pairs<T>(y));
+                }
             }
         }
     }
 }
-
-int gcd(int x, int y) { return y == 0 ? x : gcd(y, x % y); }
 
 constexpr int kThreads = 256;
 
@@ -309,19 +271,19 @@ cudaError_t launch_head_gate_t(const HeadGateArgs& a, cudaStream_t s) {
 template <typename T, int L, int VPL, bool ROPE, bool UPCAST>
 cudaError_t launch_qk_l(const QkArgs& a0, cudaStream_t s) {
     constexpr int RW = 32 / L;
-    constexpr int CH = 2;
+    constexpr int BATCH = 4;
     QkArgs a = a0;
+    const int nwarps = kThreads / 32;
     const int nsteps = (a.hq + a.hkv + RW - 1) / RW;
-    // Tile: enough tokens that the tile's units fill every warp's CH-unit
-    // rounds exactly, shrunk while the grid would leave SMs without a CTA.
-    const int per_round = (kThreads / 32) * CH;
-    int tt = per_round / gcd(nsteps, per_round);
-    if (tt > kMaxTileTokens) tt = kMaxTileTokens;
-    while (tt > 1 && (a.tokens + tt - 1) / tt < 2 * sm_count()) tt /= 2;
-    a.tile_tokens = tt;
+    // Split a token's head steps over up to 8 warps while the grid would
+    // leave SMs idle (decode-sized batches).
+    int split = 1;
+    while (split < nwarps && split < nsteps && (a.tokens * split + nwarps - 1) / nwarps < 2 * sm_count()) split *= 2;
+    a.split = split;
+    const int tt = nwarps / split;
     const size_t smem = ROPE ? sizeof(float) * 2 * tt * (a.head_dim / 2) : 0;
     const int64_t grid = (a.tokens + tt - 1) / tt;
-    qk_norm_rope_kernel<T, L, VPL, ROPE, UPCAST, CH><<<(unsigned)grid, kThreads, smem, s>>>(a);
+    qk_norm_rope_kernel<T, L, VPL, ROPE, UPCAST, BATCH><<<(unsigned)grid, kThreads, smem, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -336,13 +298,11 @@ cudaError_t launch_qk_modes(int use_rope, int upcast, const QkArgs& a, cudaStrea
 
 template <typename T>
 cudaError_t launch_qk_t(int use_rope, int upcast, const QkArgs& a, cudaStream_t s) {
+    // one 16-byte vector per lane per head (measured best at head_dim 128);
+    // two for heads of more than 32 vectors
     const int nv = a.head_dim / Vec<T>::N;
-    if (nv >= 16) {
-        const int lanes = (nv + 1) / 2;
-        if (lanes <= 8) return launch_qk_modes<T, 8, 2>(use_rope, upcast, a, s);
-        if (lanes <= 16) return launch_qk_modes<T, 16, 2>(use_rope, upcast, a, s);
-        return launch_qk_modes<T, 32, 2>(use_rope, upcast, a, s);
-    }
+    if (nv > 32) return launch_qk_modes<T, 32, 2>(use_rope, upcast, a, s);
+    if (nv > 16) return launch_qk_modes<T, 32, 1>(use_rope, upcast, a, s);
     if (nv <= 1) return launch_qk_modes<T, 1, 1>(use_rope, upcast, a, s);
     if (nv <= 2) return launch_qk_modes<T, 2, 1>(use_rope, upcast, a, s);
     if (nv <= 4) return launch_qk_modes<T, 4, 1>(use_rope, upcast, a, s);

@@ -44,7 +44,6 @@ struct HeadGateArgs {
 };
 
 constexpr int kMaxHalfDim = 128;  // head_dim <= 256
-constexpr int kMaxTileTokens = 16;  // 2 x 2 x 16 x 128 floats = 32 KB of cos/sin table
 
 struct QkArgs {
     const void* q;
@@ -58,7 +57,7 @@ struct QkArgs {
     int64_t q_stride, k_stride, q_out_stride, k_out_stride;  // elements per token
     int32_t num_seqs;
     int32_t hq, hkv, head_dim;
-    int32_t tile_tokens;        // tokens per CTA tile (<= kMaxTileTokens)
+    int32_t split;              // warps sharing one token's head steps (1, 2, 4, 8)
     int32_t pos_mode;           // 0 explicit, 1 BSHD derived, 2 THD derived
     float eps;
     float query_scale;

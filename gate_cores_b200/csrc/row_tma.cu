@@ -175,118 +175,146 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
     }
 
     // ---------------- consumer warps
+    // Element arithmetic on packed FP32 pairs (f32x2: two IEEE round-to-nearest
+    // operations per instruction); offsets and the stage walk are incremental.
+    constexpr int P = V / 2;
     bool valid[VPT];
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) valid[i] = tid + i * ncons < nvec;
-
-    // per-slot constants in registers (the pipeline, not registers, holds the
-    // rows in flight)
-    float w[HAS_GAIN ? VPT : 1][V];
-    float cth[t_is_residual(OP) ? VPT : 1][V];
-    float sth[t_is_residual(OP) ? VPT : 1][V];
+    uint32_t voff[VPT];  // this thread's byte offset of slot i within a row
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
-        const int v = valid[i] ? tid + i * ncons : 0;
+        valid[i] = tid + i * ncons < nvec;
+        voff[i] = (uint32_t)(tid + i * ncons) * 16u;
+    }
+
+    // per-slot constants in registers (the pipeline, not registers, holds the
+    // rows in flight): effective gain, cos and sin of the blend angle
+    f32x2 w[HAS_GAIN ? VPT : 1][P];
+    f32x2 cth[t_is_residual(OP) ? VPT : 1][P];
+    f32x2 sth[t_is_residual(OP) ? VPT : 1][P];
+    {
+        const f32x2 off2 = f2_make(a.gain_offset, a.gain_offset);
 #pragma unroll
-        for (int k = 0; k < SV; ++k) {
-            if constexpr (HAS_GAIN) {
-                const float4 g4 = __ldg(reinterpret_cast<const float4*>(a.gain) + v * SV + k);
-                w[i][4 * k + 0] = g4.x + a.gain_offset;
-                w[i][4 * k + 1] = g4.y + a.gain_offset;
-                w[i][4 * k + 2] = g4.z + a.gain_offset;
-                w[i][4 * k + 3] = g4.w + a.gain_offset;
-            }
-            if constexpr (t_is_residual(OP)) {
-                const float4 t4 = __ldg(reinterpret_cast<const float4*>(a.theta) + v * SV + k);
-                sincosf(t4.x, &sth[i][4 * k + 0], &cth[i][4 * k + 0]);
-                sincosf(t4.y, &sth[i][4 * k + 1], &cth[i][4 * k + 1]);
-                sincosf(t4.z, &sth[i][4 * k + 2], &cth[i][4 * k + 2]);
-                sincosf(t4.w, &sth[i][4 * k + 3], &cth[i][4 * k + 3]);
+        for (int i = 0; i < VPT; ++i) {
+            const int v = valid[i] ? tid + i * ncons : 0;
+#pragma unroll
+            for (int k = 0; k < SV; ++k) {
+                if constexpr (HAS_GAIN) {
+                    const float4 g4 = __ldg(reinterpret_cast<const float4*>(a.gain) + v * SV + k);
+                    w[i][2 * k] = f2_add(f2_make(g4.x, g4.y), off2);  // FP32 sums
+                    w[i][2 * k + 1] = f2_add(f2_make(g4.z, g4.w), off2);
+                }
+                if constexpr (t_is_residual(OP)) {
+                    const float4 t4 = __ldg(reinterpret_cast<const float4*>(a.theta) + v * SV + k);
+                    float s0, c0, s1, c1, s2, c2, s3, c3;
+                    sincosf(t4.x, &s0, &c0);
+                    sincosf(t4.y, &s1, &c1);
+                    sincosf(t4.z, &s2, &c2);
+                    sincosf(t4.w, &s3, &c3);
+                    cth[i][2 * k] = f2_make(c0, c1);
+                    cth[i][2 * k + 1] = f2_make(c2, c3);
+                    sth[i][2 * k] = f2_make(s0, s1);
+                    sth[i][2 * k + 1] = f2_make(s2, s3);
+                }
             }
         }
     }
     const float inv_width = 1.0f / (float)a.width;
 
+    // output row pointer, advanced one row per iteration
+    char* out_row = t_is_residual(OP)
+        ? reinterpret_cast<char*>(a.stream_out + r0 * a.s_out_stride)
+        : static_cast<char*>(a.y) + r0 * a.y_stride * (int64_t)sizeof(T);
+    const int64_t out_step = t_is_residual(OP) ? a.s_out_stride * (int64_t)sizeof(float)
+                                               : a.y_stride * (int64_t)sizeof(T);
+
     // After a timed-out wait a warp stops touching the ring and the outputs but
     // keeps joining the consumer barrier, so no other warp is left waiting.
     bool alive = true;
     int bank = 0;
+    int s = 0;
+    uint32_t phase = 0;
     for (int k = 0; k < n; ++k) {
-        const int s = k % S;
-        if (alive) alive = mbar_wait(&full_bar[s], (uint32_t)((k / S) & 1));
+        if (alive) alive = mbar_wait(&full_bar[s], phase);
         alive = __all_sync(0xffffffffu, alive);
-        const unsigned char* st = smem + (size_t)s * L.stage_bytes;
+        const unsigned char* st = smem + s * L.stage_bytes;
         uint4 xv[VPT], gv[OP == RowOp::kNormGate ? VPT : 1], hv[t_is_residual(OP) ? VPT * SV : 1];
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
-            const int v = tid + i * ncons;
             const bool rd = alive && valid[i];
-            xv[i] = rd ? reinterpret_cast<const uint4*>(st + L.x_off)[v] : make_uint4(0, 0, 0, 0);
+            xv[i] = rd ? *reinterpret_cast<const uint4*>(st + L.x_off + voff[i]) : make_uint4(0, 0, 0, 0);
             if constexpr (OP == RowOp::kNormGate)
-                gv[i] = rd ? reinterpret_cast<const uint4*>(st + L.g_off)[v] : make_uint4(0, 0, 0, 0);
+                gv[i] = rd ? *reinterpret_cast<const uint4*>(st + L.g_off + voff[i]) : make_uint4(0, 0, 0, 0);
             if constexpr (t_is_residual(OP)) {
 #pragma unroll
                 for (int q = 0; q < SV; ++q)
-                    hv[i * SV + q] = rd ? reinterpret_cast<const uint4*>(st + L.h_off)[v * SV + q]
+                    hv[i * SV + q] = rd ? *reinterpret_cast<const uint4*>(st + L.h_off + voff[i] * SV + 16u * q)
                                         : make_uint4(0, 0, 0, 0);
             }
         }
         // this warp is done with the stage
         __syncwarp();
         if (lane == 0 && alive) mbar_arrive(&empty_bar[s]);
+        if (++s == S) {
+            s = 0;
+            phase ^= 1u;
+        }
 
-        const int64_t row = r0 + k;
-        float xf[VPT][V];
-        float ss = 0.0f;
+        f32x2 x[VPT][P];
+        f32x2 acc[2] = {f2_make(0.0f, 0.0f), f2_make(0.0f, 0.0f)};  // 4 partial sums
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
-            unpack<T>(xv[i], xf[i]);
-            if constexpr (t_scales_first(OP) && HAS_GAIN) {
+            to_pairs<T>(xv[i], x[i]);
 #pragma unroll
-                for (int e = 0; e < V; ++e) xf[i][e] *= w[i][e];
+            for (int q = 0; q < P; ++q) {
+                if constexpr (t_scales_first(OP) && HAS_GAIN) x[i][q] = f2_mul(x[i][q], w[i][q]);
+                acc[q & 1] = f2_fma(x[i][q], x[i][q], acc[q & 1]);
             }
-            ss += sum_sq<V>(xf[i]);
         }
-        const float r = inv_rms_fast(consumer_sum(ss, red, bank, ncons), inv_width, a.eps);
+        const float part = f2_sum(acc[0]) + f2_sum(acc[1]);
+        const float r = inv_rms_fast(consumer_sum(part, red, bank, ncons), inv_width, a.eps);
+        const f32x2 r2 = f2_make(r, r);
 
         if constexpr (OP == RowOp::kRms || OP == RowOp::kInputScale || OP == RowOp::kNormGate) {
-            char* yr = static_cast<char*>(a.y) + row * a.y_stride * (int64_t)sizeof(T);
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
-                float o[V];
-                float gf[V];
-                if constexpr (OP == RowOp::kNormGate) unpack<T>(gv[i], gf);
+                f32x2 o[P];
 #pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    float t = xf[i][e] * r;
-                    if constexpr (OP == RowOp::kRms && HAS_GAIN) t = t * w[i][e];
-                    if constexpr (OP == RowOp::kNormGate) t = times_sigmoid<T>(t, gf[e]);
-                    o[e] = t;
+                for (int q = 0; q < P; ++q) {
+                    o[q] = f2_mul(x[i][q], r2);
+                    if constexpr (OP == RowOp::kRms && HAS_GAIN) o[q] = f2_mul(o[q], w[i][q]);
                 }
-                if (alive && valid[i]) st_vec(yr + (int64_t)(tid + i * ncons) * 16, pack<T>(o));
+                if constexpr (OP == RowOp::kNormGate) {
+                    float gf[V];
+                    unpack<T>(gv[i], gf);
+#pragma unroll
+                    for (int q = 0; q < P; ++q) {
+                        float lo, hi;
+                        f2_split(o[q], lo, hi);
+                        o[q] = f2_make(times_sigmoid<T>(lo, gf[2 * q]), times_sigmoid<T>(hi, gf[2 * q + 1]));
+                    }
+                }
+                if (alive && valid[i]) st_vec(out_row + voff[i], from_pairs<T>(o));
             }
         } else {
-            char* hr = reinterpret_cast<char*>(a.stream_out + row * a.s_out_stride);
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
-                float hin[V];
+                f32x2 h[P], o[P];
 #pragma unroll
-                for (int q = 0; q < SV; ++q) unpack<float>(hv[i * SV + q], hin + 4 * q);
-                float o[V];
+                for (int q = 0; q < SV; ++q) to_pairs<float>(hv[i * SV + q], h + 2 * q);
 #pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    float t = xf[i][e] * r;  // z r when the gain came first
-                    if constexpr (OP == RowOp::kResidual && HAS_GAIN) t = t * w[i][e];
-                    const float nb = round_to<T>(t);  // cast back to the branch dtype
-                    o[e] = cth[i][e] * hin[e] + sth[i][e] * nb;
+                for (int q = 0; q < P; ++q) {
+                    f32x2 t = f2_mul(x[i][q], r2);  // z r when the gain came first
+                    if constexpr (OP == RowOp::kResidual && HAS_GAIN) t = f2_mul(t, w[i][q]);
+                    const f32x2 nb = round_pair<T>(t);  // cast back to the branch dtype
+                    o[q] = f2_fma(cth[i][q], h[q], f2_mul(sth[i][q], nb));
                 }
                 if (alive && valid[i]) {
 #pragma unroll
-                    for (int q = 0; q < SV; ++q)
-                        st_vec(hr + ((int64_t)(tid + i * ncons) * SV + q) * 16, pack<float>(o + 4 * q));
+                    for (int q = 0; q < SV; ++q) st_vec(out_row + voff[i] * SV + 16u * q, from_pairs<float>(o + 2 * q));
                 }
             }
         }
+        out_row += out_step;
     }
 }
 
