@@ -39,7 +39,7 @@ CORE_ORDER = inputs.CORES
 METRIC = "tokens/s and effective HBM GB/s per fused core vs measured ~8 TB/s peak"
 DOMINANT = "norm_residual"  # largest algorithmic byte count of the five
 # sources whose change invalidates the committed dram-traffic figure of the dominant kernel
-DOMINANT_SOURCES = ("row_tma.cu", "common.cuh", "kernels.h")
+DOMINANT_SOURCES = ("row_tma.cu", "tma_pipe.cuh", "common.cuh", "kernels.h")
 KERNEL_NAMES = {c: c + "_kernel" for c in inputs.CORES}
 VARIANT = {"rms_norm": "zero-centered gain (offset 1)", "input_scale_norm": "gain U(0.5,1.5)",
            "qk_norm_rope": "RoPE in FP32 (legacy), query_scale 1, BSHD-derived positions",

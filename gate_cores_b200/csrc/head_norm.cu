@@ -10,20 +10,14 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "qk_common.cuh"
 
 namespace muse {
 namespace {
 
-// Sum of squares of one 16-byte vector (two packed partial sums).
-template <typename T> __device__ __forceinline__ float vec_sum_sq(const uint4& v) {
-    constexpr int P = Vec<T>::N / 2;
-    f32x2 p[P];
-    to_pairs<T>(v, p);
-    f32x2 acc = f2_mul(p[0], p[0]);
-#pragma unroll
-    for (int k = 1; k < P; ++k) acc = f2_fma(p[k], p[k], acc);
-    return f2_sum(acc);
-}
+using qk::rope_pair;
+using qk::token_position;
+using qk::vec_sum_sq;
 
 // ------------------------------------------------------------ core 4 per head
 
@@ -78,35 +72,6 @@ __global__ void __launch_bounds__(256) output_norm_gate_kernel(const __grid_cons
 
 // ------------------------------------------------------------------ core 3
 
-__device__ __forceinline__ int32_t token_position(const QkArgs& a, int64_t t) {
-    if (a.pos_mode == 0) return __ldg(a.positions + t);
-    if (a.pos_mode == 1) return (int32_t)(t % a.seqlen);
-    // THD: the document d with cu[d] <= t < cu[d+1]; every index read lies in
-    // [0, num_seqs - 1], whatever the array holds.
-    int lo = 0, hi = a.num_seqs;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if ((int64_t)__ldg(a.cu_seqlens + mid) <= t) lo = mid; else hi = mid;
-    }
-    return (int32_t)(t - __ldg(a.cu_seqlens + lo));
-}
-
-// Rotation of one normalised, cast pair (a, b) by (c, s).
-//   legacy / FP32 tensors: FP32 rotation (the caller casts once afterwards);
-//   v2 (bf16): each product rounded to bf16, then the sum, rounded by the caller.
-template <typename T, bool UPCAST>
-__device__ __forceinline__ f32x2 rope_pair(f32x2 n, float c, float s) {
-    float a, b;
-    f2_split(n, a, b);
-    if constexpr (UPCAST) {
-        return f2_make(a * c - b * s, a * s + b * c);
-    } else {
-        const uint32_t p = pack_bf16x2(a * c, b * s);
-        const uint32_t q = pack_bf16x2(a * s, b * c);
-        return f2_make(bf16_lo(p) - bf16_hi(p), bf16_lo(q) + bf16_hi(q));
-    }
-}
-
 // One CTA per tile of tokens; each warp owns one token (or, with split > 1,
 // one of `split` ranges of that token's head steps).  The CTA first fills a
 // shared table with cos/sin of every (token, pair) angle of the tile - one
@@ -116,8 +81,8 @@ __device__ __forceinline__ f32x2 rope_pair(f32x2 n, float c, float s) {
 // and then its key heads are walked in steps of RW heads, BATCH steps at a
 // time with all their loads in flight; element arithmetic runs on packed FP32
 // pairs and each pair is unpacked once.
-template <typename T, int L, int VPL, bool ROPE, bool UPCAST, int BATCH>
-__global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant__ QkArgs a) {
+template <typename T, int L, int VPL, bool ROPE, bool UPCAST, int BATCH, int MINB>
+__global__ void __launch_bounds__(256, MINB) qk_norm_rope_kernel(const __grid_constant__ QkArgs a) {
     constexpr int V = Vec<T>::N;
     constexpr int P = V / 2;  // pairs per vector
     constexpr int RW = 32 / L;
@@ -240,6 +205,10 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant
 }
 
 constexpr int kThreads = 256;
+// Resident CTAs per SM the Q/K kernel's registers are sized for: 4 (32 warps)
+// keeps enough loads in flight to cover HBM latency (measured: 2 resident
+// CTAs reach about 2/3 of the copy bandwidth, 4 about 9/10).
+constexpr int kQkMinBlocks = 4;
 
 template <typename T, int L, int VPL, int CH>
 cudaError_t launch_head_gate_l(const HeadGateArgs& a, cudaStream_t s) {
@@ -283,7 +252,7 @@ cudaError_t launch_qk_l(const QkArgs& a0, cudaStream_t s) {
     const int tt = nwarps / split;
     const size_t smem = ROPE ? sizeof(float) * 2 * tt * (a.head_dim / 2) : 0;
     const int64_t grid = (a.tokens + tt - 1) / tt;
-    qk_norm_rope_kernel<T, L, VPL, ROPE, UPCAST, BATCH><<<(unsigned)grid, kThreads, smem, s>>>(a);
+    qk_norm_rope_kernel<T, L, VPL, ROPE, UPCAST, BATCH, kQkMinBlocks><<<(unsigned)grid, kThreads, smem, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -301,7 +270,6 @@ cudaError_t launch_qk_t(int use_rope, int upcast, const QkArgs& a, cudaStream_t 
     // one 16-byte vector per lane per head (measured best at head_dim 128);
     // two for heads of more than 32 vectors
     const int nv = a.head_dim / Vec<T>::N;
-    if (nv > 32) return launch_qk_modes<T, 32, 2>(use_rope, upcast, a, s);
     if (nv > 16) return launch_qk_modes<T, 32, 1>(use_rope, upcast, a, s);
     if (nv <= 1) return launch_qk_modes<T, 1, 1>(use_rope, upcast, a, s);
     if (nv <= 2) return launch_qk_modes<T, 2, 1>(use_rope, upcast, a, s);

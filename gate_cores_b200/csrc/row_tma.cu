@@ -23,67 +23,17 @@ namespace muse {
 
 __device__ unsigned int g_device_error;  // bit 0: an mbarrier wait timed out
 
+}  // namespace muse
+
+#include "tma_pipe.cuh"
+
+namespace muse {
 namespace {
 
-constexpr uint32_t kSpinLimit = 1u << 24;
+using namespace pipe;
 
 __host__ __device__ constexpr bool t_is_residual(RowOp op) { return op == RowOp::kResidual || op == RowOp::kResidualIS; }
 __host__ __device__ constexpr bool t_scales_first(RowOp op) { return op == RowOp::kInputScale || op == RowOp::kResidualIS; }
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    return done != 0;
-}
-// Bounded wait for the phase of the given parity; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    atomicOr(&g_device_error, 1u);
-    return false;
-}
-// Bulk copy global -> shared, completing `bytes` on the mbarrier.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
-        : "memory");
-}
-// Barrier among the consumer threads only (named barrier 1).
-__device__ __forceinline__ void consumer_sync(int nthreads) {
-    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
-}
-
-// Sum over the consumer threads; two banks of partials, one barrier per call.
-__device__ __forceinline__ float consumer_sum(float v, float (*red)[32], int& bank, int ncons) {
-    v = group_sum<32>(v);
-    const int nw = ncons >> 5;
-    if (nw == 1) return v;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0) red[bank][warp] = v;
-    consumer_sync(ncons);
-    float t = lane < nw ? red[bank][lane] : 0.0f;
-    bank ^= 1;
-    return group_sum<32>(t);
-}
 
 template <typename T, RowOp OP>
 struct TmaShape {
@@ -431,3 +381,4 @@ cudaError_t read_device_error(unsigned int* out, bool clear) {
 }
 
 }  // namespace muse
+
