@@ -6,12 +6,43 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace muse {
 
 // Elements of T in one 16-byte vector.
 template <typename T> struct Vec;
 template <> struct Vec<__nv_bfloat16> { static constexpr int N = 8; };
 template <> struct Vec<float> { static constexpr int N = 4; };
+
+// Programmatic dependent launch.  Every kernel of the library starts with
+// pdl_begin(): it lets the next kernel of the stream begin launching (its CTAs
+// take SM slots as this grid's CTAs retire), then waits until the previous
+// kernel of the stream has completed and its writes are visible.  Nothing is
+// read or written before the wait.  Both instructions are no-ops in a launch
+// without the programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_begin() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Launch with programmatic stream serialization allowed (the kernel must
+// begin with pdl_begin()).  Returns the launch error.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Streaming 16-byte load: cached in L2 only (every input byte is read once).
 __device__ __forceinline__ uint4 ld_stream(const void* p) {

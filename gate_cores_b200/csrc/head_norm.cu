@@ -15,7 +15,6 @@
 namespace muse {
 namespace {
 
-using qk::rope_pair;
 using qk::token_position;
 using qk::vec_sum_sq;
 
@@ -25,6 +24,7 @@ using qk::vec_sum_sq;
 // steps of RW rows; all their loads are issued before any arithmetic.
 template <typename T, int L, int VPL, int CH>
 __global__ void __launch_bounds__(256) output_norm_gate_kernel(const __grid_constant__ HeadGateArgs a) {
+    pdl_begin();
     constexpr int V = Vec<T>::N;
     constexpr int RW = 32 / L;
     const int lane = threadIdx.x & 31;
@@ -79,12 +79,15 @@ __global__ void __launch_bounds__(256) output_norm_gate_kernel(const __grid_cons
 // VPL vectors in registers: a lane covers the same element positions of every
 // head, so the values serve all heads of the token.  The token's query heads
 // and then its key heads are walked in steps of RW heads, BATCH steps at a
-// time with all their loads in flight; element arithmetic runs on packed FP32
-// pairs and each pair is unpacked once.
-template <typename T, int L, int VPL, bool ROPE, bool UPCAST, int BATCH, int MINB>
+// time with all their loads in flight.  Element arithmetic runs on packed FP32
+// pairs in the rotation-pair packing of to_eo (two packed multiply-adds per
+// two rotations).  TAIL = false is the instance for shapes without partial
+// vectors, heads or batches (every predicate drops out).
+template <typename T, int L, int VPL, bool ROPE, bool UPCAST, bool TAIL, int BATCH, int MINB>
 __global__ void __launch_bounds__(256, MINB) qk_norm_rope_kernel(const __grid_constant__ QkArgs a) {
+    pdl_begin();
     constexpr int V = Vec<T>::N;
-    constexpr int P = V / 2;  // pairs per vector
+    constexpr int H = qk::EoPack<T>::H;
     constexpr int RW = 32 / L;
     extern __shared__ float table[];  // [cos | sin][tile tokens][head_dim / 2]
     const int lane = threadIdx.x & 31;
@@ -101,6 +104,19 @@ __global__ void __launch_bounds__(256, MINB) qk_norm_rope_kernel(const __grid_co
     const int ntok = (int)min((int64_t)tt, a.tokens - t0);
     float* cs = table;
     float* sn = table + tt * half;
+    const int tok = warp / split;
+    const int part = warp - tok * split;
+    const int64_t t = t0 + tok;
+    const uint32_t head_bytes = (uint32_t)a.head_dim * sizeof(T);
+
+    const int nst_q = (a.hq + RW - 1) / RW;
+    const int nst = nst_q + (a.hkv + RW - 1) / RW;
+    const int spw = (nst + split - 1) / split;
+    const int g_begin = part * spw, g_end = min(nst, g_begin + spw);
+    const int q_hi = min(g_end, nst_q);   // query steps [g_begin, q_hi)
+    const int k_lo = max(g_begin, nst_q) - nst_q, k_hi = g_end - nst_q;  // key steps [k_lo, k_hi)
+    const char* q_src = static_cast<const char*>(a.q) + t * a.q_stride * (int64_t)sizeof(T);
+    const char* k_src = static_cast<const char*>(a.k) + t * a.k_stride * (int64_t)sizeof(T);
 
     if constexpr (ROPE) {
         for (int k = warp; k < ntok; k += nwarps) {
@@ -119,88 +135,96 @@ __global__ void __launch_bounds__(256, MINB) qk_norm_rope_kernel(const __grid_co
         }
         __syncthreads();
     }
-    const int tok = warp / split;
     if (tok >= ntok) return;
-    const int part = warp - tok * split;
-    const int64_t t = t0 + tok;
 
-    // this lane's vectors of a head: sub, sub + L, ...
+    // this lane's vectors of a head: sub, sub + L, ...; the cos / sin / -sin
+    // of their rotation pairs in the packing of to_eo (8-byte table reads:
+    // half and the pair offsets are even)
     bool vok[VPL];
     uint32_t voff[VPL];
-    float cv[VPL][P], sv[VPL][P];
+    f32x2 c2[VPL][H], s2[VPL][H], n2[VPL][H];
 #pragma unroll
     for (int k = 0; k < VPL; ++k) {
         const int vi = sub + k * L;
-        vok[k] = vi < nvec;
+        vok[k] = !TAIL || vi < nvec;
         voff[k] = (uint32_t)vi * 16u;
         if constexpr (ROPE) {
-            const int tb = tok * half + (vok[k] ? vi * P : 0);
+            const int tb = tok * half + (vok[k] ? vi * (V / 2) : 0);
 #pragma unroll
-            for (int j = 0; j < P; ++j) {
-                cv[k][j] = cs[tb + j];
-                sv[k][j] = sn[tb + j];
+            for (int j = 0; j < H; ++j) {
+                c2[k][j] = *reinterpret_cast<const f32x2*>(cs + tb + 2 * j);
+                s2[k][j] = *reinterpret_cast<const f32x2*>(sn + tb + 2 * j);
+                n2[k][j] = f2_mul(s2[k][j], f2_make(-1.0f, -1.0f));
             }
         }
     }
-    const uint32_t head_bytes = (uint32_t)a.head_dim * sizeof(T);
+    const uint32_t step_bytes = head_bytes * RW;
     const f32x2 qs2 = f2_make(a.query_scale, a.query_scale);
-    const int nst_q = (a.hq + RW - 1) / RW;
-    const int nst = nst_q + (a.hkv + RW - 1) / RW;
-    const int spw = (nst + split - 1) / split;
-    const int g_begin = part * spw, g_end = min(nst, g_begin + spw);
 
-    // segment 0: query heads, segment 1: key heads
+    // Steps [s_lo, s_hi) of one segment (the query or the key heads);
+    // SCALE: multiply by query_scale and cast again after the norm's cast.
+    auto run = [&](auto scale_tag, const char* seg, char* dst, int s_lo, int s_hi, int count) {
+        constexpr bool SCALE = decltype(scale_tag)::value;
+        const char* src = seg + (uint32_t)slot * head_bytes;
+        dst += (uint32_t)slot * head_bytes;
 #pragma unroll 1
-    for (int seg = 0; seg < 2; ++seg) {
-        const int s_lo = max(g_begin, seg == 0 ? 0 : nst_q) - (seg == 0 ? 0 : nst_q);
-        const int s_hi = min(g_end, seg == 0 ? nst_q : nst) - (seg == 0 ? 0 : nst_q);
-        if (s_lo >= s_hi) continue;
-        const int count = seg == 0 ? a.hq : a.hkv;
-        const bool scale = seg == 0 && a.query_scale != 1.0f;
-        const char* src = seg == 0 ? static_cast<const char*>(a.q) + t * a.q_stride * (int64_t)sizeof(T)
-                                   : static_cast<const char*>(a.k) + t * a.k_stride * (int64_t)sizeof(T);
-        char* dst = seg == 0 ? static_cast<char*>(a.q_out) + t * a.q_out_stride * (int64_t)sizeof(T)
-                             : static_cast<char*>(a.k_out) + t * a.k_out_stride * (int64_t)sizeof(T);
         for (int st0 = s_lo; st0 < s_hi; st0 += BATCH) {
             uint4 xv[BATCH][VPL];
             bool hv[BATCH];
 #pragma unroll
             for (int b = 0; b < BATCH; ++b) {
-                const int head = (st0 + b) * RW + slot;
-                hv[b] = st0 + b < s_hi && head < count;
-                const char* hs = src + (uint32_t)head * head_bytes;
+                hv[b] = !TAIL || (st0 + b < s_hi && (st0 + b) * RW + slot < count);
+                const char* hs = src + (uint32_t)(st0 + b) * step_bytes;
 #pragma unroll
                 for (int k = 0; k < VPL; ++k)
                     xv[b][k] = (hv[b] && vok[k]) ? ld_stream(hs + voff[k]) : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
             for (int b = 0; b < BATCH; ++b) {
-                f32x2 x[VPL][P];
+                f32x2 e[VPL][H], o[VPL][H];
                 f32x2 acc = f2_make(0.0f, 0.0f);
 #pragma unroll
                 for (int k = 0; k < VPL; ++k) {
-                    to_pairs<T>(xv[b][k], x[k]);
+                    qk::to_eo<T>(xv[b][k], e[k], o[k]);
 #pragma unroll
-                    for (int q = 0; q < P; ++q) acc = f2_fma(x[k][q], x[k][q], acc);
+                    for (int j = 0; j < H; ++j) {
+                        acc = f2_fma(e[k][j], e[k][j], acc);
+                        acc = f2_fma(o[k][j], o[k][j], acc);
+                    }
                 }
                 const float r = inv_rms_fast(group_sum<L>(f2_sum(acc)), inv_width, a.eps);
                 const f32x2 r2 = f2_make(r, r);
-                const int head = (st0 + b) * RW + slot;
-                char* hd = dst + (uint32_t)head * head_bytes;
+                char* hd = dst + (uint32_t)(st0 + b) * step_bytes;
 #pragma unroll
                 for (int k = 0; k < VPL; ++k) {
-                    f32x2 y[P];
 #pragma unroll
-                    for (int q = 0; q < P; ++q) {
-                        f32x2 n = round_pair<T>(f2_mul(x[k][q], r2));     // cast to the Q/K dtype
-                        if (scale) n = round_pair<T>(f2_mul(n, qs2));     // query_scale, cast again
-                        if constexpr (ROPE) n = rope_pair<T, UPCAST>(n, cv[k][q], sv[k][q]);
-                        y[q] = n;
+                    for (int j = 0; j < H; ++j) {
+                        f32x2 ev = round_pair<T>(f2_mul(e[k][j], r2));  // cast to the Q/K dtype
+                        f32x2 ov = round_pair<T>(f2_mul(o[k][j], r2));
+                        if constexpr (SCALE) {                         // query_scale, cast again
+                            ev = round_pair<T>(f2_mul(ev, qs2));
+                            ov = round_pair<T>(f2_mul(ov, qs2));
+                        }
+                        if constexpr (ROPE) qk::rope_eo<T, UPCAST>(ev, ov, c2[k][j], s2[k][j], n2[k][j]);
+                        e[k][j] = ev;
+                        o[k][j] = ov;
                     }
-                    if (hv[b] && vok[k]) st_vec(hd + voff[k], from_pairs<T>(y));
+                    if (hv[b] && vok[k]) st_vec(hd + voff[k], qk::from_eo<T>(e[k], o[k]));
                 }
             }
         }
+    };
+
+    if (g_begin < q_hi) {
+        char* dst = static_cast<char*>(a.q_out) + t * a.q_out_stride * (int64_t)sizeof(T);
+        if (a.query_scale != 1.0f)
+            run(std::true_type{}, q_src, dst, g_begin, q_hi, a.hq);
+        else
+            run(std::false_type{}, q_src, dst, g_begin, q_hi, a.hq);
+    }
+    if (k_lo < k_hi) {
+        char* dst = static_cast<char*>(a.k_out) + t * a.k_out_stride * (int64_t)sizeof(T);
+        run(std::false_type{}, k_src, dst, k_lo, k_hi, a.hkv);
     }
 }
 
@@ -215,8 +239,7 @@ cudaError_t launch_head_gate_l(const HeadGateArgs& a, cudaStream_t s) {
     constexpr int RW = 32 / L;
     const int64_t rows_per_cta = (int64_t)(kThreads / 32) * CH * RW;
     const int64_t grid = (a.rows + rows_per_cta - 1) / rows_per_cta;
-    output_norm_gate_kernel<T, L, VPL, CH><<<(unsigned)grid, kThreads, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(output_norm_gate_kernel<T, L, VPL, CH>, (unsigned)grid, kThreads, 0, s, a);
 }
 
 // Lanes per head: NV / VPL rounded up to a power of two; two vectors per lane
@@ -243,17 +266,24 @@ cudaError_t launch_qk_l(const QkArgs& a0, cudaStream_t s) {
     constexpr int BATCH = 4;
     QkArgs a = a0;
     const int nwarps = kThreads / 32;
-    const int nsteps = (a.hq + a.hkv + RW - 1) / RW;
+    const int nst_q = (a.hq + RW - 1) / RW, nst_k = (a.hkv + RW - 1) / RW;
     // Split a token's head steps over up to 8 warps while the grid would
     // leave SMs idle (decode-sized batches).
     int split = 1;
-    while (split < nwarps && split < nsteps && (a.tokens * split + nwarps - 1) / nwarps < 2 * sm_count()) split *= 2;
+    while (split < nwarps && split < nst_q + nst_k &&
+           (a.tokens * split + nwarps - 1) / nwarps < 2 * sm_count())
+        split *= 2;
     a.split = split;
     const int tt = nwarps / split;
     const size_t smem = ROPE ? sizeof(float) * 2 * tt * (a.head_dim / 2) : 0;
     const int64_t grid = (a.tokens + tt - 1) / tt;
-    qk_norm_rope_kernel<T, L, VPL, ROPE, UPCAST, BATCH, kQkMinBlocks><<<(unsigned)grid, kThreads, smem, s>>>(a);
-    return cudaGetLastError();
+    const bool exact = split == 1 && a.head_dim / Vec<T>::N == L * VPL && a.hq % RW == 0 &&
+                       a.hkv % RW == 0 && nst_q % BATCH == 0 && nst_k % BATCH == 0;
+    if (exact)
+        return launch_pdl(qk_norm_rope_kernel<T, L, VPL, ROPE, UPCAST, false, BATCH, kQkMinBlocks>,
+                          (unsigned)grid, kThreads, smem, s, a);
+    return launch_pdl(qk_norm_rope_kernel<T, L, VPL, ROPE, UPCAST, true, BATCH, kQkMinBlocks>,
+                      (unsigned)grid, kThreads, smem, s, a);
 }
 
 template <typename T, int L, int VPL>

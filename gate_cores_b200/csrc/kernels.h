@@ -58,7 +58,6 @@ struct QkArgs {
     int32_t num_seqs;
     int32_t hq, hkv, head_dim;
     int32_t split;              // warps sharing one token's head steps (1, 2, 4, 8)
-    int32_t tokens_per_warp;    // consecutive tokens one warp streams through
     int32_t pos_mode;           // 0 explicit, 1 BSHD derived, 2 THD derived
     float eps;
     float query_scale;

@@ -31,19 +31,59 @@ __device__ __forceinline__ int32_t token_position(const QkArgs& a, int64_t t) {
     return (int32_t)(t - __ldg(a.cu_seqlens + lo));
 }
 
-// Rotation of one normalised, cast pair (a, b) by (c, s).
-//   legacy / FP32 tensors: FP32 rotation (the caller casts once afterwards);
-//   v2 (bf16): each product rounded to bf16, then the sum, rounded by the caller.
+// ---- Rotation-pair packing.  A 16-byte vector holds Vec<T>::N elements, i.e.
+// N / 2 rotation pairs (2i, 2i + 1).  The Q/K kernel holds them as packed FP32
+// pairs that group like members of two neighbouring rotation pairs: ev[j]
+// holds the first members of rotation pairs 2j and 2j + 1, od[j] the second
+// members.  The rotation is then elementwise on (ev, od) and costs two packed
+// multiply-adds per two rotation pairs.  H = N / 4 packs of each kind.
+template <typename T> struct EoPack { static constexpr int H = Vec<T>::N / 4; };
+
+template <typename T> __device__ __forceinline__ void to_eo(const uint4& v, f32x2* ev, f32x2* od);
+template <> __device__ __forceinline__ void to_eo<__nv_bfloat16>(const uint4& v, f32x2* ev, f32x2* od) {
+    ev[0] = f2_make(bf16_lo(v.x), bf16_lo(v.y));
+    od[0] = f2_make(bf16_hi(v.x), bf16_hi(v.y));
+    ev[1] = f2_make(bf16_lo(v.z), bf16_lo(v.w));
+    od[1] = f2_make(bf16_hi(v.z), bf16_hi(v.w));
+}
+template <> __device__ __forceinline__ void to_eo<float>(const uint4& v, f32x2* ev, f32x2* od) {
+    ev[0] = f2_make(__uint_as_float(v.x), __uint_as_float(v.z));
+    od[0] = f2_make(__uint_as_float(v.y), __uint_as_float(v.w));
+}
+
+// Inverse of to_eo (bf16: round to nearest even).
+template <typename T> __device__ __forceinline__ uint4 from_eo(const f32x2* ev, const f32x2* od);
+template <> __device__ __forceinline__ uint4 from_eo<__nv_bfloat16>(const f32x2* ev, const f32x2* od) {
+    float e0, e1, e2, e3, o0, o1, o2, o3;
+    f2_split(ev[0], e0, e1);
+    f2_split(od[0], o0, o1);
+    f2_split(ev[1], e2, e3);
+    f2_split(od[1], o2, o3);
+    return make_uint4(pack_bf16x2(e0, o0), pack_bf16x2(e1, o1), pack_bf16x2(e2, o2), pack_bf16x2(e3, o3));
+}
+template <> __device__ __forceinline__ uint4 from_eo<float>(const f32x2* ev, const f32x2* od) {
+    float e0, e1, o0, o1;
+    f2_split(ev[0], e0, e1);
+    f2_split(od[0], o0, o1);
+    return make_uint4(__float_as_uint(e0), __float_as_uint(o0), __float_as_uint(e1), __float_as_uint(o1));
+}
+
+// Rotation of normalised, cast members (e, o) of two rotation pairs by
+// angles with cosines c and sines s (ns = -s):
+//   FP32 rotation: e' = e c - o s, o' = e s + o c, each one product rounded and
+//   one fused multiply-add (the caller casts once afterwards);
+//   v2 (bf16): each product rounded to bf16, then the FP32 sum (the caller
+//   casts the sum); -(o s) rounds to exactly the negated bf16 of o s.
 template <typename T, bool UPCAST>
-__device__ __forceinline__ f32x2 rope_pair(f32x2 n, float c, float s) {
-    float a, b;
-    f2_split(n, a, b);
+__device__ __forceinline__ void rope_eo(f32x2& e, f32x2& o, f32x2 c, f32x2 s, f32x2 ns) {
     if constexpr (UPCAST) {
-        return f2_make(a * c - b * s, a * s + b * c);
+        const f32x2 e2 = f2_fma(o, ns, f2_mul(e, c));
+        o = f2_fma(e, s, f2_mul(o, c));
+        e = e2;
     } else {
-        const uint32_t p = pack_bf16x2(a * c, b * s);
-        const uint32_t q = pack_bf16x2(a * s, b * c);
-        return f2_make(bf16_lo(p) - bf16_hi(p), bf16_lo(q) + bf16_hi(q));
+        const f32x2 e2 = f2_add(round_pair<T>(f2_mul(e, c)), round_pair<T>(f2_mul(o, ns)));
+        o = f2_add(round_pair<T>(f2_mul(e, s)), round_pair<T>(f2_mul(o, c)));
+        e = e2;
     }
 }
 

@@ -230,22 +230,27 @@ __device__ __forceinline__ void row_norm_body(const RowArgs& a) {
 // One entry symbol per core, so launch lists and profiles name the core.
 template <typename T, int VPT, bool G, int S, bool CSM>
 __global__ void __launch_bounds__(kMaxThreads) rms_norm_regs_kernel(const __grid_constant__ RowArgs a) {
+    pdl_begin();
     row_norm_body<T, RowOp::kRms, VPT, G, S, CSM>(a);
 }
 template <typename T, int VPT, bool G, int S, bool CSM>
 __global__ void __launch_bounds__(kMaxThreads) input_scale_norm_regs_kernel(const __grid_constant__ RowArgs a) {
+    pdl_begin();
     row_norm_body<T, RowOp::kInputScale, VPT, G, S, CSM>(a);
 }
 template <typename T, int VPT, bool G, int S, bool CSM>
 __global__ void __launch_bounds__(kMaxThreads) output_norm_gate_row_regs_kernel(const __grid_constant__ RowArgs a) {
+    pdl_begin();
     row_norm_body<T, RowOp::kNormGate, VPT, G, S, CSM>(a);
 }
 template <typename T, int VPT, bool G, int S, bool CSM>
 __global__ void __launch_bounds__(kMaxThreads) norm_residual_regs_kernel(const __grid_constant__ RowArgs a) {
+    pdl_begin();
     row_norm_body<T, RowOp::kResidual, VPT, G, S, CSM>(a);
 }
 template <typename T, int VPT, bool G, int S, bool CSM>
 __global__ void __launch_bounds__(kMaxThreads) norm_residual_input_scale_regs_kernel(const __grid_constant__ RowArgs a) {
+    pdl_begin();
     row_norm_body<T, RowOp::kResidualIS, VPT, G, S, CSM>(a);
 }
 
@@ -283,8 +288,7 @@ cudaError_t launch_row_g(const RowArgs& a0, int nvec, cudaStream_t s) {
         if (e != cudaSuccess) return e;
     }
     const int64_t grid = (a.rows + a.rows_per_cta - 1) / a.rows_per_cta;
-    kern<<<(unsigned)grid, nt, smem, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(kern, (unsigned)grid, (unsigned)nt, smem, s, a);
 }
 
 template <typename T, RowOp OP, int VPT>

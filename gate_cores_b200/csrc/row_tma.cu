@@ -271,22 +271,27 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
 // One entry symbol per core, so launch lists and profiles name the core.
 template <typename T, int VPT, bool G, int S>
 __global__ void __launch_bounds__(512 + 32) rms_norm_kernel(const __grid_constant__ RowArgs a) {
+    pdl_begin();
     row_tma_body<T, RowOp::kRms, VPT, G, S>(a);
 }
 template <typename T, int VPT, bool G, int S>
 __global__ void __launch_bounds__(512 + 32) input_scale_norm_kernel(const __grid_constant__ RowArgs a) {
+    pdl_begin();
     row_tma_body<T, RowOp::kInputScale, VPT, G, S>(a);
 }
 template <typename T, int VPT, bool G, int S>
 __global__ void __launch_bounds__(512 + 32) output_norm_gate_row_kernel(const __grid_constant__ RowArgs a) {
+    pdl_begin();
     row_tma_body<T, RowOp::kNormGate, VPT, G, S>(a);
 }
 template <typename T, int VPT, bool G, int S>
 __global__ void __launch_bounds__(512 + 32) norm_residual_kernel(const __grid_constant__ RowArgs a) {
+    pdl_begin();
     row_tma_body<T, RowOp::kResidual, VPT, G, S>(a);
 }
 template <typename T, int VPT, bool G, int S>
 __global__ void __launch_bounds__(512 + 32) norm_residual_input_scale_kernel(const __grid_constant__ RowArgs a) {
+    pdl_begin();
     row_tma_body<T, RowOp::kResidualIS, VPT, G, S>(a);
 }
 
@@ -318,8 +323,7 @@ cudaError_t launch_row_tma_s(const RowArgs& a0, int nvec, cudaStream_t s) {
     if (grid < 1) grid = 1;
     a.rows_per_cta = (int32_t)((a.rows + grid - 1) / grid);
     grid = (a.rows + a.rows_per_cta - 1) / a.rows_per_cta;
-    kern<<<(unsigned)grid, threads, smem, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(kern, (unsigned)grid, (unsigned)threads, smem, s, a);
 }
 
 template <typename T, RowOp OP, int VPT, bool G>
