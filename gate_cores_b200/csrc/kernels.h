@@ -28,7 +28,7 @@ struct RowArgs {
     int64_t rows;
     int64_t x_stride, y_stride, gate_stride, s_in_stride, s_out_stride;
     int32_t width;
-    int32_t rows_per_cta;   // set by the launcher
+    int32_t rows_per_cta;   // set by the launcher (register-staged row kernels)
     float gain_offset;
     float eps;
 };

@@ -1,7 +1,7 @@
 // Row-wide normalisation kernels (cores 1, 2, 5 and core 4 with one norm per
 // token) on a TMA bulk-copy pipeline.
 //
-// Each CTA owns a contiguous chunk of rows.  One producer warp streams whole
+// The rows are dealt round-robin to the CTAs.  One producer warp streams whole
 // rows (activation row, plus the gate row for core 4 or the FP32 stream row
 // for core 5) from global memory into a ring of S shared-memory stages with
 // cp.async.bulk, each stage tracked by a "full" mbarrier (transaction bytes)
@@ -78,9 +78,13 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
     const int nvec = a.width / V;
     const StageLayout L = stage_layout<T, OP>(a.width);
 
-    const int64_t r0 = (int64_t)blockIdx.x * a.rows_per_cta;
-    const int64_t r1 = min(r0 + (int64_t)a.rows_per_cta, a.rows);
-    const int n = (int)max((int64_t)0, r1 - r0);
+    // This CTA's rows: r0, r0 + step, ... - rows interleaved across the grid,
+    // so at any time the CTAs stream one compact window of the tensors
+    // (measured slightly ahead of contiguous chunks per CTA when the previous
+    // kernel left dirty lines in L2).
+    const int64_t step = gridDim.x;
+    const int64_t r0 = blockIdx.x;
+    const int n = (int)max((int64_t)0, (a.rows - r0 + step - 1) / step);
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
@@ -104,7 +108,7 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
                 if (k >= S) ok = mbar_wait(&empty_bar[s], (uint32_t)((k / S - 1) & 1));
                 if (!ok) break;
                 unsigned char* st = smem + (size_t)s * L.stage_bytes;
-                const int64_t row = r0 + k;
+                const int64_t row = r0 + k * step;
                 mbar_arrive_expect_tx(&full_bar[s], bytes);
                 bulk_g2s(st + L.x_off, static_cast<const char*>(a.x) + row * a.x_stride * (int64_t)sizeof(T),
                          L.x_bytes, &full_bar[s]);
@@ -174,8 +178,8 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
     char* out_row = t_is_residual(OP)
         ? reinterpret_cast<char*>(a.stream_out + r0 * a.s_out_stride)
         : static_cast<char*>(a.y) + r0 * a.y_stride * (int64_t)sizeof(T);
-    const int64_t out_step = t_is_residual(OP) ? a.s_out_stride * (int64_t)sizeof(float)
-                                               : a.y_stride * (int64_t)sizeof(T);
+    const int64_t out_step = step * (t_is_residual(OP) ? a.s_out_stride * (int64_t)sizeof(float)
+                                                      : a.y_stride * (int64_t)sizeof(T));
 
     // After a timed-out wait a warp stops touching the ring and the outputs but
     // keeps joining the consumer barrier, so no other warp is left waiting.
@@ -321,8 +325,6 @@ cudaError_t launch_row_tma_s(const RowArgs& a0, int nvec, cudaStream_t s) {
     int64_t grid = (int64_t)per_sm * sm_count();
     if (grid > a.rows) grid = a.rows;
     if (grid < 1) grid = 1;
-    a.rows_per_cta = (int32_t)((a.rows + grid - 1) / grid);
-    grid = (a.rows + a.rows_per_cta - 1) / a.rows_per_cta;
     return launch_pdl(kern, (unsigned)grid, (unsigned)threads, smem, s, a);
 }
 
