@@ -132,8 +132,8 @@ def muse_norm_residual(stream_in, branch, stream_out, branch_dtype, rows, hidden
 
 
 def muse_device_error(clear: bool = False) -> int:
-    """Device-side error word of the current device (bit 0: a bounded mbarrier
-    wait in a row kernel timed out).  Synchronous."""
+    """Device-side error flags of the current device (bit 0: a bounded mbarrier
+    wait in a row kernel timed out; bit 1: one in the Q/K kernel).  Synchronous."""
     flags = ctypes.c_uint(0)
     _call("muse_device_error", ctypes.byref(flags), int(clear))
     return flags.value

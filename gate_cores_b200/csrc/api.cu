@@ -364,7 +364,12 @@ muse_status muse_norm_residual(const float* stream_in, const void* branch, float
 
 muse_status muse_device_error(unsigned int* flags, int clear) {
     if (!flags) return fail(MUSE_ERR_INVALID_ARGUMENT, "muse_device_error: null flags");
-    return from_cuda(muse::read_device_error(flags, clear != 0), "muse_device_error");
+    // bit 0: the row pipeline's word, bit 1: the Q/K ring's word
+    unsigned int row = 0, qk = 0;
+    cudaError_t e = muse::read_device_error(&row, clear != 0);
+    if (e == cudaSuccess) e = muse::read_qk_device_error(&qk, clear != 0);
+    *flags = (row ? 1u : 0u) | (qk ? 2u : 0u);
+    return from_cuda(e, "muse_device_error");
 }
 
 muse_status muse_stream_copy(const void* src, void* dst, int64_t bytes, cudaStream_t stream) {

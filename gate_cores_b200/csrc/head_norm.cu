@@ -14,6 +14,14 @@
 
 namespace muse {
 namespace {
+__device__ unsigned int g_device_error;  // nonzero: an mbarrier wait of the Q/K ring timed out
+}  // namespace
+}  // namespace muse
+
+#include "tma_pipe.cuh"
+
+namespace muse {
+namespace {
 
 using qk::token_position;
 using qk::vec_sum_sq;
@@ -73,28 +81,34 @@ __global__ void __launch_bounds__(256) output_norm_gate_kernel(const __grid_cons
 // ------------------------------------------------------------------ core 3
 
 // One CTA per tile of tokens; each warp owns one token (or, with split > 1,
-// one of `split` ranges of that token's head steps).  The CTA first fills a
-// shared table with cos/sin of every (token, pair) angle of the tile - one
-// sincosf per pair per token - and each lane then keeps the cos/sin of its own
-// VPL vectors in registers: a lane covers the same element positions of every
-// head, so the values serve all heads of the token.  The token's query heads
-// and then its key heads are walked in steps of RW heads, BATCH steps at a
-// time with all their loads in flight.  Element arithmetic runs on packed FP32
+// one of `split` ranges of that token's head steps).  The token's query heads
+// and then its key heads are walked in steps of RW heads (L lanes x one
+// 16-byte vector per head); the steps are grouped in batches of BATCH, and
+// each warp streams its batches through its own ring of R shared-memory slots
+// with cp.async.bulk (one request per batch, issued by lane 0, completed on
+// the slot's mbarrier).  The first R batches go out before anything else, so
+// the CTA builds its cos/sin table - one sincosf per pair per token, shared by
+// all heads of the token - while they are in flight; a slot is refilled as
+// soon as the warp has read it, so every warp keeps R batches in flight
+// without holding them in registers.  Element arithmetic runs on packed FP32
 // pairs in the rotation-pair packing of to_eo (two packed multiply-adds per
 // two rotations).  TAIL = false is the instance for shapes without partial
-// vectors, heads or batches (every predicate drops out).
-template <typename T, int L, int VPL, bool ROPE, bool UPCAST, bool TAIL, int BATCH, int MINB>
+// vectors, heads or batches (every predicate drops out).  Every mbarrier wait
+// is bounded; a timeout sets the error word and the warp stops, after its
+// copies in flight have landed (bounded again).
+template <typename T, int L, bool ROPE, bool UPCAST, bool TAIL, int BATCH, int R, int MINB>
 __global__ void __launch_bounds__(256, MINB) qk_norm_rope_kernel(const __grid_constant__ QkArgs a) {
     pdl_begin();
     constexpr int V = Vec<T>::N;
     constexpr int H = qk::EoPack<T>::H;
     constexpr int RW = 32 / L;
-    extern __shared__ float table[];  // [cos | sin][tile tokens][head_dim / 2]
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t bars[8][R];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int nwarps = blockDim.x >> 5;
     const int split = a.split;
-    const int tt = nwarps / split;  // tokens per tile
+    const int tt = nwarps / split;
     const int sub = lane % L;
     const int slot = lane / L;
     const int nvec = a.head_dim / V;
@@ -102,21 +116,51 @@ __global__ void __launch_bounds__(256, MINB) qk_norm_rope_kernel(const __grid_co
     const float inv_width = 1.0f / (float)a.head_dim;
     const int64_t t0 = (int64_t)blockIdx.x * tt;
     const int ntok = (int)min((int64_t)tt, a.tokens - t0);
-    float* cs = table;
-    float* sn = table + tt * half;
+    float* cs = reinterpret_cast<float*>(smem_raw);
+    float* sn = cs + tt * half;
     const int tok = warp / split;
     const int part = warp - tok * split;
     const int64_t t = t0 + tok;
     const uint32_t head_bytes = (uint32_t)a.head_dim * sizeof(T);
+    const uint32_t slot_bytes = (BATCH * RW * head_bytes + 127u) & ~127u;
+    unsigned char* ring = smem_raw + ((2u * tt * half * 4u + 127u) & ~127u) + (uint32_t)warp * R * slot_bytes;
 
     const int nst_q = (a.hq + RW - 1) / RW;
     const int nst = nst_q + (a.hkv + RW - 1) / RW;
     const int spw = (nst + split - 1) / split;
     const int g_begin = part * spw, g_end = min(nst, g_begin + spw);
-    const int q_hi = min(g_end, nst_q);   // query steps [g_begin, q_hi)
-    const int k_lo = max(g_begin, nst_q) - nst_q, k_hi = g_end - nst_q;  // key steps [k_lo, k_hi)
+    const int q_hi = min(g_end, nst_q);
+    const int k_lo = max(g_begin, nst_q) - nst_q, k_hi = g_end - nst_q;
+    const int nbq = q_hi > g_begin ? (q_hi - g_begin + BATCH - 1) / BATCH : 0;
+    const int nbk = k_hi > k_lo ? (k_hi - k_lo + BATCH - 1) / BATCH : 0;
+    const int nb = tok < ntok ? nbq + nbk : 0;
     const char* q_src = static_cast<const char*>(a.q) + t * a.q_stride * (int64_t)sizeof(T);
     const char* k_src = static_cast<const char*>(a.k) + t * a.k_stride * (int64_t)sizeof(T);
+
+    // batch j: first step, end of its segment, head count, source row
+    auto batch = [&](int j, int& st0, int& s_hi, int& count, bool& isq) {
+        isq = j < nbq;
+        st0 = isq ? g_begin + j * BATCH : k_lo + (j - nbq) * BATCH;
+        s_hi = isq ? q_hi : k_hi;
+        count = isq ? a.hq : a.hkv;
+    };
+    auto issue = [&](int j) {
+        int st0, s_hi, count;
+        bool isq;
+        batch(j, st0, s_hi, count, isq);
+        const int h0 = st0 * RW, h1 = min(count, min(st0 + BATCH, s_hi) * RW);
+        const uint32_t bytes = (uint32_t)(h1 - h0) * head_bytes;
+        uint64_t* bar = &bars[warp][j % R];
+        pipe::mbar_arrive_expect_tx(bar, bytes);
+        pipe::bulk_g2s(ring + (j % R) * slot_bytes, (isq ? q_src : k_src) + (uint32_t)h0 * head_bytes, bytes, bar);
+    };
+    int issued = 0;
+    if (lane == 0 && nb > 0) {
+        for (int r = 0; r < R; ++r) pipe::mbar_init(&bars[warp][r], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (; issued < min(R, nb); ++issued) issue(issued);
+    }
+    __syncwarp();
 
     if constexpr (ROPE) {
         for (int k = warp; k < ntok; k += nwarps) {
@@ -135,103 +179,98 @@ __global__ void __launch_bounds__(256, MINB) qk_norm_rope_kernel(const __grid_co
         }
         __syncthreads();
     }
-    if (tok >= ntok) return;
+    if (nb == 0) return;
 
-    // this lane's vectors of a head: sub, sub + L, ...; the cos / sin / -sin
-    // of their rotation pairs in the packing of to_eo (8-byte table reads:
-    // half and the pair offsets are even)
-    bool vok[VPL];
-    uint32_t voff[VPL];
-    f32x2 c2[VPL][H], s2[VPL][H], n2[VPL][H];
+    const bool vok = !TAIL || sub < nvec;
+    const uint32_t voff = (uint32_t)sub * 16u;
+    f32x2 c2[H], s2[H], n2[H];
+    if constexpr (ROPE) {
+        const int tb = tok * half + (vok ? sub * (V / 2) : 0);
 #pragma unroll
-    for (int k = 0; k < VPL; ++k) {
-        const int vi = sub + k * L;
-        vok[k] = !TAIL || vi < nvec;
-        voff[k] = (uint32_t)vi * 16u;
-        if constexpr (ROPE) {
-            const int tb = tok * half + (vok[k] ? vi * (V / 2) : 0);
-#pragma unroll
-            for (int j = 0; j < H; ++j) {
-                c2[k][j] = *reinterpret_cast<const f32x2*>(cs + tb + 2 * j);
-                s2[k][j] = *reinterpret_cast<const f32x2*>(sn + tb + 2 * j);
-                n2[k][j] = f2_mul(s2[k][j], f2_make(-1.0f, -1.0f));
-            }
+        for (int j = 0; j < H; ++j) {
+            c2[j] = *reinterpret_cast<const f32x2*>(cs + tb + 2 * j);
+            s2[j] = *reinterpret_cast<const f32x2*>(sn + tb + 2 * j);
+            n2[j] = f2_mul(s2[j], f2_make(-1.0f, -1.0f));
         }
     }
-    const uint32_t step_bytes = head_bytes * RW;
     const f32x2 qs2 = f2_make(a.query_scale, a.query_scale);
+    const bool scaled = a.query_scale != 1.0f;
+    char* q_dst = static_cast<char*>(a.q_out) + t * a.q_out_stride * (int64_t)sizeof(T) + (uint32_t)slot * head_bytes;
+    char* k_dst = static_cast<char*>(a.k_out) + t * a.k_out_stride * (int64_t)sizeof(T) + (uint32_t)slot * head_bytes;
 
-    // Steps [s_lo, s_hi) of one segment (the query or the key heads);
-    // SCALE: multiply by query_scale and cast again after the norm's cast.
-    auto run = [&](auto scale_tag, const char* seg, char* dst, int s_lo, int s_hi, int count) {
+    auto compute = [&](auto scale_tag, const uint4 (&xv)[BATCH], const bool (&hv)[BATCH], char* dst) {
         constexpr bool SCALE = decltype(scale_tag)::value;
-        const char* src = seg + (uint32_t)slot * head_bytes;
-        dst += (uint32_t)slot * head_bytes;
-#pragma unroll 1
-        for (int st0 = s_lo; st0 < s_hi; st0 += BATCH) {
-            uint4 xv[BATCH][VPL];
-            bool hv[BATCH];
 #pragma unroll
-            for (int b = 0; b < BATCH; ++b) {
-                hv[b] = !TAIL || (st0 + b < s_hi && (st0 + b) * RW + slot < count);
-                const char* hs = src + (uint32_t)(st0 + b) * step_bytes;
+        for (int b = 0; b < BATCH; ++b) {
+            f32x2 e[H], o[H];
+            f32x2 acc = f2_make(0.0f, 0.0f);
+            qk::to_eo<T>(xv[b], e, o);
 #pragma unroll
-                for (int k = 0; k < VPL; ++k)
-                    xv[b][k] = (hv[b] && vok[k]) ? ld_stream(hs + voff[k]) : make_uint4(0, 0, 0, 0);
+            for (int j = 0; j < H; ++j) {
+                acc = f2_fma(e[j], e[j], acc);
+                acc = f2_fma(o[j], o[j], acc);
             }
+            const float r = inv_rms_fast(group_sum<L>(f2_sum(acc)), inv_width, a.eps);
+            const f32x2 r2 = f2_make(r, r);
 #pragma unroll
-            for (int b = 0; b < BATCH; ++b) {
-                f32x2 e[VPL][H], o[VPL][H];
-                f32x2 acc = f2_make(0.0f, 0.0f);
-#pragma unroll
-                for (int k = 0; k < VPL; ++k) {
-                    qk::to_eo<T>(xv[b][k], e[k], o[k]);
-#pragma unroll
-                    for (int j = 0; j < H; ++j) {
-                        acc = f2_fma(e[k][j], e[k][j], acc);
-                        acc = f2_fma(o[k][j], o[k][j], acc);
-                    }
+            for (int j = 0; j < H; ++j) {
+                f32x2 ev = round_pair<T>(f2_mul(e[j], r2));  // cast to the Q/K dtype
+                f32x2 ov = round_pair<T>(f2_mul(o[j], r2));
+                if constexpr (SCALE) {                      // query_scale, cast again
+                    ev = round_pair<T>(f2_mul(ev, qs2));
+                    ov = round_pair<T>(f2_mul(ov, qs2));
                 }
-                const float r = inv_rms_fast(group_sum<L>(f2_sum(acc)), inv_width, a.eps);
-                const f32x2 r2 = f2_make(r, r);
-                char* hd = dst + (uint32_t)(st0 + b) * step_bytes;
-#pragma unroll
-                for (int k = 0; k < VPL; ++k) {
-#pragma unroll
-                    for (int j = 0; j < H; ++j) {
-                        f32x2 ev = round_pair<T>(f2_mul(e[k][j], r2));  // cast to the Q/K dtype
-                        f32x2 ov = round_pair<T>(f2_mul(o[k][j], r2));
-                        if constexpr (SCALE) {                         // query_scale, cast again
-                            ev = round_pair<T>(f2_mul(ev, qs2));
-                            ov = round_pair<T>(f2_mul(ov, qs2));
-                        }
-                        if constexpr (ROPE) qk::rope_eo<T, UPCAST>(ev, ov, c2[k][j], s2[k][j], n2[k][j]);
-                        e[k][j] = ev;
-                        o[k][j] = ov;
-                    }
-                    if (hv[b] && vok[k]) st_vec(hd + voff[k], qk::from_eo<T>(e[k], o[k]));
-                }
+                if constexpr (ROPE) qk::rope_eo<T, UPCAST>(ev, ov, c2[j], s2[j], n2[j]);
+                e[j] = ev;
+                o[j] = ov;
             }
+            if (hv[b]) st_vec(dst + (uint32_t)(b * RW) * head_bytes + voff, qk::from_eo<T>(e, o));
         }
     };
 
-    if (g_begin < q_hi) {
-        char* dst = static_cast<char*>(a.q_out) + t * a.q_out_stride * (int64_t)sizeof(T);
-        if (a.query_scale != 1.0f)
-            run(std::true_type{}, q_src, dst, g_begin, q_hi, a.hq);
+    bool alive = true;
+    int j = 0;
+#pragma unroll 1
+    for (; j < nb; ++j) {
+        alive = __all_sync(0xffffffffu, alive && pipe::mbar_wait(&bars[warp][j % R], (uint32_t)((j / R) & 1)));
+        if (!alive) break;
+        int st0, s_hi, count;
+        bool isq;
+        batch(j, st0, s_hi, count, isq);
+        const unsigned char* sl = ring + (j % R) * slot_bytes + (uint32_t)slot * head_bytes + voff;
+        uint4 xv[BATCH];
+        bool hv[BATCH];
+#pragma unroll
+        for (int b = 0; b < BATCH; ++b) {
+            hv[b] = vok && (!TAIL || (st0 + b < s_hi && (st0 + b) * RW + slot < count));
+            xv[b] = hv[b] ? *reinterpret_cast<const uint4*>(sl + (uint32_t)(b * RW) * head_bytes) : make_uint4(0, 0, 0, 0);
+        }
+        // the warp is done with the slot: refill it with batch j + R
+        __syncwarp();
+        if (lane == 0 && issued < nb) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue(issued);
+            ++issued;
+        }
+        char* dst = (isq ? q_dst : k_dst) + (uint32_t)(st0 * RW) * head_bytes;
+        if (isq && scaled)
+            compute(std::true_type{}, xv, hv, dst);
         else
-            run(std::false_type{}, q_src, dst, g_begin, q_hi, a.hq);
+            compute(std::false_type{}, xv, hv, dst);
     }
-    if (k_lo < k_hi) {
-        char* dst = static_cast<char*>(a.k_out) + t * a.k_out_stride * (int64_t)sizeof(T);
-        run(std::false_type{}, k_src, dst, k_lo, k_hi, a.hkv);
-    }
+    // after a timed-out wait: let this warp's copies still in flight land
+    if (lane == 0)
+        for (int k = j; k < issued; ++k)
+            if (!pipe::mbar_wait(&bars[warp][k % R], (uint32_t)((k / R) & 1))) break;
 }
 
 constexpr int kThreads = 256;
-// Resident CTAs per SM the Q/K kernel's registers are sized for: 4 (32 warps)
-// keeps enough loads in flight to cover HBM latency (measured: 2 resident
-// CTAs reach about 2/3 of the copy bandwidth, 4 about 9/10).
+// Q/K kernel: 4 head steps per batch, a ring of 3 batches per warp (48 KB of
+// slots per CTA), registers for 4 resident CTAs (32 warps) per SM - measured
+// best on B200 at prefill sizes, where it runs at the speed of a plain copy of
+// the same bytes.
+constexpr int kQkBatch = 4;
+constexpr int kQkRing = 3;
 constexpr int kQkMinBlocks = 4;
 
 template <typename T, int L, int VPL, int CH>
@@ -260,10 +299,10 @@ cudaError_t launch_head_gate_t(const HeadGateArgs& a, cudaStream_t s) {
     return launch_head_gate_l<T, 16, 1, 2>(a, s);
 }
 
-template <typename T, int L, int VPL, bool ROPE, bool UPCAST>
+template <typename T, int L, bool ROPE, bool UPCAST>
 cudaError_t launch_qk_l(const QkArgs& a0, cudaStream_t s) {
     constexpr int RW = 32 / L;
-    constexpr int BATCH = 4;
+    constexpr int BATCH = kQkBatch;
     QkArgs a = a0;
     const int nwarps = kThreads / 32;
     const int nst_q = (a.hq + RW - 1) / RW, nst_k = (a.hkv + RW - 1) / RW;
@@ -275,37 +314,42 @@ cudaError_t launch_qk_l(const QkArgs& a0, cudaStream_t s) {
         split *= 2;
     a.split = split;
     const int tt = nwarps / split;
-    const size_t smem = ROPE ? sizeof(float) * 2 * tt * (a.head_dim / 2) : 0;
+    const uint32_t head_bytes = (uint32_t)a.head_dim * (uint32_t)sizeof(T);
+    const size_t table = ((size_t)2 * tt * (a.head_dim / 2) * 4 + 127) & ~(size_t)127;
+    const size_t slot = ((size_t)BATCH * RW * head_bytes + 127) & ~(size_t)127;
+    const size_t smem = table + (size_t)nwarps * kQkRing * slot;
     const int64_t grid = (a.tokens + tt - 1) / tt;
-    const bool exact = split == 1 && a.head_dim / Vec<T>::N == L * VPL && a.hq % RW == 0 &&
+    const bool exact = split == 1 && a.head_dim / Vec<T>::N == L && a.hq % RW == 0 &&
                        a.hkv % RW == 0 && nst_q % BATCH == 0 && nst_k % BATCH == 0;
-    if (exact)
-        return launch_pdl(qk_norm_rope_kernel<T, L, VPL, ROPE, UPCAST, false, BATCH, kQkMinBlocks>,
-                          (unsigned)grid, kThreads, smem, s, a);
-    return launch_pdl(qk_norm_rope_kernel<T, L, VPL, ROPE, UPCAST, true, BATCH, kQkMinBlocks>,
-                      (unsigned)grid, kThreads, smem, s, a);
-}
-
-template <typename T, int L, int VPL>
-cudaError_t launch_qk_modes(int use_rope, int upcast, const QkArgs& a, cudaStream_t s) {
-    if (!use_rope) return launch_qk_l<T, L, VPL, false, true>(a, s);
-    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-        if (!upcast) return launch_qk_l<T, L, VPL, true, false>(a, s);
+    auto kern = exact ? qk_norm_rope_kernel<T, L, ROPE, UPCAST, false, BATCH, kQkRing, kQkMinBlocks>
+                      : qk_norm_rope_kernel<T, L, ROPE, UPCAST, true, BATCH, kQkRing, kQkMinBlocks>;
+    if (smem > 48 * 1024) {
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
     }
-    return launch_qk_l<T, L, VPL, true, true>(a, s);
+    return launch_pdl(kern, (unsigned)grid, kThreads, smem, s, a);
 }
 
+template <typename T, int L>
+cudaError_t launch_qk_modes(int use_rope, int upcast, const QkArgs& a, cudaStream_t s) {
+    if (!use_rope) return launch_qk_l<T, L, false, true>(a, s);
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        if (!upcast) return launch_qk_l<T, L, true, false>(a, s);
+    }
+    return launch_qk_l<T, L, true, true>(a, s);
+}
+
+// Lanes per head: the head's 16-byte vectors rounded up to a power of two
+// (heads are at most 512 bytes, so one vector per lane always suffices).
 template <typename T>
 cudaError_t launch_qk_t(int use_rope, int upcast, const QkArgs& a, cudaStream_t s) {
-    // one 16-byte vector per lane per head (measured best at head_dim 128);
-    // two for heads of more than 32 vectors
     const int nv = a.head_dim / Vec<T>::N;
-    if (nv > 16) return launch_qk_modes<T, 32, 1>(use_rope, upcast, a, s);
-    if (nv <= 1) return launch_qk_modes<T, 1, 1>(use_rope, upcast, a, s);
-    if (nv <= 2) return launch_qk_modes<T, 2, 1>(use_rope, upcast, a, s);
-    if (nv <= 4) return launch_qk_modes<T, 4, 1>(use_rope, upcast, a, s);
-    if (nv <= 8) return launch_qk_modes<T, 8, 1>(use_rope, upcast, a, s);
-    return launch_qk_modes<T, 16, 1>(use_rope, upcast, a, s);
+    if (nv > 16) return launch_qk_modes<T, 32>(use_rope, upcast, a, s);
+    if (nv <= 1) return launch_qk_modes<T, 1>(use_rope, upcast, a, s);
+    if (nv <= 2) return launch_qk_modes<T, 2>(use_rope, upcast, a, s);
+    if (nv <= 4) return launch_qk_modes<T, 4>(use_rope, upcast, a, s);
+    if (nv <= 8) return launch_qk_modes<T, 8>(use_rope, upcast, a, s);
+    return launch_qk_modes<T, 16>(use_rope, upcast, a, s);
 }
 
 }  // namespace
@@ -318,6 +362,15 @@ cudaError_t launch_qk(int dtype, int use_rope, int upcast_rope, const QkArgs& a,
     // FP32 tensors rotate in FP32 in both modes.
     if (dtype != 0) return launch_qk_t<float>(use_rope, 1, a, s);
     return launch_qk_t<__nv_bfloat16>(use_rope, upcast_rope, a, s);
+}
+
+cudaError_t read_qk_device_error(unsigned int* out, bool clear) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_device_error, sizeof(unsigned int));
+    if (e == cudaSuccess && clear) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
+    }
+    return e;
 }
 
 }  // namespace muse

@@ -69,8 +69,11 @@ struct QkArgs {
 // launch_row_regs (register-staged, row_norm.cu) for rows too wide to stage.
 cudaError_t launch_row(int dtype, RowOp op, const RowArgs& a, cudaStream_t s);
 cudaError_t launch_row_regs(int dtype, RowOp op, const RowArgs& a, cudaStream_t s);
-// Device-side error word (bit 0: a bounded mbarrier wait timed out).
+// Device-side error words: nonzero once a bounded mbarrier wait of the row
+// pipeline (read_device_error) or of the Q/K ring (read_qk_device_error)
+// timed out.
 cudaError_t read_device_error(unsigned int* out, bool clear);
+cudaError_t read_qk_device_error(unsigned int* out, bool clear);
 cudaError_t launch_head_gate(int dtype, const HeadGateArgs& a, cudaStream_t s);
 cudaError_t launch_qk(int dtype, int use_rope, int upcast_rope, const QkArgs& a, cudaStream_t s);
 cudaError_t launch_copy(const void* src, void* dst, int64_t bytes, cudaStream_t s);

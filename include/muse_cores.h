@@ -160,13 +160,14 @@ muse_status muse_norm_residual(const float* stream_in, const void* branch, float
                                int input_scale, float norm_eps, cudaStream_t stream);
 
 /*
- * Device-side error word of the current device, for diagnostics.  The row
- * kernels stream rows through shared memory with bulk copies tracked by
- * mbarriers; every wait on one is bounded, and a wait that gives up sets bit 0
- * of this word (and the affected kernel stops writing).  *flags receives the
- * word; clear != 0 resets it.  Synchronous: it waits for the device.  Returns
- * MUSE_ERR_INVALID_ARGUMENT for a NULL flags pointer, MUSE_ERR_CUDA if the
- * copy fails.
+ * Device-side error flags of the current device, for diagnostics.  The row
+ * kernels (cores 1, 2, 5, core 4 per token) and the Q/K kernel (core 3) stream
+ * their inputs through shared memory with bulk copies tracked by mbarriers;
+ * every wait on one is bounded, and a wait that gives up sets bit 0 (row
+ * kernels) or bit 1 (Q/K kernel) of the flags (and the affected warps stop
+ * writing).  *flags receives them; clear != 0 resets them.  Synchronous: it
+ * waits for the device.  Returns MUSE_ERR_INVALID_ARGUMENT for a NULL flags
+ * pointer, MUSE_ERR_CUDA if the copy fails.
  */
 muse_status muse_device_error(unsigned int* flags, int clear);
 
