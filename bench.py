@@ -203,6 +203,38 @@ class Step:
         return list(self.out.values())
 
 
+def per_core_isolated(st: "Step", peak: float, flush: torch.Tensor | None, warmup: int = 10,
+                      reps: int = 50):
+    """Each core launched alone: `warmup` launches, then the median of `reps`
+    launches timed with CUDA events around each one on the launching stream.
+    With `flush`, a read pass over that buffer (> L2, reading leaves no dirty
+    lines) precedes every launch, so each launch starts from a clean, cold L2;
+    without it, L2 stays warm (the decode latency figures)."""
+    stream = torch.cuda.current_stream()
+    out = {}
+    for c in CORE_ORDER:
+        ev = []
+        torch.cuda.synchronize()
+        # hold the GPU for a few ms so that the host queues every launch ahead
+        # of the device: the events then time the kernels, not the host
+        torch.cuda._sleep(20_000_000)
+        for i in range(warmup + reps):
+            if flush is not None:
+                flush.amax()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            st.launch(c)
+            e1.record(stream)
+            if i >= warmup:
+                ev.append((e0, e1))
+        torch.cuda.synchronize()
+        us = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+        nb = algo_bytes(st.wl, c, st.T)
+        gbs = nb / (us * 1e-6) / 1e9
+        out[c] = {"us": round(us, 3), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+    return out
+
+
 def time_copy_kernel(gib: float = 1.0, reps: int = 10) -> float:
     n = int(gib * (1 << 30)) // 16 * 16
     src = torch.empty(n, dtype=torch.uint8, device="cuda")
@@ -331,6 +363,18 @@ def run_ours(args, world, rank, local):
                 "kernel": KERNEL_NAMES[DOMINANT], "peak_source": peak_kind,
                 "algo_bytes_per_launch": dom["algo_bytes"]}
 
+    # Each core alone on the same batch, L2 read-flushed before every launch;
+    # and the decode batch (128 tokens), whose launches are latency-bound.
+    flush = torch.empty(64 << 20, dtype=torch.int64, device="cuda").fill_(1)  # 512 MiB
+    isolated = per_core_isolated(st, peak, flush)
+    dec = Step(WORKLOADS["decode_t128_h4096"], seed=rank)
+    decode_cold = per_core_isolated(dec, peak, flush)
+    decode_warm = per_core_isolated(dec, peak, None)
+    decode = {c: {"us_cold_l2": decode_cold[c]["us"], "us_warm_l2": decode_warm[c]["us"]}
+              for c in CORE_ORDER}
+    del flush, dec
+    torch.cuda.empty_cache()
+
     e2e = run_e2e(st, args, world) if args.e2e else None
 
     cpu = None
@@ -349,13 +393,18 @@ def run_ours(args, world, rank, local):
                        "l2": "no flush: each step streams %.2f GB, > 126 MB L2"
                              % (sum(algo_bytes(wl, c, T) for c in CORE_ORDER) / 1e9)},
             "per_core": per_core,
+            "per_core_isolated": isolated,
+            "decode_t128_h4096_latency": decode,
             "roofline": roofline,
             "copy_kernel_gbs": None if copy_gbs is None else round(copy_gbs, 1),
             "e2e": e2e,
             "cpu_baseline": cpu,
             "gpu_launches": len(CORE_ORDER) * args.steps,
             "kernel_timing": "per_core and roofline: a second pass of the same K steps with "
-                             "CUDA events around each launch (the timed region has none)",
+                             "CUDA events around each launch (the timed region has none); "
+                             "per_core_isolated: each core alone, median of 50 launches, "
+                             "a 512 MiB read pass (clean L2) before each; decode latency: "
+                             "median of 50, cold (read-flushed) and warm L2",
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

@@ -335,10 +335,11 @@ cudaError_t launch_row_tma_v(const RowArgs& a, int nvec, int stages, cudaStream_
 }
 
 // Launch shape, measured on B200 at prefill sizes (H = 4096): two or three
-// stages per CTA and as many CTAs per SM as fit beat deeper rings (3 to 4
-// CTAs of 256 consumers for 8 KB rows: 91% of the HBM copy bandwidth; 2 CTAs
-// for core 5's 24 KB rows: 93%).  Core 5 keeps at most 2 slots per consumer
-// thread (its 24 per-slot constants live in registers).
+// stages per CTA and as many CTAs per SM as fit beat deeper rings (4 CTAs of
+// 256 consumers for 8 KB rows; 2 CTAs of 512 consumers, one slot each, for
+// core 5's 24 KB rows - ahead of 256 consumers x 2 slots inside the five-core
+// step).  Core 5 keeps at most 2 slots per consumer thread (its 24 per-slot
+// constants live in registers).
 constexpr uint32_t kRingMaxBytes = 200 * 1024;
 constexpr int kConsumers = 256;
 
@@ -352,7 +353,7 @@ cudaError_t launch_row_op(const RowArgs& a, cudaStream_t s) {
     const bool g = a.gain != nullptr;
     // slots per consumer thread: the fewest that fit a row into kConsumers
     // threads (core 5: at most 2 slots, up to twice the consumers)
-    if (nvec <= kConsumers)
+    if (nvec <= kConsumers || (t_is_residual(OP) && nvec <= 2 * kConsumers))
         return g ? launch_row_tma_v<T, OP, 1, true>(a, nvec, stages, s) : launch_row_tma_v<T, OP, 1, false>(a, nvec, stages, s);
     if (nvec <= 2 * kConsumers || (t_is_residual(OP) && nvec <= 4 * kConsumers))
         return g ? launch_row_tma_v<T, OP, 2, true>(a, nvec, stages, s) : launch_row_tma_v<T, OP, 2, false>(a, nvec, stages, s);
