@@ -299,6 +299,59 @@ def cpu_baseline(wl, seconds: float = 12.0, chunk: int = 256):
                       f"{el:.1f} s single-threaded double-precision oracle"}
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline_threads(wl, seconds: float = 8.0, chunk: int = 64, threads: int | None = None):
+    """The same oracle over row chunks on all host cores: threads pull chunks
+    of `chunk` tokens from a shared counter (the oracle's C routines run
+    without the interpreter lock), all five cores per chunk, until `seconds`
+    elapse or the batch is done."""
+    import threading
+
+    import numpy as np
+
+    from tests import harness
+
+    n = threads or min(os.cpu_count() or 1, 128)
+    host = {c: harness.make(wl.name, c, harness.DEFAULT_VARIANT[c]) for c in CORE_ORDER}
+    T = num_tokens(wl)
+    lock = threading.Lock()
+    state = {"next": 0, "done": 0}
+    t0 = time.perf_counter()
+
+    def work():
+        while time.perf_counter() - t0 < seconds:
+            with lock:
+                lo = state["next"]
+                if lo >= T:
+                    return
+                state["next"] = min(T, lo + chunk)
+            rows = np.arange(lo, min(T, lo + chunk))
+            for c in CORE_ORDER:
+                harness.run_oracle(wl.name, c, host[c], rows)
+            with lock:
+                state["done"] += len(rows)
+
+    ts = [threading.Thread(target=work) for _ in range(n)]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+    el = time.perf_counter() - t0
+    return {"value": state["done"] / el, "unit": "tokens/s", "cores": n, "kind": "oracle",
+            "cpu_model": cpu_model(),
+            "sample": f"{state['done']} of {T} tokens of {wl.name}, all five cores, {el:.1f} s, "
+                      f"double-precision oracle over {chunk}-token chunks on {n} threads"}
+
+
 def run_ours(args, world, rank, local):
     wl = WORKLOADS[args.workload]
     torch.manual_seed(0)
@@ -377,9 +430,10 @@ def run_ours(args, world, rank, local):
 
     e2e = run_e2e(st, args, world) if args.e2e else None
 
-    cpu = None
+    cpu = cpu_par = None
     if rank == 0 and world == 1 and args.cpu_baseline:
         cpu = cpu_baseline(wl)
+        cpu_par = cpu_baseline_threads(wl)
     barrier(world)
     if rank == 0:
         line = {
@@ -399,6 +453,7 @@ def run_ours(args, world, rank, local):
             "copy_kernel_gbs": None if copy_gbs is None else round(copy_gbs, 1),
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "cpu_baseline_all_cores": cpu_par,
             "gpu_launches": len(CORE_ORDER) * args.steps,
             "kernel_timing": "per_core and roofline: a second pass of the same K steps with "
                              "CUDA events around each launch (the timed region has none); "
