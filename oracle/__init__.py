@@ -64,9 +64,23 @@ def _load():
                 c_int, P, P, i64, i32, i32, i32, f32, P, P, P, P]
             lib.muse_oracle_norm_residual.argtypes = [
                 P, c_int, P, i64, i64, P, f32, P, c_int, f32, P, P, P, P]
+            lib.muse_oracle_rms_norm_bwd.argtypes = [c_int, P, P, i64, i64, P, f32, f32,
+                                                     P, P, P, P, P, P, P]
+            lib.muse_oracle_input_scale_norm_bwd.argtypes = lib.muse_oracle_rms_norm_bwd.argtypes
+            lib.muse_oracle_qk_norm_rope_bwd.argtypes = [
+                c_int, P, P, P, P, i64, i32, i32, i32, P, f32, f32, c_int, f32, c_int,
+                P, P, P, P, P, P, P, P]
+            lib.muse_oracle_output_norm_gate_bwd.argtypes = [
+                c_int, P, P, P, i64, i32, i32, i32, f32, P, P, P, P, P, P, P, P]
+            lib.muse_oracle_norm_residual_bwd.argtypes = [
+                P, c_int, P, P, i64, i64, P, f32, P, c_int, f32, c_int,
+                P, P, P, P, P, P, P, P, P, P, P, P, P, P]
             for name in ("muse_oracle_inv_freq", "muse_oracle_positions", "muse_oracle_rms_norm",
                          "muse_oracle_input_scale_norm", "muse_oracle_qk_norm_rope",
-                         "muse_oracle_output_norm_gate", "muse_oracle_norm_residual"):
+                         "muse_oracle_output_norm_gate", "muse_oracle_norm_residual",
+                         "muse_oracle_rms_norm_bwd", "muse_oracle_input_scale_norm_bwd",
+                         "muse_oracle_qk_norm_rope_bwd", "muse_oracle_output_norm_gate_bwd",
+                         "muse_oracle_norm_residual_bwd"):
                 getattr(lib, name).restype = c_int
             _lib = lib
     return _lib
@@ -208,3 +222,94 @@ def norm_residual(stream, branch, theta, gain=None, gain_offset=0.0, input_scale
         _ptr(theta), int(input_scale), norm_eps, _ptr(out), _ptr(lo), _ptr(hi), _ptr(mag)),
         "norm_residual")
     return out, lo, hi, mag
+
+
+# ------------------------------------------------------------------ backward
+# Each returns the input gradients as (out, lo, hi, mag) tuples and the
+# parameter gradients as (lo, hi, mag) double triples (None without a gain).
+
+
+def _rows_bwd(fn, what, x, dy, gain, gain_offset, eps):
+    x = _c(x)
+    dy = _c(dy)
+    gain = _c(gain)
+    assert dy.shape == x.shape and dy.dtype == x.dtype
+    hidden = x.shape[-1]
+    rows = x.size // hidden
+    dx = np.empty_like(x)
+    lo, hi, mag = _checks(x.shape)
+    glo, ghi, gmag = _checks((hidden,)) if gain is not None else (None, None, None)
+    _check(fn(_dt(x), _ptr(x), _ptr(dy), rows, hidden, _ptr(gain), gain_offset, eps, _ptr(dx),
+              _ptr(lo), _ptr(hi), _ptr(mag), _ptr(glo), _ptr(ghi), _ptr(gmag)), what)
+    return (dx, lo, hi, mag), (None if gain is None else (glo, ghi, gmag))
+
+
+def rms_norm_bwd(x, dy, gain=None, gain_offset=0.0, eps=1e-6):
+    """Core 1 backward: (dx, dgain)."""
+    return _rows_bwd(_load().muse_oracle_rms_norm_bwd, "rms_norm_bwd", x, dy, gain, gain_offset,
+                     eps)
+
+
+def input_scale_norm_bwd(x, dy, gain=None, gain_offset=0.0, eps=1e-6):
+    """Core 2 backward: (dx, dgain)."""
+    return _rows_bwd(_load().muse_oracle_input_scale_norm_bwd, "input_scale_norm_bwd", x, dy,
+                     gain, gain_offset, eps)
+
+
+def qk_norm_rope_bwd(q, k, dq_out, dk_out, pos, eps=1e-6, query_scale=1.0, use_rope=True,
+                     rope_base=10000.0, round_grads=True):
+    """Core 3 backward (FP32 rotation): (dq, dk)."""
+    q, k, dq_out, dk_out = _c(q), _c(k), _c(dq_out), _c(dk_out)
+    pos = None if pos is None else np.ascontiguousarray(pos, dtype=np.int32)
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    assert dq_out.shape == q.shape and dk_out.shape == k.shape
+    dq = np.empty_like(q)
+    dk = np.empty_like(k)
+    ql, qh, qm = _checks(q.shape)
+    kl, kh, km = _checks(k.shape)
+    _check(_load().muse_oracle_qk_norm_rope_bwd(
+        _dt(q), _ptr(q), _ptr(k), _ptr(dq_out), _ptr(dk_out), T, hq, hkv, d, _ptr(pos), eps,
+        query_scale, int(use_rope), rope_base, int(round_grads), _ptr(dq), _ptr(ql), _ptr(qh),
+        _ptr(qm), _ptr(dk), _ptr(kl), _ptr(kh), _ptr(km)), "qk_norm_rope_bwd")
+    return (dq, ql, qh, qm), (dk, kl, kh, km)
+
+
+def output_norm_gate_bwd(o, g, dy, norm_group=None, eps=1e-6):
+    """Core 4 backward: (do, dg)."""
+    o, g, dy = _c(o), _c(g), _c(dy)
+    T, heads, d = o.shape
+    ng = d if norm_group is None else norm_group
+    d_o = np.empty_like(o)
+    dg = np.empty_like(o)
+    ol, oh, om = _checks(o.shape)
+    gl, gh, gm = _checks(o.shape)
+    _check(_load().muse_oracle_output_norm_gate_bwd(
+        _dt(o), _ptr(o), _ptr(g), _ptr(dy), T, heads, d, ng, eps, _ptr(d_o), _ptr(ol), _ptr(oh),
+        _ptr(om), _ptr(dg), _ptr(gl), _ptr(gh), _ptr(gm)), "output_norm_gate_bwd")
+    return (d_o, ol, oh, om), (dg, gl, gh, gm)
+
+
+def norm_residual_bwd(stream, branch, dstream_out, theta, gain=None, gain_offset=0.0,
+                      input_scale=False, norm_eps=1e-6, round_grads=True):
+    """Core 5 backward: (dstream, dbranch, dgain, dtheta)."""
+    stream = np.ascontiguousarray(stream, dtype=np.float32)
+    dstream_out = np.ascontiguousarray(dstream_out, dtype=np.float32)
+    branch = _c(branch)
+    theta = np.ascontiguousarray(theta, dtype=np.float32)
+    gain = _c(gain)
+    hidden = stream.shape[-1]
+    rows = stream.size // hidden
+    ds = np.empty_like(stream)
+    db = np.empty_like(branch)
+    sl, sh, sm = _checks(stream.shape)
+    bl, bh, bm = _checks(stream.shape)
+    glo, ghi, gmag = _checks((hidden,)) if gain is not None else (None, None, None)
+    tlo, thi, tmag = _checks((hidden,))
+    _check(_load().muse_oracle_norm_residual_bwd(
+        _ptr(stream), _dt(branch), _ptr(branch), _ptr(dstream_out), rows, hidden, _ptr(gain),
+        gain_offset, _ptr(theta), int(input_scale), norm_eps, int(round_grads), _ptr(ds),
+        _ptr(sl), _ptr(sh), _ptr(sm), _ptr(db), _ptr(bl), _ptr(bh), _ptr(bm), _ptr(glo),
+        _ptr(ghi), _ptr(gmag), _ptr(tlo), _ptr(thi), _ptr(tmag)), "norm_residual_bwd")
+    return ((ds, sl, sh, sm), (db, bl, bh, bm), None if gain is None else (glo, ghi, gmag),
+            (tlo, thi, tmag))

@@ -430,3 +430,369 @@ int muse_oracle_norm_residual(const float* stream, int branch_dtype, const void*
     }
     return 0;
 }
+
+/* ================================================================ backward
+ *
+ * The cores run under autograd (the page's _checkpoint_recomputed_math keeps
+ * them outside checkpoint caching while "autograd ... still run[s]").  Their
+ * backward is therefore the derivative of the forward map above, evaluated
+ * from the saved forward inputs with r recomputed, where every dtype boundary
+ * the forward materialises passes the gradient through and rounds it to that
+ * tensor's dtype (the gradient of a cast is the incoming gradient cast back):
+ *   - the output cast of each core: dy arrives in the output dtype;
+ *   - core 3: the gradient of the normalised Q/K (and of the scaled query) is
+ *     rounded to the Q/K dtype;
+ *   - core 5: the gradient of the cast branch nb is rounded to the branch
+ *     dtype;
+ *   - input gradients are cast once to the input dtype; parameter gradients
+ *     (gain, theta) are FP32 sums over all rows.
+ * round_grads = 0 drops the intermediate roundings (the exact derivative;
+ * used by the pins).
+ *
+ * Check arrays: as for the forward, lo/hi bracket the exact pre-cast value
+ * over the admissible values of every intermediate cast (forward casts whose
+ * values enter the gradient, and gradient casts), and mag is the sum of the
+ * magnitudes of the terms of the last expression, with each inner sum
+ * counted by the magnitudes of its own terms.  Parameter gradients come as
+ * [lo, hi] and mag over the row sum.
+ */
+
+typedef struct {
+    double lo, hi, rn; /* bracket and the round-to-nearest path value */
+} ival;
+
+static ival iv_exact(double v) { ival r = {v, v, v}; return r; }
+
+static ival iv_cast(int dtype, double v, int round) {
+    if (!round) return iv_exact(v);
+    double c[2];
+    const int n = cast_candidates(dtype, v, c);
+    ival r = {c[0], c[0], c[0]};
+    if (n == 2) { r.lo = fmin(c[0], c[1]); r.hi = fmax(c[0], c[1]); }
+    return r;
+}
+
+/* interval times a real scalar */
+static ival iv_scale(ival a, double s) {
+    ival r;
+    r.rn = a.rn * s;
+    const double p = a.lo * s, q = a.hi * s;
+    r.lo = fmin(p, q);
+    r.hi = fmax(p, q);
+    return r;
+}
+
+static ival iv_add(ival a, ival b) {
+    ival r = {a.lo + b.lo, a.hi + b.hi, a.rn + b.rn};
+    return r;
+}
+
+static double iv_absmax(ival a) { return fmax(fabs(a.lo), fabs(a.hi)); }
+
+/* Gradient of one normalised row.  mode 0 (core 1 form): y = x r(x) w;
+ * mode 1 (core 2 form): z = x w, y = z r(z).  g = dL/dy per element (an
+ * interval when it passed a rounded cast).  Fills dx (interval + mag) and, if
+ * dw_term is not NULL, each row's term of the gain gradient.
+ *   mode 0: dx_k = r w_k g_k - r^3 x_k C / H,  C = sum_j g_j w_j x_j;
+ *           dW_k += g_k x_k r
+ *   mode 1: dz_k = r g_k - r^3 z_k C / H,      C = sum_j g_j z_j;
+ *           dx_k = dz_k w_k;                    dW_k += dz_k x_k */
+static void norm_row_bwd(int mode, int64_t H, const double* x, const double* w, float eps,
+                         const ival* g, ival* dx, double* dx_mag, ival* dw_term,
+                         double* dw_mag) {
+    double ss = 0.0;
+    for (int64_t j = 0; j < H; ++j) {
+        const double u = mode ? x[j] * w[j] : x[j];
+        ss += u * u;
+    }
+    const double r = inv_rms(ss, H, eps);
+    const double r3 = r * r * r;
+    ival C = iv_exact(0.0);
+    double Cabs = 0.0;
+    for (int64_t j = 0; j < H; ++j) {
+        const double f = mode ? x[j] * w[j] : w[j] * x[j];
+        C = iv_add(C, iv_scale(g[j], f));
+        Cabs += iv_absmax(g[j]) * fabs(f);
+    }
+    for (int64_t k = 0; k < H; ++k) {
+        const double u = mode ? x[k] * w[k] : x[k];
+        const double a = mode ? r : r * w[k];
+        ival d = iv_add(iv_scale(g[k], a), iv_scale(C, -r3 * u / (double)H));
+        double m = iv_absmax(g[k]) * fabs(a) + r3 * fabs(u) * Cabs / (double)H;
+        if (mode) {
+            if (dw_term) {
+                dw_term[k] = iv_scale(d, x[k]);
+                dw_mag[k] = m * fabs(x[k]);
+            }
+            d = iv_scale(d, w[k]);
+            m *= fabs(w[k]);
+        } else if (dw_term) {
+            dw_term[k] = iv_scale(g[k], x[k] * r);
+            dw_mag[k] = iv_absmax(g[k]) * fabs(x[k] * r);
+        }
+        dx[k] = d;
+        dx_mag[k] = m;
+    }
+}
+
+static void acc_param(double* lo, double* hi, double* mag, int64_t k, ival t, double m) {
+    if (lo) lo[k] += t.lo;
+    if (hi) hi[k] += t.hi;
+    if (mag) mag[k] += m;
+}
+
+static void zero_n(double* p, int64_t n) {
+    if (p) memset(p, 0, sizeof(double) * (size_t)n);
+}
+
+static int rows_bwd(int mode, int dtype, const void* x, const void* dy, int64_t rows,
+                    int64_t hidden, const float* gain, float gain_offset, float eps, void* dx,
+                    double* lo, double* hi, double* mag, double* dgain_lo, double* dgain_hi,
+                    double* dgain_mag) {
+    if (!valid_dtype(dtype) || rows < 0 || hidden <= 0 || (rows && (!x || !dy || !dx))) return -1;
+    double* xv = (double*)malloc(sizeof(double) * (size_t)hidden * 3);
+    ival* g = (ival*)malloc(sizeof(ival) * (size_t)hidden * 3);
+    double* dm = (double*)malloc(sizeof(double) * (size_t)hidden * 2);
+    if (!xv || !g || !dm) { free(xv); free(g); free(dm); return -1; }
+    double* w = xv + hidden;
+    ival* d = g + hidden;
+    ival* wt = g + 2 * hidden;
+    double* wm = dm + hidden;
+    for (int64_t j = 0; j < hidden; ++j) w[j] = eff_gain(gain, gain_offset, j);
+    zero_n(dgain_lo, hidden);
+    zero_n(dgain_hi, hidden);
+    zero_n(dgain_mag, hidden);
+    for (int64_t r = 0; r < rows; ++r) {
+        const int64_t base = r * hidden;
+        for (int64_t j = 0; j < hidden; ++j) {
+            xv[j] = load_elem(dtype, x, base + j);
+            g[j] = iv_exact(load_elem(dtype, dy, base + j));
+        }
+        norm_row_bwd(mode, hidden, xv, w, eps, g, d, dm, gain ? wt : NULL, wm);
+        for (int64_t j = 0; j < hidden; ++j) {
+            store_elem(dtype, dx, base + j, d[j].rn);
+            put_check(lo, hi, mag, base + j, d[j].lo, d[j].hi, dm[j]);
+            if (gain) acc_param(dgain_lo, dgain_hi, dgain_mag, j, wt[j], wm[j]);
+        }
+    }
+    free(xv);
+    free(g);
+    free(dm);
+    return 0;
+}
+
+int muse_oracle_rms_norm_bwd(int dtype, const void* x, const void* dy, int64_t rows,
+                             int64_t hidden, const float* gain, float gain_offset, float eps,
+                             void* dx, double* lo, double* hi, double* mag, double* dgain_lo,
+                             double* dgain_hi, double* dgain_mag) {
+    return rows_bwd(0, dtype, x, dy, rows, hidden, gain, gain_offset, eps, dx, lo, hi, mag,
+                    dgain_lo, dgain_hi, dgain_mag);
+}
+
+int muse_oracle_input_scale_norm_bwd(int dtype, const void* x, const void* dy, int64_t rows,
+                                     int64_t hidden, const float* gain, float gain_offset,
+                                     float eps, void* dx, double* lo, double* hi, double* mag,
+                                     double* dgain_lo, double* dgain_hi, double* dgain_mag) {
+    return rows_bwd(1, dtype, x, dy, rows, hidden, gain, gain_offset, eps, dx, lo, hi, mag,
+                    dgain_lo, dgain_hi, dgain_mag);
+}
+
+/* sigmoid'(v) = e^-|v| / (1 + e^-|v|)^2 (the form without cancellation). */
+static double dsigmoid(double v) {
+    const double t = exp(-fabs(v));
+    return t / ((1.0 + t) * (1.0 + t));
+}
+
+int muse_oracle_output_norm_gate_bwd(int dtype, const void* o, const void* g, const void* dy,
+                                     int64_t tokens, int32_t heads, int32_t head_dim,
+                                     int32_t norm_group, float eps, void* d_o, double* do_lo,
+                                     double* do_hi, double* do_mag, void* dg, double* dg_lo,
+                                     double* dg_hi, double* dg_mag) {
+    if (!valid_dtype(dtype) || tokens < 0 || heads <= 0 || head_dim <= 0) return -1;
+    const int64_t width = (int64_t)heads * head_dim;
+    if (norm_group != head_dim && norm_group != width) return -1;
+    if (tokens && (!o || !g || !dy || !d_o || !dg)) return -1;
+    double* ov = (double*)malloc(sizeof(double) * (size_t)norm_group * 3);
+    ival* gr = (ival*)malloc(sizeof(ival) * (size_t)norm_group * 2);
+    if (!ov || !gr) { free(ov); free(gr); return -1; }
+    double* one = ov + norm_group;
+    double* dm = ov + 2 * (int64_t)norm_group;
+    ival* dd = gr + norm_group;
+    for (int32_t j = 0; j < norm_group; ++j) one[j] = 1.0;
+    const int64_t groups = tokens * width / norm_group;
+    for (int64_t gi = 0; gi < groups; ++gi) {
+        const int64_t base = gi * norm_group;
+        double ss = 0.0;
+        for (int32_t j = 0; j < norm_group; ++j) {
+            ov[j] = load_elem(dtype, o, base + j);
+            ss += ov[j] * ov[j];
+        }
+        const double r = inv_rms(ss, norm_group, eps);
+        for (int32_t j = 0; j < norm_group; ++j) {
+            const double gv = load_elem(dtype, g, base + j);
+            const double dyv = load_elem(dtype, dy, base + j);
+            const double s = 1.0 / (1.0 + exp(-gv));
+            gr[j] = iv_exact(dyv * s); /* dL/dn, n = o r */
+            const double dgv = dyv * ov[j] * r * dsigmoid(gv);
+            store_elem(dtype, dg, base + j, dgv);
+            put_check(dg_lo, dg_hi, dg_mag, base + j, dgv, dgv, fabs(dgv));
+        }
+        norm_row_bwd(0, norm_group, ov, one, eps, gr, dd, dm, NULL, NULL);
+        for (int32_t j = 0; j < norm_group; ++j) {
+            store_elem(dtype, d_o, base + j, dd[j].rn);
+            put_check(do_lo, do_hi, do_mag, base + j, dd[j].lo, dd[j].hi, dm[j]);
+        }
+    }
+    free(ov);
+    free(gr);
+    return 0;
+}
+
+int muse_oracle_norm_residual_bwd(const float* stream, int branch_dtype, const void* branch,
+                                  const float* dstream_out, int64_t rows, int64_t hidden,
+                                  const float* gain, float gain_offset, const float* theta,
+                                  int input_scale, float norm_eps, int round_grads,
+                                  float* dstream, double* ds_lo, double* ds_hi, double* ds_mag,
+                                  void* dbranch, double* db_lo, double* db_hi, double* db_mag,
+                                  double* dgain_lo, double* dgain_hi, double* dgain_mag,
+                                  double* dtheta_lo, double* dtheta_hi, double* dtheta_mag) {
+    if (!valid_dtype(branch_dtype) || rows < 0 || hidden <= 0) return -1;
+    if (rows && (!stream || !branch || !dstream_out || !theta || !dstream || !dbranch)) return -1;
+    double* bv = (double*)malloc(sizeof(double) * (size_t)hidden * 4);
+    ival* gr = (ival*)malloc(sizeof(ival) * (size_t)hidden * 3);
+    if (!bv || !gr) { free(bv); free(gr); return -1; }
+    double* w = bv + hidden;
+    double* dm = bv + 2 * hidden;
+    double* wm = bv + 3 * hidden;
+    ival* dd = gr + hidden;
+    ival* wt = gr + 2 * hidden;
+    const int mode = input_scale ? 1 : 0;
+    for (int64_t j = 0; j < hidden; ++j) w[j] = eff_gain(gain, gain_offset, j);
+    zero_n(dgain_lo, hidden);
+    zero_n(dgain_hi, hidden);
+    zero_n(dgain_mag, hidden);
+    zero_n(dtheta_lo, hidden);
+    zero_n(dtheta_hi, hidden);
+    zero_n(dtheta_mag, hidden);
+    for (int64_t r = 0; r < rows; ++r) {
+        const int64_t base = r * hidden;
+        double ss = 0.0;
+        for (int64_t j = 0; j < hidden; ++j) {
+            bv[j] = load_elem(branch_dtype, branch, base + j);
+            const double u = mode ? bv[j] * w[j] : bv[j];
+            ss += u * u;
+        }
+        const double inv = inv_rms(ss, hidden, norm_eps);
+        for (int64_t j = 0; j < hidden; ++j) {
+            const double c = cos((double)theta[j]), s = sin((double)theta[j]);
+            const double dh = (double)dstream_out[base + j];
+            const double h = (double)stream[base + j];
+            /* dL/dh = cos(theta) dh' (FP32 output) */
+            dstream[base + j] = (float)(c * dh);
+            put_check(ds_lo, ds_hi, ds_mag, base + j, c * dh, c * dh, fabs(c * dh));
+            /* dL/dnb = sin(theta) dh', rounded to the branch dtype */
+            gr[j] = iv_cast(branch_dtype, s * dh, round_grads);
+            /* dL/dtheta = dh' (-sin(theta) h + cos(theta) nb), nb the forward's cast value */
+            const double v = mode ? (bv[j] * w[j]) * inv : (bv[j] * inv) * w[j];
+            const ival nb = iv_cast(branch_dtype, v, 1);
+            const ival t = iv_add(iv_exact(-s * h * dh), iv_scale(nb, c * dh));
+            acc_param(dtheta_lo, dtheta_hi, dtheta_mag, j, t,
+                      fabs(dh) * (fabs(s * h) + fabs(c) * iv_absmax(nb)));
+        }
+        norm_row_bwd(mode, hidden, bv, w, norm_eps, gr, dd, dm, gain ? wt : NULL, wm);
+        for (int64_t j = 0; j < hidden; ++j) {
+            store_elem(branch_dtype, dbranch, base + j, dd[j].rn);
+            put_check(db_lo, db_hi, db_mag, base + j, dd[j].lo, dd[j].hi, dm[j]);
+            if (gain) acc_param(dgain_lo, dgain_hi, dgain_mag, j, wt[j], wm[j]);
+        }
+    }
+    free(bv);
+    free(gr);
+    return 0;
+}
+
+/* Core 3 backward, FP32 (legacy) rotation.  Per head:
+ *   dm = R(phi)^T dy                     (FP32: da = c dy0 + s dy1, db = -s dy0 + c dy1)
+ *   dn2 = cast(dm)                       (gradient of the rotated-in value, Q/K dtype)
+ *   query heads: dn1 = cast(dn2 * query_scale); key heads: dn1 = dn2
+ *   dx = r dn1 - r^3 x (sum_j dn1_j x_j) / d, cast to the Q/K dtype. */
+static void qk_head_bwd(int dtype, const void* x, const void* dy, int64_t base, int32_t d,
+                        const float* inv_freq, int32_t pos, int use_rope, float eps,
+                        int is_query, float query_scale, int round_grads, double* xv,
+                        double* one, ival* gr, ival* dd, double* dm, void* dx, double* lo,
+                        double* hi, double* mag) {
+    for (int32_t j = 0; j < d; ++j) xv[j] = load_elem(dtype, x, base + j);
+    for (int32_t i = 0; i < d / 2; ++i) {
+        double m0, m1;
+        const double y0 = load_elem(dtype, dy, base + 2 * i);
+        const double y1 = load_elem(dtype, dy, base + 2 * i + 1);
+        if (use_rope) {
+            const float phi = (float)pos * inv_freq[i];
+            const double c = cos((double)phi), s = sin((double)phi);
+            m0 = c * y0 + s * y1;
+            m1 = -s * y0 + c * y1;
+        } else {
+            m0 = y0;
+            m1 = y1;
+        }
+        const double m[2] = {m0, m1};
+        for (int e = 0; e < 2; ++e) {
+            const ival n2 = iv_cast(dtype, m[e], round_grads);
+            ival n1 = n2;
+            if (is_query) {
+                /* each admissible dn2 scaled, then cast again */
+                const ival a = iv_cast(dtype, n2.lo * (double)query_scale, round_grads);
+                const ival b = iv_cast(dtype, n2.hi * (double)query_scale, round_grads);
+                const ival p = iv_cast(dtype, n2.rn * (double)query_scale, round_grads);
+                n1.lo = fmin(fmin(a.lo, b.lo), fmin(a.hi, b.hi));
+                n1.hi = fmax(fmax(a.lo, b.lo), fmax(a.hi, b.hi));
+                n1.rn = p.rn;
+            }
+            gr[2 * i + e] = n1;
+        }
+    }
+    norm_row_bwd(0, d, xv, one, eps, gr, dd, dm, NULL, NULL);
+    for (int32_t j = 0; j < d; ++j) {
+        store_elem(dtype, dx, base + j, dd[j].rn);
+        put_check(lo, hi, mag, base + j, dd[j].lo, dd[j].hi, dm[j]);
+    }
+}
+
+int muse_oracle_qk_norm_rope_bwd(int dtype, const void* q, const void* k, const void* dq_out,
+                                 const void* dk_out, int64_t tokens, int32_t hq, int32_t hkv,
+                                 int32_t head_dim, const int32_t* pos, float eps,
+                                 float query_scale, int use_rope, float rope_base,
+                                 int round_grads, void* dq, double* dq_lo, double* dq_hi,
+                                 double* dq_mag, void* dk, double* dk_lo, double* dk_hi,
+                                 double* dk_mag) {
+    if (!valid_dtype(dtype) || tokens < 0 || hq <= 0 || hkv <= 0 || head_dim <= 0 ||
+        (head_dim & 1))
+        return -1;
+    if (tokens && (!q || !k || !dq_out || !dk_out || !dq || !dk || (use_rope && !pos))) return -1;
+    float* inv_freq = (float*)malloc(sizeof(float) * (size_t)(head_dim / 2));
+    double* xv = (double*)malloc(sizeof(double) * (size_t)head_dim * 3);
+    ival* gr = (ival*)malloc(sizeof(ival) * (size_t)head_dim * 2);
+    if (!inv_freq || !xv || !gr) { free(inv_freq); free(xv); free(gr); return -1; }
+    if (use_rope && muse_oracle_inv_freq(head_dim, rope_base, inv_freq) != 0) {
+        free(inv_freq); free(xv); free(gr); return -1;
+    }
+    double* one = xv + head_dim;
+    double* dm = xv + 2 * (int64_t)head_dim;
+    ival* dd = gr + head_dim;
+    for (int32_t j = 0; j < head_dim; ++j) one[j] = 1.0;
+    for (int64_t t = 0; t < tokens; ++t) {
+        const int32_t p = use_rope ? pos[t] : 0;
+        for (int32_t h = 0; h < hq; ++h)
+            qk_head_bwd(dtype, q, dq_out, (t * hq + h) * (int64_t)head_dim, head_dim, inv_freq, p,
+                        use_rope, eps, 1, query_scale, round_grads, xv, one, gr, dd, dm, dq,
+                        dq_lo, dq_hi, dq_mag);
+        for (int32_t h = 0; h < hkv; ++h)
+            qk_head_bwd(dtype, k, dk_out, (t * hkv + h) * (int64_t)head_dim, head_dim, inv_freq,
+                        p, use_rope, eps, 0, 1.0f, round_grads, xv, one, gr, dd, dm, dk, dk_lo,
+                        dk_hi, dk_mag);
+    }
+    free(inv_freq);
+    free(xv);
+    free(gr);
+    return 0;
+}

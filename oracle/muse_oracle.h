@@ -119,6 +119,60 @@ int muse_oracle_norm_residual(const float* stream, int branch_dtype, const void*
                               float norm_eps, float* out, double* lo, double* hi,
                               double* mag);
 
+/* ---------------------------------------------------------------- backward
+ *
+ * Gradients of the five cores (the cores run under autograd): the derivative
+ * of each forward map, where every dtype boundary the forward materialises
+ * passes the gradient back rounded to that tensor's dtype (round_grads != 0;
+ * 0 gives the exact derivative).  Input gradients in the input dtype with
+ * lo/hi/mag as for the forward; parameter gradients (gain, theta) as [lo, hi]
+ * of the exact FP32-free row sum and the sum of the magnitudes of its terms.
+ * Any check or parameter array may be NULL.
+ *
+ * Core 1:  g = dy * w_eff;  dx = r g - r^3 x (sum_j g_j x_j) / H;
+ *          dgain = sum over rows of dy * x * r.
+ * Core 2:  z = x * w_eff;  dz = r dy - r^3 z (sum_j dy_j z_j) / H;
+ *          dx = dz * w_eff;  dgain = sum over rows of dz * x. */
+int muse_oracle_rms_norm_bwd(int dtype, const void* x, const void* dy, int64_t rows,
+                             int64_t hidden, const float* gain, float gain_offset, float eps,
+                             void* dx, double* lo, double* hi, double* mag, double* dgain_lo,
+                             double* dgain_hi, double* dgain_mag);
+int muse_oracle_input_scale_norm_bwd(int dtype, const void* x, const void* dy, int64_t rows,
+                                     int64_t hidden, const float* gain, float gain_offset,
+                                     float eps, void* dx, double* lo, double* hi, double* mag,
+                                     double* dgain_lo, double* dgain_hi, double* dgain_mag);
+
+/* Core 3, FP32 (legacy) rotation: dm = R(phi)^T dy; dn = cast(dm), query
+ * heads dn = cast(dn * query_scale); dx = r dn - r^3 x (sum_j dn_j x_j) / d. */
+int muse_oracle_qk_norm_rope_bwd(int dtype, const void* q, const void* k, const void* dq_out,
+                                 const void* dk_out, int64_t tokens, int32_t hq, int32_t hkv,
+                                 int32_t head_dim, const int32_t* pos, float eps,
+                                 float query_scale, int use_rope, float rope_base,
+                                 int round_grads, void* dq, double* dq_lo, double* dq_hi,
+                                 double* dq_mag, void* dk, double* dk_lo, double* dk_hi,
+                                 double* dk_mag);
+
+/* Core 4: s = sigmoid(g), n = o r(o); dn = dy s;
+ * do = r dn - r^3 o (sum_j dn_j o_j) / G;  dg = dy n s (1 - s). */
+int muse_oracle_output_norm_gate_bwd(int dtype, const void* o, const void* g, const void* dy,
+                                     int64_t tokens, int32_t heads, int32_t head_dim,
+                                     int32_t norm_group, float eps, void* d_o, double* do_lo,
+                                     double* do_hi, double* do_mag, void* dg, double* dg_lo,
+                                     double* dg_hi, double* dg_mag);
+
+/* Core 5: dh = cos(theta) dh';  dnb = cast_branch(sin(theta) dh');
+ * dbranch = core 1 (input_scale == 0) or core 2 backward of dnb;
+ * dgain = that backward's gain gradient;
+ * dtheta = sum over rows of dh' (-sin(theta) h + cos(theta) nb). */
+int muse_oracle_norm_residual_bwd(const float* stream, int branch_dtype, const void* branch,
+                                  const float* dstream_out, int64_t rows, int64_t hidden,
+                                  const float* gain, float gain_offset, const float* theta,
+                                  int input_scale, float norm_eps, int round_grads,
+                                  float* dstream, double* ds_lo, double* ds_hi, double* ds_mag,
+                                  void* dbranch, double* db_lo, double* db_hi, double* db_mag,
+                                  double* dgain_lo, double* dgain_hi, double* dgain_mag,
+                                  double* dtheta_lo, double* dtheta_hi, double* dtheta_mag);
+
 #ifdef __cplusplus
 }
 #endif
