@@ -230,20 +230,30 @@ def test_qk_norm_rope_bwd_matches_autograd(use_rope):
 
 
 def test_qk_norm_rope_bwd_rounded_gradient_composes():
-    # round_grads: the key gradient is the plain norm backward of
-    # bf16(R^T dy), with R the FP32-angle rotation
+    # round_grads: the key gradient is the plain norm backward of bf16(R^T dy),
+    # the query gradient that of bf16(bf16(R^T dy) * query_scale), with R the
+    # FP32-angle rotation
     rng = np.random.default_rng(11)
-    T, D, eps, base = 2, 32, 1e-6, 5e5
+    T, D, eps, base, qs = 2, 32, 1e-6, 5e5, 0.3
     qb, kb = rnd_bf16((T, 1, D), rng), rnd_bf16((T, 1, D), rng)
     dqb, dkb = rnd_bf16((T, 1, D), rng), rnd_bf16((T, 1, D), rng)
     pos = np.array([3, 4000], np.int32)
-    _, (dk, klo, khi, _) = oracle.qk_norm_rope_bwd(qb, kb, dqb, dkb, pos, eps, 1.0, True, base)
+    (dq, qlo, qhi, _), (dk, klo, khi, _) = oracle.qk_norm_rope_bwd(qb, kb, dqb, dkb, pos, eps, qs,
+                                                                    True, base)
     inv = oracle.inv_freq(D, base).astype(np.float32)
     phi = (pos.astype(np.float32)[:, None] * inv[None, :]).astype(np.float32).astype(np.float64)
-    dy = bf16_vals(dkb)[:, 0, :]
-    a, b = dy[:, 0::2], dy[:, 1::2]
-    m = np.stack([np.cos(phi) * a + np.sin(phi) * b, -np.sin(phi) * a + np.cos(phi) * b], -1)
-    dn = oracle.round_bf16(m.reshape(T, D))
+
+    def rt(dyb):
+        dy = bf16_vals(dyb)[:, 0, :]
+        a, b = dy[:, 0::2], dy[:, 1::2]
+        m = np.stack([np.cos(phi) * a + np.sin(phi) * b, -np.sin(phi) * a + np.cos(phi) * b], -1)
+        return oracle.round_bf16(m.reshape(T, D))
+
+    dn = rt(dkb)
     (dx, lo, _, _), _ = oracle.rms_norm_bwd(kb[:, 0, :], dn, None, 0.0, eps)
     assert np.array_equal(dk[:, 0, :], dx)
     assert np.all(klo[:, 0, :] <= lo) and np.all(lo <= khi[:, 0, :])
+    dn = oracle.round_bf16(bf16_vals(rt(dqb)) * qs)
+    (dx, lo, _, _), _ = oracle.rms_norm_bwd(qb[:, 0, :], dn, None, 0.0, eps)
+    assert np.array_equal(dq[:, 0, :], dx)
+    assert np.all(qlo[:, 0, :] <= lo) and np.all(lo <= qhi[:, 0, :])
