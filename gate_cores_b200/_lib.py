@@ -29,6 +29,8 @@ EXPORTS = (
     "muse_version", "muse_status_string", "muse_last_error", "muse_rms_norm",
     "muse_input_scale_norm", "muse_qk_norm_rope", "muse_output_norm_gate",
     "muse_norm_residual", "muse_device_error", "muse_stream_copy",
+    "muse_norm_backward_workspace_bytes", "muse_rms_norm_backward",
+    "muse_input_scale_norm_backward", "muse_norm_residual_backward",
 )
 
 
@@ -72,8 +74,16 @@ def load() -> ctypes.CDLL:
         lib.muse_norm_residual.argtypes = [P, P, P, c_int, i64, i64, P, f32, P, c_int, f32, P]
         lib.muse_stream_copy.argtypes = [P, P, i64, P]
         lib.muse_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), c_int]
+        sz = ctypes.c_size_t
+        lib.muse_norm_backward_workspace_bytes.argtypes = [i64, i64]
+        rbwd = [P, P, P, c_int, i64, i64, i64, i64, i64, P, f32, f32, P, P, sz, P]
+        lib.muse_rms_norm_backward.argtypes = rbwd
+        lib.muse_input_scale_norm_backward.argtypes = rbwd
+        lib.muse_norm_residual_backward.argtypes = [P, P, P, P, P, c_int, i64, i64, P, f32, P,
+                                                    c_int, f32, P, P, P, sz, P]
         for name in EXPORTS[3:]:
             getattr(lib, name).restype = c_int
+        lib.muse_norm_backward_workspace_bytes.restype = sz
         _lib = lib
         return lib
 
@@ -141,3 +151,30 @@ def muse_device_error(clear: bool = False) -> int:
 
 def muse_stream_copy(src, dst, nbytes, stream) -> None:
     _call("muse_stream_copy", src, dst, nbytes, stream)
+
+
+def muse_norm_backward_workspace_bytes(rows, hidden) -> int:
+    return load().muse_norm_backward_workspace_bytes(rows, hidden)
+
+
+def muse_rms_norm_backward(x, dy, dx, dtype, rows, hidden, x_row_stride, dy_row_stride,
+                           dx_row_stride, gain, gain_offset, eps, dgain, workspace,
+                           workspace_bytes, stream) -> None:
+    _call("muse_rms_norm_backward", x, dy, dx, dtype, rows, hidden, x_row_stride, dy_row_stride,
+          dx_row_stride, gain, gain_offset, eps, dgain, workspace, workspace_bytes, stream)
+
+
+def muse_input_scale_norm_backward(x, dy, dx, dtype, rows, hidden, x_row_stride, dy_row_stride,
+                                   dx_row_stride, gain, gain_offset, eps, dgain, workspace,
+                                   workspace_bytes, stream) -> None:
+    _call("muse_input_scale_norm_backward", x, dy, dx, dtype, rows, hidden, x_row_stride,
+          dy_row_stride, dx_row_stride, gain, gain_offset, eps, dgain, workspace, workspace_bytes,
+          stream)
+
+
+def muse_norm_residual_backward(stream_in, branch, dstream_out, dstream_in, dbranch, branch_dtype,
+                                rows, hidden, gain, gain_offset, theta, input_scale, norm_eps,
+                                dgain, dtheta, workspace, workspace_bytes, stream) -> None:
+    _call("muse_norm_residual_backward", stream_in, branch, dstream_out, dstream_in, dbranch,
+          branch_dtype, rows, hidden, gain, gain_offset, theta, int(input_scale), norm_eps, dgain,
+          dtheta, workspace, workspace_bytes, stream)

@@ -195,3 +195,77 @@ def stream_copy(src: torch.Tensor, dst: torch.Tensor, stream=None) -> torch.Tens
         raise ValueError("src and dst must be contiguous and of equal byte size")
     _lib.muse_stream_copy(src.data_ptr(), dst.data_ptr(), nbytes, _stream(stream))
     return dst
+
+
+# ------------------------------------------------------------------ backward
+
+
+def _workspace(rows: int, hidden: int, device, workspace):
+    need = _lib.muse_norm_backward_workspace_bytes(rows, hidden)
+    if workspace is None:
+        return torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+    if workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace needs {need} bytes")
+    return workspace
+
+
+def _row_bwd(fn, x, dy, gain, gain_offset, eps, dx, want_dgain, workspace, stream):
+    _cuda(x, dy, gain, dx)
+    if dy.shape != x.shape or dy.dtype != x.dtype:
+        raise ValueError("dy must match x")
+    dx = _out_like(x, dx)
+    rows, hidden, xs = _rows(x)
+    _, _, dys = _rows(dy)
+    _, _, dxs = _rows(dx)
+    g = _gain(gain)
+    dgain = None
+    ws = None
+    if want_dgain and g is not None:
+        dgain = torch.empty(hidden, dtype=torch.float32, device=x.device)
+        ws = _workspace(rows, hidden, x.device, workspace)
+    fn(x.data_ptr(), dy.data_ptr(), dx.data_ptr(), _dtype(x), rows, hidden, xs, dys, dxs, _ptr(g),
+       gain_offset, eps, _ptr(dgain), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream))
+    return dx, dgain
+
+
+def rms_norm_backward(x, dy, gain=None, gain_offset: float = 0.0, eps: float = 1e-6, dx=None,
+                      want_dgain: bool = True, workspace=None, stream=None):
+    """Backward of core 1: returns (dx, dgain); dgain is None without a gain."""
+    return _row_bwd(_lib.muse_rms_norm_backward, x, dy, gain, gain_offset, eps, dx, want_dgain,
+                    workspace, stream)
+
+
+def input_scale_norm_backward(x, dy, gain=None, gain_offset: float = 0.0, eps: float = 1e-6,
+                              dx=None, want_dgain: bool = True, workspace=None, stream=None):
+    """Backward of core 2: returns (dx, dgain); dgain is None without a gain."""
+    return _row_bwd(_lib.muse_input_scale_norm_backward, x, dy, gain, gain_offset, eps, dx,
+                    want_dgain, workspace, stream)
+
+
+def norm_residual_backward(stream_in, branch, dstream_out, theta, gain=None,
+                           gain_offset: float = 0.0, input_scale: bool = False,
+                           norm_eps: float = 1e-6, want_params: bool = True, workspace=None,
+                           stream=None):
+    """Backward of core 5: returns (dstream_in, dbranch, dgain, dtheta)."""
+    _cuda(stream_in, branch, dstream_out, theta, gain)
+    if stream_in.dtype != torch.float32 or dstream_out.dtype != torch.float32:
+        raise TypeError("stream tensors must be float32")
+    if not (stream_in.is_contiguous() and branch.is_contiguous() and dstream_out.is_contiguous()):
+        raise ValueError("stream, branch and dstream_out must be contiguous")
+    hidden = stream_in.shape[-1]
+    rows = stream_in.numel() // hidden
+    dsi = torch.empty_like(stream_in)
+    db = torch.empty_like(branch)
+    g = _gain(gain)
+    dgain = dtheta = ws = None
+    if want_params:
+        dtheta = torch.empty(hidden, dtype=torch.float32, device=stream_in.device)
+        if g is not None:
+            dgain = torch.empty(hidden, dtype=torch.float32, device=stream_in.device)
+        ws = _workspace(rows, hidden, stream_in.device, workspace)
+    _lib.muse_norm_residual_backward(
+        stream_in.data_ptr(), branch.data_ptr(), dstream_out.data_ptr(), dsi.data_ptr(),
+        db.data_ptr(), _dtype(branch), rows, hidden, _ptr(g), gain_offset,
+        theta.contiguous().data_ptr(), input_scale, norm_eps, _ptr(dgain), _ptr(dtheta), _ptr(ws),
+        0 if ws is None else ws.numel(), _stream(stream))
+    return dsi, db, dgain, dtheta

@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <map>
 #include <mutex>
+#include <initializer_list>
 #include <tuple>
 
 #include "kernels.h"
@@ -115,6 +116,77 @@ muse_status row_entry(muse::RowOp op, const void* x, void* y, muse_dtype dtype, 
     a.gain_offset = gain_offset;
     a.eps = eps;
     return from_cuda(muse::launch_row(dtype, op, a, stream), name);
+}
+
+// Shared checks of the row backward entry points: the workspace and the
+// parameter-gradient outputs must not overlap each other or any tensor.
+muse_status bwd_workspace_check(const char* name, int64_t rows, int64_t hidden, void* ws,
+                                size_t ws_bytes, bool needed) {
+    if (!needed) return MUSE_OK;
+    const size_t need = muse::row_bwd_workspace_bytes(rows, (int32_t)hidden);
+    if (!ws || ws_bytes < need)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: workspace of %zu bytes needed, %zu given", name, need,
+                    ws ? ws_bytes : (size_t)0);
+    if (!aligned(ws, 16)) return fail(MUSE_ERR_UNSUPPORTED, "%s: workspace not 16-byte aligned", name);
+    return MUSE_OK;
+}
+
+bool any_overlap(const Span& a, std::initializer_list<Span> others) {
+    for (const Span& o : others)
+        if (overlap(a, o)) return true;
+    return false;
+}
+
+muse_status row_bwd_entry(bool input_scale, const void* x, const void* dy, void* dx,
+                          muse_dtype dtype, int64_t rows, int64_t hidden, int64_t xs,
+                          int64_t dys, int64_t dxs, const float* gain, float gain_offset,
+                          float eps, float* dgain, void* ws, size_t ws_bytes, cudaStream_t stream,
+                          const char* name) {
+    if (!valid_dtype(dtype)) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, (int)dtype);
+    if (rows < 0 || hidden <= 0)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: rows=%lld hidden=%lld", name, (long long)rows, (long long)hidden);
+    if (!finite(eps) || eps < 0.0f || !finite(gain_offset))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: eps must be finite and >= 0, gain_offset finite", name);
+    if (xs < hidden || dys < hidden || dxs < hidden)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: row strides must be >= hidden", name);
+    if (dgain && !gain) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: dgain requested without a gain", name);
+    if (rows == 0) {
+        if (dgain) return from_cuda(cudaMemsetAsync(dgain, 0, sizeof(float) * (size_t)hidden, stream), name);
+        return MUSE_OK;
+    }
+    if (!x || !dy || !dx) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null x, dy or dx", name);
+    const int64_t es = elem_size(dtype);
+    if (!aligned(x, 16) || !aligned(dy, 16) || !aligned(dx, 16) || (hidden * es) % 16 || (xs * es) % 16 ||
+        (dys * es) % 16 || (dxs * es) % 16)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: pointers, row widths and strides must be 16-byte multiples", name);
+    if ((gain && !aligned(gain, 16)) || (dgain && !aligned(dgain, 16)))
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: gain / dgain not 16-byte aligned", name);
+    if (hidden / vec_elems(dtype) > muse::kBwdMaxVectors)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: rows of more than %d 16-byte vectors", name, muse::kBwdMaxVectors);
+    muse_status st = bwd_workspace_check(name, rows, hidden, ws, ws_bytes, dgain != nullptr);
+    if (st != MUSE_OK) return st;
+    const Span sx = span(x, rows, hidden, xs, es), sdy = span(dy, rows, hidden, dys, es);
+    const Span sdx = span(dx, rows, hidden, dxs, es);
+    const Span sg = span(gain, gain ? 1 : 0, hidden, hidden, 4), sdg = span(dgain, dgain ? 1 : 0, hidden, hidden, 4);
+    const Span sws = span(ws, dgain ? 1 : 0, (int64_t)ws_bytes, (int64_t)ws_bytes, 1);
+    if (bad_alias(sdx, sx, true) || bad_alias(sdx, sdy, true) || any_overlap(sdx, {sg, sdg, sws}) ||
+        any_overlap(sdg, {sx, sdy, sg, sws}) || any_overlap(sws, {sx, sdy, sg}))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: an output or the workspace overlaps another tensor", name);
+    muse::RowBwdArgs a{};
+    a.x = x;
+    a.dy = dy;
+    a.dx = dx;
+    a.gain = gain;
+    a.part_gain = static_cast<float*>(ws);
+    a.rows = rows;
+    a.x_stride = xs;
+    a.dy_stride = dys;
+    a.dx_stride = dxs;
+    a.width = (int32_t)hidden;
+    a.gain_offset = gain_offset;
+    a.eps = eps;
+    const muse::BwdOp op = input_scale ? muse::BwdOp::kInputScale : muse::BwdOp::kRms;
+    return from_cuda(muse::launch_row_bwd(dtype, op, a, dgain, nullptr, stream), name);
 }
 
 }  // namespace
@@ -362,13 +434,107 @@ muse_status muse_norm_residual(const float* stream_in, const void* branch, float
     return from_cuda(muse::launch_row(branch_dtype, op, a, stream), name);
 }
 
+size_t muse_norm_backward_workspace_bytes(int64_t rows, int64_t hidden) {
+    if (rows <= 0 || hidden <= 0 || hidden > (int64_t)1 << 30) return 0;
+    return muse::row_bwd_workspace_bytes(rows, (int32_t)hidden);
+}
+
+muse_status muse_rms_norm_backward(const void* x, const void* dy, void* dx, muse_dtype dtype,
+                                   int64_t rows, int64_t hidden, int64_t x_row_stride,
+                                   int64_t dy_row_stride, int64_t dx_row_stride,
+                                   const float* gain, float gain_offset, float eps, float* dgain,
+                                   void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    return row_bwd_entry(false, x, dy, dx, dtype, rows, hidden, x_row_stride, dy_row_stride,
+                         dx_row_stride, gain, gain_offset, eps, dgain, workspace, workspace_bytes,
+                         stream, "muse_rms_norm_backward");
+}
+
+muse_status muse_input_scale_norm_backward(const void* x, const void* dy, void* dx,
+                                           muse_dtype dtype, int64_t rows, int64_t hidden,
+                                           int64_t x_row_stride, int64_t dy_row_stride,
+                                           int64_t dx_row_stride, const float* gain,
+                                           float gain_offset, float eps, float* dgain,
+                                           void* workspace, size_t workspace_bytes,
+                                           cudaStream_t stream) {
+    return row_bwd_entry(true, x, dy, dx, dtype, rows, hidden, x_row_stride, dy_row_stride,
+                         dx_row_stride, gain, gain_offset, eps, dgain, workspace, workspace_bytes,
+                         stream, "muse_input_scale_norm_backward");
+}
+
+muse_status muse_norm_residual_backward(const float* stream_in, const void* branch,
+                                        const float* dstream_out, float* dstream_in,
+                                        void* dbranch, muse_dtype branch_dtype, int64_t rows,
+                                        int64_t hidden, const float* gain, float gain_offset,
+                                        const float* theta, int input_scale, float norm_eps,
+                                        float* dgain, float* dtheta, void* workspace,
+                                        size_t workspace_bytes, cudaStream_t stream) {
+    const char* name = "muse_norm_residual_backward";
+    if (!valid_dtype(branch_dtype)) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, (int)branch_dtype);
+    if (rows < 0 || hidden <= 0)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: rows=%lld hidden=%lld", name, (long long)rows, (long long)hidden);
+    if (!finite(norm_eps) || norm_eps < 0.0f || !finite(gain_offset))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: norm_eps must be finite and >= 0, gain_offset finite", name);
+    if (dgain && !gain) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: dgain requested without a gain", name);
+    if (rows == 0) {
+        cudaError_t e = cudaSuccess;
+        if (dgain) e = cudaMemsetAsync(dgain, 0, sizeof(float) * (size_t)hidden, stream);
+        if (e == cudaSuccess && dtheta) e = cudaMemsetAsync(dtheta, 0, sizeof(float) * (size_t)hidden, stream);
+        return from_cuda(e, name);
+    }
+    if (!stream_in || !branch || !dstream_out || !dstream_in || !dbranch || !theta)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null tensor", name);
+    const int64_t es = elem_size(branch_dtype);
+    if (!aligned(stream_in, 16) || !aligned(branch, 16) || !aligned(dstream_out, 16) || !aligned(dstream_in, 16) ||
+        !aligned(dbranch, 16) || (hidden * es) % 16)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: pointers and row widths must be 16-byte multiples", name);
+    if (!aligned(theta, 16) || (gain && !aligned(gain, 16)) || (dgain && !aligned(dgain, 16)) ||
+        (dtheta && !aligned(dtheta, 16)))
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: theta / gain / dgain / dtheta not 16-byte aligned", name);
+    if (hidden / vec_elems(branch_dtype) > muse::kBwdMaxVectors)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: rows of more than %d 16-byte vectors", name, muse::kBwdMaxVectors);
+    muse_status st = bwd_workspace_check(name, rows, hidden, workspace, workspace_bytes, dgain || dtheta);
+    if (st != MUSE_OK) return st;
+    const Span sh = span(stream_in, rows, hidden, hidden, 4), sdo = span(dstream_out, rows, hidden, hidden, 4);
+    const Span sb = span(branch, rows, hidden, hidden, es), sdb = span(dbranch, rows, hidden, hidden, es);
+    const Span sdi = span(dstream_in, rows, hidden, hidden, 4), sth = span(theta, 1, hidden, hidden, 4);
+    const Span sg = span(gain, gain ? 1 : 0, hidden, hidden, 4), sdg = span(dgain, dgain ? 1 : 0, hidden, hidden, 4);
+    const Span sdt = span(dtheta, dtheta ? 1 : 0, hidden, hidden, 4);
+    const Span sws = span(workspace, (dgain || dtheta) ? 1 : 0, (int64_t)workspace_bytes, (int64_t)workspace_bytes, 1);
+    bool bad = bad_alias(sdi, sdo, true) || any_overlap(sdi, {sh, sb, sdb, sth, sg, sdg, sdt, sws});
+    bad = bad || bad_alias(sdb, sb, true) || any_overlap(sdb, {sh, sdo, sth, sg, sdg, sdt, sws});
+    bad = bad || any_overlap(sdg, {sh, sdo, sb, sth, sg, sdt, sws}) || any_overlap(sdt, {sh, sdo, sb, sth, sg, sws});
+    bad = bad || any_overlap(sws, {sh, sdo, sb, sth, sg});
+    if (bad) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: an output or the workspace overlaps another tensor", name);
+    muse::RowBwdArgs a{};
+    a.x = branch;
+    a.dy = dstream_out;
+    a.stream_in = stream_in;
+    a.dx = dbranch;
+    a.dstream_in = dstream_in;
+    a.gain = gain;
+    a.theta = theta;
+    a.rows = rows;
+    a.x_stride = a.dy_stride = a.dx_stride = hidden;
+    a.width = (int32_t)hidden;
+    a.gain_offset = gain_offset;
+    a.eps = norm_eps;
+    if (dgain || dtheta) {
+        const int64_t cap = (int64_t)(muse::row_bwd_workspace_bytes(rows, (int32_t)hidden) / 2 / sizeof(float));
+        a.part_gain = static_cast<float*>(workspace);
+        a.part_theta = static_cast<float*>(workspace) + cap;
+    }
+    const muse::BwdOp op = input_scale ? muse::BwdOp::kResidualIS : muse::BwdOp::kResidual;
+    return from_cuda(muse::launch_row_bwd(branch_dtype, op, a, dgain, dtheta, stream), name);
+}
+
 muse_status muse_device_error(unsigned int* flags, int clear) {
     if (!flags) return fail(MUSE_ERR_INVALID_ARGUMENT, "muse_device_error: null flags");
-    // bit 0: the row pipeline's word, bit 1: the Q/K ring's word
-    unsigned int row = 0, qk = 0;
+    // bit 0: the row pipeline's word, bit 1: the Q/K ring's, bit 2: the row backward's
+    unsigned int row = 0, qk = 0, bwd = 0;
     cudaError_t e = muse::read_device_error(&row, clear != 0);
     if (e == cudaSuccess) e = muse::read_qk_device_error(&qk, clear != 0);
-    *flags = (row ? 1u : 0u) | (qk ? 2u : 0u);
+    if (e == cudaSuccess) e = muse::read_bwd_device_error(&bwd, clear != 0);
+    *flags = (row ? 1u : 0u) | (qk ? 2u : 0u) | (bwd ? 4u : 0u);
     return from_cuda(e, "muse_device_error");
 }
 

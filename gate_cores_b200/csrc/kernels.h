@@ -43,6 +43,36 @@ struct HeadGateArgs {
     float eps;
 };
 
+// Backward of the row-wide cores (cores 1, 2, 5): one row per token.
+enum class BwdOp : int {
+    kRms = 0,          // core 1
+    kInputScale = 1,   // core 2
+    kResidual = 2,     // core 5, gain after the norm
+    kResidualIS = 3,   // core 5, gain before the norm
+};
+
+struct RowBwdArgs {
+    const void* x;          // x (cores 1, 2) or the branch (core 5)
+    const void* dy;         // dL/dy (cores 1, 2; x's dtype) or dL/dstream_out (core 5; FP32)
+    const float* stream_in; // core 5: the forward's stream h
+    void* dx;               // dL/dx (cores 1, 2) or dL/dbranch (core 5), x's dtype
+    float* dstream_in;      // core 5: dL/dh
+    const float* gain;      // may be null (no gain gradient then)
+    const float* theta;     // core 5
+    float* part_gain;       // [grid][width] per-CTA partial gain gradients, or null
+    float* part_theta;      // core 5: [grid][width] per-CTA partial theta gradients
+    int64_t rows;
+    int64_t x_stride, dy_stride, dx_stride;  // elements; core 5 rows are contiguous
+    int32_t width;
+    float gain_offset;
+    float eps;
+};
+
+// Largest row (in 16-byte vectors) the row backward handles, and the
+// workspace it needs for `rows` rows of `width` elements.
+constexpr int kBwdMaxVectors = 1024;
+size_t row_bwd_workspace_bytes(int64_t rows, int32_t width);
+
 constexpr int kMaxHalfDim = 128;  // head_dim <= 256
 
 struct QkArgs {
@@ -74,9 +104,15 @@ cudaError_t launch_row_regs(int dtype, RowOp op, const RowArgs& a, cudaStream_t 
 // timed out.
 cudaError_t read_device_error(unsigned int* out, bool clear);
 cudaError_t read_qk_device_error(unsigned int* out, bool clear);
+cudaError_t read_bwd_device_error(unsigned int* out, bool clear);
 cudaError_t launch_head_gate(int dtype, const HeadGateArgs& a, cudaStream_t s);
 cudaError_t launch_qk(int dtype, int use_rope, int upcast_rope, const QkArgs& a, cudaStream_t s);
 cudaError_t launch_copy(const void* src, void* dst, int64_t bytes, cudaStream_t s);
+// Row backward: per-CTA partials into a.part_gain / a.part_theta (the caller's
+// workspace), then a deterministic reduction into dgain / dtheta (either may
+// be null).
+cudaError_t launch_row_bwd(int dtype, BwdOp op, RowBwdArgs a, float* dgain, float* dtheta,
+                           cudaStream_t s);
 
 // Device facts for grid sizing (cached per device).
 int sm_count();

@@ -1,0 +1,433 @@
+// Backward of the row-wide cores: core 1 (_rms_norm_core), core 2
+// (_input_scale_norm_core) and core 5 (_norm_residual_core with the
+// per-channel cos/sin blend).  The cores run under autograd, so the backward
+// is the derivative of each forward map, evaluated from the saved forward
+// inputs with r recomputed; every dtype boundary the forward materialises
+// passes the gradient back rounded to that tensor's dtype.
+//
+//   core 1:  g = dy w;  dx = r g - r^3 x (sum_j g_j x_j) / H;
+//            dgain += dy x r
+//   core 2:  z = x w;  dz = r dy - r^3 z (sum_j dy_j z_j) / H;
+//            dx = dz w;  dgain += dz x
+//   core 5:  dh = cos(theta) dh';  dnb = cast_branch(sin(theta) dh');
+//            dbranch = the core 1 (or core 2) form applied to dnb;
+//            dtheta += dh' (-sin(theta) h + cos(theta) nb), nb the forward's
+//            cast branch
+//
+// Same pipeline as the forward row kernels (row_tma.cu): a producer warp
+// streams each row's inputs (x and dy; core 5: branch, dh' and h) into a ring
+// of shared-memory stages with cp.async.bulk; the consumer warps reduce the
+// row's two sums (sum of squares and the gradient dot product) with one
+// named barrier and write the input gradients.  The rows are dealt
+// round-robin to a persistent grid; each consumer thread owns the same
+// columns in every row, so it accumulates its columns' gain / theta
+// gradients in registers and writes one partial row per CTA into the
+// caller's workspace, which a second kernel sums in a fixed order.
+#include <type_traits>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace muse {
+namespace {
+__device__ unsigned int g_device_error;  // nonzero: an mbarrier wait of the row backward timed out
+}  // namespace
+}  // namespace muse
+
+#include "tma_pipe.cuh"
+
+namespace muse {
+namespace {
+
+using namespace pipe;
+
+__host__ __device__ constexpr bool b_is_res(BwdOp op) { return op == BwdOp::kResidual || op == BwdOp::kResidualIS; }
+__host__ __device__ constexpr bool b_gain_first(BwdOp op) { return op == BwdOp::kInputScale || op == BwdOp::kResidualIS; }
+
+// At most this many resident CTAs per SM (bounds the workspace).
+constexpr int kBwdMaxCtasPerSm = 4;
+
+__host__ __device__ inline uint32_t al128(uint32_t v) { return (v + 127u) & ~127u; }
+
+struct BwdLayout {
+    uint32_t x_bytes, dy_bytes, h_bytes, dy_off, h_off, stage_bytes;
+};
+
+template <typename T, BwdOp OP>
+__host__ __device__ inline BwdLayout bwd_layout(int width) {
+    BwdLayout L;
+    L.x_bytes = (uint32_t)width * sizeof(T);
+    L.dy_bytes = (uint32_t)width * (b_is_res(OP) ? 4u : (uint32_t)sizeof(T));
+    L.h_bytes = b_is_res(OP) ? (uint32_t)width * 4u : 0u;
+    L.dy_off = al128(L.x_bytes);
+    L.h_off = L.dy_off + al128(L.dy_bytes);
+    L.stage_bytes = L.h_off + al128(L.h_bytes);
+    return L;
+}
+
+// Sums of two values over the consumer threads; two banks, one barrier.
+__device__ __forceinline__ float2 consumer_sum2(float a, float b, float (*red)[2][32], int& bank, int ncons) {
+    a = group_sum<32>(a);
+    b = group_sum<32>(b);
+    const int nw = ncons >> 5;
+    if (nw == 1) return make_float2(a, b);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        red[bank][0][warp] = a;
+        red[bank][1][warp] = b;
+    }
+    consumer_sync(ncons);
+    const float ta = lane < nw ? red[bank][0][lane] : 0.0f;
+    const float tb = lane < nw ? red[bank][1][lane] : 0.0f;
+    bank ^= 1;
+    return make_float2(group_sum<32>(ta), group_sum<32>(tb));
+}
+
+// 16-byte vector of T at byte offset `off` of a shared stage -> V floats.
+template <typename T>
+__device__ __forceinline__ void ld_stage(const unsigned char* p, float* f) {
+    unpack<T>(*reinterpret_cast<const uint4*>(p), f);
+}
+// V floats of an FP32 row at element offset e0 of a shared stage.
+template <int V>
+__device__ __forceinline__ void ld_stage_f32(const unsigned char* p, float* f) {
+#pragma unroll
+    for (int q = 0; q < V / 4; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(p + 16 * q);
+        f[4 * q] = v.x; f[4 * q + 1] = v.y; f[4 * q + 2] = v.z; f[4 * q + 3] = v.w;
+    }
+}
+template <int V>
+__device__ __forceinline__ void st_f32(float* p, const float* f) {
+#pragma unroll
+    for (int q = 0; q < V / 4; ++q)
+        *reinterpret_cast<float4*>(p + 4 * q) = make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
+}
+
+template <typename T, BwdOp OP, int VPT, bool G, int S>
+__device__ __forceinline__ void row_bwd_body(const RowBwdArgs& a) {
+    constexpr int V = Vec<T>::N;
+    constexpr bool RES = b_is_res(OP);
+    constexpr bool FIRST = b_gain_first(OP);
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ float red[2][2][32];
+    __shared__ __align__(8) uint64_t full_bar[S];
+    __shared__ __align__(8) uint64_t empty_bar[S];
+
+    const int ncons = blockDim.x - 32;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int nvec = a.width / V;
+    const BwdLayout L = bwd_layout<T, OP>(a.width);
+    const int64_t step = gridDim.x;
+    const int64_t r0 = blockIdx.x;
+    const int n = (int)max((int64_t)0, (a.rows - r0 + step - 1) / step);
+    const uint32_t dy_es = RES ? 4u : (uint32_t)sizeof(T);
+
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], (uint32_t)(ncons >> 5));
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (warp == (ncons >> 5)) {
+        // ---------------- producer warp: lane 0 issues whole-row bulk copies
+        if (lane == 0) {
+            const uint32_t bytes = L.x_bytes + L.dy_bytes + L.h_bytes;
+            int issued = 0;
+            for (int k = 0; k < n; ++k) {
+                const int s = k % S;
+                if (k >= S && !mbar_wait(&empty_bar[s], (uint32_t)((k / S - 1) & 1))) break;
+                unsigned char* st = smem + (size_t)s * L.stage_bytes;
+                const int64_t row = r0 + k * step;
+                mbar_arrive_expect_tx(&full_bar[s], bytes);
+                bulk_g2s(st, static_cast<const char*>(a.x) + row * a.x_stride * (int64_t)sizeof(T), L.x_bytes, &full_bar[s]);
+                bulk_g2s(st + L.dy_off, static_cast<const char*>(a.dy) + row * a.dy_stride * (int64_t)dy_es,
+                         L.dy_bytes, &full_bar[s]);
+                if constexpr (RES)
+                    bulk_g2s(st + L.h_off, a.stream_in + row * (int64_t)a.width, L.h_bytes, &full_bar[s]);
+                ++issued;
+            }
+            for (int k = max(0, issued - S); k < issued; ++k)
+                if (!mbar_wait(&full_bar[k % S], (uint32_t)((k / S) & 1))) break;
+        }
+        return;
+    }
+
+    // ---------------- consumer warps: slot i covers vector tid + i * ncons
+    bool valid[VPT];
+    int col[VPT];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        valid[i] = tid + i * ncons < nvec;
+        col[i] = valid[i] ? (tid + i * ncons) * V : 0;
+    }
+    float w[VPT][V], cth[RES ? VPT : 1][V], sth[RES ? VPT : 1][V];
+    float acc_g[G ? VPT : 1][V], acc_t[RES ? VPT : 1][V];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+            w[i][e] = G ? __ldg(a.gain + col[i] + e) + a.gain_offset : 1.0f;  // FP32 sum
+            if constexpr (G) acc_g[i][e] = 0.0f;
+            if constexpr (RES) {
+                float sv, cv;
+                sincosf(__ldg(a.theta + col[i] + e), &sv, &cv);
+                cth[i][e] = cv;
+                sth[i][e] = sv;
+                acc_t[i][e] = 0.0f;
+            }
+        }
+    }
+    const float inv_width = 1.0f / (float)a.width;
+    char* dx_row = static_cast<char*>(a.dx) + r0 * a.dx_stride * (int64_t)sizeof(T);
+    const int64_t dx_step = step * a.dx_stride * (int64_t)sizeof(T);
+    float* dh_row = RES ? a.dstream_in + r0 * (int64_t)a.width : nullptr;
+    const int64_t dh_step = step * (int64_t)a.width;
+
+    bool alive = true;
+    int bank = 0;
+    int s = 0;
+    uint32_t phase = 0;
+    for (int k = 0; k < n; ++k) {
+        if (alive) alive = mbar_wait(&full_bar[s], phase);
+        alive = __all_sync(0xffffffffu, alive);
+        const unsigned char* st = smem + s * L.stage_bytes;
+        float x[VPT][V], g[VPT][V], h[RES ? VPT : 1][V];
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            if (alive && valid[i]) {
+                ld_stage<T>(st + (uint32_t)col[i] * sizeof(T), x[i]);
+                if constexpr (RES) {
+                    ld_stage_f32<V>(st + L.dy_off + (uint32_t)col[i] * 4u, g[i]);
+                    ld_stage_f32<V>(st + L.h_off + (uint32_t)col[i] * 4u, h[i]);
+                } else {
+                    ld_stage<T>(st + L.dy_off + (uint32_t)col[i] * sizeof(T), g[i]);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < V; ++e) {
+                    x[i][e] = 0.0f;
+                    g[i][e] = 0.0f;
+                    if constexpr (RES) h[i][e] = 0.0f;
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0 && alive) mbar_arrive(&empty_bar[s]);
+        if (++s == S) {
+            s = 0;
+            phase ^= 1u;
+        }
+
+        // core 5: the blend's gradient reaching the cast branch, rounded to it
+        float dh[RES ? VPT : 1][V];
+        if constexpr (RES) {
+#pragma unroll
+            for (int i = 0; i < VPT; ++i)
+#pragma unroll
+                for (int e = 0; e < V; ++e) {
+                    dh[i][e] = g[i][e];
+                    g[i][e] = round_to<T>(sth[i][e] * dh[i][e]);
+                }
+        }
+        // row sums: mean square of the normalised input, gradient dot product
+        float ss = 0.0f, cd = 0.0f;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i)
+#pragma unroll
+            for (int e = 0; e < V; ++e) {
+                const float u = FIRST ? x[i][e] * w[i][e] : x[i][e];
+                ss = fmaf(u, u, ss);
+                cd = fmaf(FIRST ? g[i][e] : g[i][e] * w[i][e], u, cd);
+            }
+        const float2 tot = consumer_sum2(ss, cd, red, bank, ncons);
+        const float r = inv_rms_fast(tot.x, inv_width, a.eps);
+        const float cr = r * r * r * tot.y * inv_width;
+
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            float dx[V];
+#pragma unroll
+            for (int e = 0; e < V; ++e) {
+                if constexpr (FIRST) {
+                    const float u = x[i][e] * w[i][e];
+                    const float dz = r * g[i][e] - cr * u;
+                    dx[e] = dz * w[i][e];
+                    if constexpr (G) acc_g[i][e] = fmaf(dz, x[i][e], acc_g[i][e]);
+                } else {
+                    dx[e] = (r * w[i][e]) * g[i][e] - cr * x[i][e];
+                    if constexpr (G) acc_g[i][e] = fmaf(g[i][e], x[i][e] * r, acc_g[i][e]);
+                }
+            }
+            if (alive && valid[i]) st_vec(dx_row + (uint32_t)col[i] * sizeof(T), pack<T>(dx));
+            if constexpr (RES) {
+                float dhs[V];
+#pragma unroll
+                for (int e = 0; e < V; ++e) {
+                    dhs[e] = cth[i][e] * dh[i][e];
+                    const float v = FIRST ? (x[i][e] * w[i][e]) * r : (x[i][e] * r) * w[i][e];
+                    const float nb = round_to<T>(v);  // the forward's cast branch
+                    acc_t[i][e] = fmaf(dh[i][e], fmaf(-sth[i][e], h[i][e], cth[i][e] * nb), acc_t[i][e]);
+                }
+                if (alive && valid[i]) st_f32<V>(dh_row + col[i], dhs);
+            }
+        }
+        dx_row += dx_step;
+        if constexpr (RES) dh_row += dh_step;
+    }
+
+    // one partial row of the parameter gradients per CTA
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        if (!valid[i]) continue;
+        if constexpr (G)
+            if (a.part_gain) st_f32<V>(a.part_gain + (int64_t)blockIdx.x * a.width + col[i], acc_g[i]);
+        if constexpr (RES)
+            if (a.part_theta) st_f32<V>(a.part_theta + (int64_t)blockIdx.x * a.width + col[i], acc_t[i]);
+    }
+}
+
+// One entry symbol per core.
+template <typename T, int VPT, bool G, int S>
+__global__ void __launch_bounds__(512 + 32) rms_norm_bwd_kernel(const __grid_constant__ RowBwdArgs a) {
+    pdl_begin();
+    row_bwd_body<T, BwdOp::kRms, VPT, G, S>(a);
+}
+template <typename T, int VPT, bool G, int S>
+__global__ void __launch_bounds__(512 + 32) input_scale_norm_bwd_kernel(const __grid_constant__ RowBwdArgs a) {
+    pdl_begin();
+    row_bwd_body<T, BwdOp::kInputScale, VPT, G, S>(a);
+}
+template <typename T, int VPT, bool G, int S>
+__global__ void __launch_bounds__(512 + 32) norm_residual_bwd_kernel(const __grid_constant__ RowBwdArgs a) {
+    pdl_begin();
+    row_bwd_body<T, BwdOp::kResidual, VPT, G, S>(a);
+}
+template <typename T, int VPT, bool G, int S>
+__global__ void __launch_bounds__(512 + 32) norm_residual_input_scale_bwd_kernel(const __grid_constant__ RowBwdArgs a) {
+    pdl_begin();
+    row_bwd_body<T, BwdOp::kResidualIS, VPT, G, S>(a);
+}
+
+template <typename T, BwdOp OP, int VPT, bool G, int S>
+constexpr auto row_bwd_kernel() {
+    if constexpr (OP == BwdOp::kRms) return rms_norm_bwd_kernel<T, VPT, G, S>;
+    else if constexpr (OP == BwdOp::kInputScale) return input_scale_norm_bwd_kernel<T, VPT, G, S>;
+    else if constexpr (OP == BwdOp::kResidual) return norm_residual_bwd_kernel<T, VPT, G, S>;
+    else return norm_residual_input_scale_bwd_kernel<T, VPT, G, S>;
+}
+
+// out[c] = sum over parts of part[p][c], in a fixed order: 8 interleaved
+// partial sums per column, combined in order.
+__global__ void __launch_bounds__(256) param_grad_reduce_kernel(const float* __restrict__ part, int nparts,
+                                                                int width, float* __restrict__ out) {
+    pdl_begin();
+    __shared__ float sm[8][33];
+    const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
+    const int c = blockIdx.x * 32 + lane;
+    float acc = 0.0f;
+    if (c < width)
+        for (int p = grp; p < nparts; p += 8) acc += part[(int64_t)p * width + c];
+    sm[grp][lane] = acc;
+    __syncthreads();
+    if (grp == 0 && c < width) {
+        float t = sm[0][lane];
+#pragma unroll
+        for (int q = 1; q < 8; ++q) t += sm[q][lane];
+        out[c] = t;
+    }
+}
+
+int bwd_grid_cap() { return kBwdMaxCtasPerSm * sm_count(); }
+
+template <typename T, BwdOp OP, int VPT, bool G, int S>
+cudaError_t launch_bwd_s(RowBwdArgs a, int nvec, float* dgain, float* dtheta, cudaStream_t s) {
+    const int ncons = ((nvec + VPT - 1) / VPT + 31) / 32 * 32;
+    const int threads = ncons + 32;
+    const BwdLayout L = bwd_layout<T, OP>(a.width);
+    const size_t smem = (size_t)S * L.stage_bytes;
+    auto kern = row_bwd_kernel<T, OP, VPT, G, S>();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int per_sm = min(blocks_per_sm((const void*)kern, threads, smem), kBwdMaxCtasPerSm);
+    int64_t grid = (int64_t)per_sm * sm_count();
+    if (grid > a.rows) grid = a.rows;
+    if (grid < 1) grid = 1;
+    if (!(G && dgain)) a.part_gain = nullptr;
+    if (!dtheta) a.part_theta = nullptr;
+    e = launch_pdl(kern, (unsigned)grid, (unsigned)threads, smem, s, a);
+    if (e != cudaSuccess) return e;
+    const unsigned rgrid = (unsigned)((a.width + 31) / 32);
+    if (a.part_gain) {
+        e = launch_pdl(param_grad_reduce_kernel, rgrid, 256u, 0, s, (const float*)a.part_gain, (int)grid, (int)a.width, dgain);
+        if (e != cudaSuccess) return e;
+    }
+    if constexpr (b_is_res(OP)) {
+        if (a.part_theta)
+            e = launch_pdl(param_grad_reduce_kernel, rgrid, 256u, 0, s, (const float*)a.part_theta, (int)grid, (int)a.width, dtheta);
+    }
+    return e;
+}
+
+template <typename T, BwdOp OP, int VPT>
+cudaError_t launch_bwd_v(const RowBwdArgs& a, int nvec, float* dgain, float* dtheta, cudaStream_t s) {
+    const BwdLayout L = bwd_layout<T, OP>(a.width);
+    const bool g = a.gain != nullptr;
+    if (L.stage_bytes < 16 * 1024)
+        return g ? launch_bwd_s<T, OP, VPT, true, 3>(a, nvec, dgain, dtheta, s)
+                 : launch_bwd_s<T, OP, VPT, false, 3>(a, nvec, dgain, dtheta, s);
+    return g ? launch_bwd_s<T, OP, VPT, true, 2>(a, nvec, dgain, dtheta, s)
+             : launch_bwd_s<T, OP, VPT, false, 2>(a, nvec, dgain, dtheta, s);
+}
+
+// Slots per consumer thread: one up to 256 vectors (core 5: 512), then two,
+// then four (cores 1, 2).
+template <typename T, BwdOp OP>
+cudaError_t launch_bwd_op(const RowBwdArgs& a, float* dgain, float* dtheta, cudaStream_t s) {
+    const int nvec = a.width / Vec<T>::N;
+    if (nvec <= 256 || (b_is_res(OP) && nvec <= 512)) return launch_bwd_v<T, OP, 1>(a, nvec, dgain, dtheta, s);
+    if constexpr (b_is_res(OP)) {
+        return launch_bwd_v<T, OP, 2>(a, nvec, dgain, dtheta, s);
+    } else {
+        if (nvec <= 512) return launch_bwd_v<T, OP, 2>(a, nvec, dgain, dtheta, s);
+        return launch_bwd_v<T, OP, 4>(a, nvec, dgain, dtheta, s);
+    }
+}
+
+template <typename T>
+cudaError_t launch_bwd_t(BwdOp op, const RowBwdArgs& a, float* dgain, float* dtheta, cudaStream_t s) {
+    switch (op) {
+        case BwdOp::kRms: return launch_bwd_op<T, BwdOp::kRms>(a, dgain, dtheta, s);
+        case BwdOp::kInputScale: return launch_bwd_op<T, BwdOp::kInputScale>(a, dgain, dtheta, s);
+        case BwdOp::kResidual: return launch_bwd_op<T, BwdOp::kResidual>(a, dgain, dtheta, s);
+        case BwdOp::kResidualIS: return launch_bwd_op<T, BwdOp::kResidualIS>(a, dgain, dtheta, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+size_t row_bwd_workspace_bytes(int64_t rows, int32_t width) {
+    const int64_t grid = min(rows, (int64_t)bwd_grid_cap());
+    return (size_t)(grid < 1 ? 1 : grid) * (size_t)width * sizeof(float) * 2;
+}
+
+cudaError_t launch_row_bwd(int dtype, BwdOp op, RowBwdArgs a, float* dgain, float* dtheta, cudaStream_t s) {
+    return dtype == 0 ? launch_bwd_t<__nv_bfloat16>(op, a, dgain, dtheta, s)
+                      : launch_bwd_t<float>(op, a, dgain, dtheta, s);
+}
+
+cudaError_t read_bwd_device_error(unsigned int* out, bool clear) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_device_error, sizeof(unsigned int));
+    if (e == cudaSuccess && clear) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
+    }
+    return e;
+}
+
+}  // namespace muse

@@ -139,6 +139,13 @@ def theta(wl: Workload, seed: int, tag: str = "theta") -> torch.Tensor:
     return u * float(math.pi / 2)
 
 
+def upstream_grad(wl: Workload, seed: int, tag: str, shape, dtype=torch.bfloat16) -> torch.Tensor:
+    """Incoming gradient dL/d(output) for the backward calls: N(0, 1) drawn in
+    FP32 and rounded to dtype (no outlier channels)."""
+    x = torch.randn(shape, generator=_gen(seed, wl.name, "grad", tag), dtype=torch.float32)
+    return x.to(dtype)
+
+
 @dataclass
 class CoreInputs:
     """Host tensors for one core on one workload."""

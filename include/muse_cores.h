@@ -39,6 +39,7 @@
 #ifndef MUSE_CORES_H
 #define MUSE_CORES_H
 
+#include <stddef.h>
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
@@ -159,13 +160,87 @@ muse_status muse_norm_residual(const float* stream_in, const void* branch, float
                                const float* gain, float gain_offset, const float* theta,
                                int input_scale, float norm_eps, cudaStream_t stream);
 
+/* ------------------------------------------------------------------ backward
+ *
+ * The cores run under autograd: the layers page keeps them outside
+ * activation-checkpoint caching while "autograd and the enclosing activation
+ * checkpoint still run" (_checkpoint_recomputed_math).  The backward calls
+ * below compute the derivative of each forward map from the saved forward
+ * inputs (r is recomputed), in FP32, where every dtype boundary the forward
+ * materialises passes the gradient back rounded to that tensor's dtype, as
+ * autograd does through a cast.  Input gradients keep the input dtype;
+ * parameter gradients (gain, theta) are FP32 sums over all rows, reduced in a
+ * fixed order (bit-reproducible on a given GPU model).
+ *
+ * Parameter gradients need a caller-owned device workspace of
+ * muse_norm_backward_workspace_bytes(rows, hidden) bytes (16-byte aligned;
+ * it holds one partial row per CTA; contents on entry are ignored, on return
+ * undefined).  Pass dgain / dtheta = NULL to skip a parameter gradient; the
+ * workspace may then be NULL too.  Backward rows are limited to 1024 16-byte
+ * vectors (8192 bf16 or 4096 f32 elements); wider rows return
+ * MUSE_ERR_UNSUPPORTED.  Aliasing: dx may be the very same memory as x or dy
+ * (dstream_in as dstream_out, dbranch as branch); dgain, dtheta and the
+ * workspace must not overlap anything.  With rows == 0, dgain / dtheta are
+ * set to zero.
+ */
+
+/* Workspace bytes the row backward calls need for `rows` rows of `hidden`
+ * elements on the current device (0 for invalid sizes). */
+size_t muse_norm_backward_workspace_bytes(int64_t rows, int64_t hidden);
+
+/*
+ * Backward of core 1 (_rms_norm_core).  With w = gain + gain_offset (or 1),
+ * r = 1/sqrt(mean(x^2) + eps):
+ *   g = dy * w;  dx = r g - r^3 x (sum_j g_j x_j) / hidden;
+ *   dgain[j] = sum over rows of dy[j] x[j] r   (when dgain != NULL).
+ * x, dy, dx [rows, hidden] in dtype with their own row strides (elements).
+ */
+muse_status muse_rms_norm_backward(const void* x, const void* dy, void* dx, muse_dtype dtype,
+                                   int64_t rows, int64_t hidden, int64_t x_row_stride,
+                                   int64_t dy_row_stride, int64_t dx_row_stride,
+                                   const float* gain, float gain_offset, float eps, float* dgain,
+                                   void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Backward of core 2 (_input_scale_norm_core).  z = x w, r = r(z):
+ *   dz = r dy - r^3 z (sum_j dy_j z_j) / hidden;  dx = dz w;
+ *   dgain[j] = sum over rows of dz[j] x[j].
+ */
+muse_status muse_input_scale_norm_backward(const void* x, const void* dy, void* dx,
+                                           muse_dtype dtype, int64_t rows, int64_t hidden,
+                                           int64_t x_row_stride, int64_t dy_row_stride,
+                                           int64_t dx_row_stride, const float* gain,
+                                           float gain_offset, float eps, float* dgain,
+                                           void* workspace, size_t workspace_bytes,
+                                           cudaStream_t stream);
+
+/*
+ * Backward of core 5 (_norm_residual_core, blend h' = cos(theta) h +
+ * sin(theta) nb).  Given the forward's stream_in h, branch and theta, and
+ * dstream_out = dL/dh':
+ *   dstream_in = cos(theta) dstream_out                       (FP32);
+ *   dnb = cast_branch(sin(theta) dstream_out);
+ *   dbranch = the core 1 (input_scale == 0) or core 2 backward of dnb;
+ *   dgain = that backward's gain gradient;
+ *   dtheta[j] = sum over rows of dstream_out (-sin(theta) h + cos(theta) nb),
+ *     nb the forward's cast normalised branch.
+ * All rows contiguous [rows, hidden].
+ */
+muse_status muse_norm_residual_backward(const float* stream_in, const void* branch,
+                                        const float* dstream_out, float* dstream_in,
+                                        void* dbranch, muse_dtype branch_dtype, int64_t rows,
+                                        int64_t hidden, const float* gain, float gain_offset,
+                                        const float* theta, int input_scale, float norm_eps,
+                                        float* dgain, float* dtheta, void* workspace,
+                                        size_t workspace_bytes, cudaStream_t stream);
+
 /*
  * Device-side error flags of the current device, for diagnostics.  The row
- * kernels (cores 1, 2, 5, core 4 per token) and the Q/K kernel (core 3) stream
- * their inputs through shared memory with bulk copies tracked by mbarriers;
- * every wait on one is bounded, and a wait that gives up sets bit 0 (row
- * kernels) or bit 1 (Q/K kernel) of the flags (and the affected warps stop
- * writing).  *flags receives them; clear != 0 resets them.  Synchronous: it
+ * kernels (cores 1, 2, 5, core 4 per token), the Q/K kernel (core 3) and the
+ * row backward kernels stream their inputs through shared memory with bulk
+ * copies tracked by mbarriers; every wait on one is bounded, and a wait that
+ * gives up sets bit 0 (row kernels), bit 1 (Q/K kernel) or bit 2 (row
+ * backward) of the flags (and the affected warps stop writing).  *flags receives them; clear != 0 resets them.  Synchronous: it
  * waits for the device.  Returns MUSE_ERR_INVALID_ARGUMENT for a NULL flags
  * pointer, MUSE_ERR_CUDA if the copy fails.
  */
