@@ -459,16 +459,33 @@ int muse_oracle_norm_residual(const float* stream, int branch_dtype, const void*
 
 typedef struct {
     double lo, hi, rn; /* bracket and the round-to-nearest path value */
+    double m;          /* magnitude its FP32 evaluation error is relative to */
 } ival;
 
-static ival iv_exact(double v) { ival r = {v, v, v}; return r; }
+static ival iv_exact(double v) { ival r = {v, v, v, fabs(v)}; return r; }
 
 static ival iv_cast(int dtype, double v, int round) {
     if (!round) return iv_exact(v);
     double c[2];
     const int n = cast_candidates(dtype, v, c);
-    ival r = {c[0], c[0], c[0]};
-    if (n == 2) { r.lo = fmin(c[0], c[1]); r.hi = fmax(c[0], c[1]); }
+    ival r = {c[0], c[0], c[0], fabs(c[0])};
+    if (n == 2) { r.lo = fmin(c[0], c[1]); r.hi = fmax(c[0], c[1]); r.m = fmax(fabs(r.lo), fabs(r.hi)); }
+    return r;
+}
+
+/* A cast whose argument is an FP32-evaluated sum of terms of total magnitude
+ * `terms`: its evaluation error is relative to `terms`, not to the possibly
+ * cancelling value, so every bf16 value within 2^-20 * max(|v|, terms) of v
+ * is an admissible result (the rule of cast_candidates with the sum's own
+ * magnitude); an FP32 cast keeps one value and carries `terms` forward as
+ * the magnitude later allowances scale with. */
+static ival iv_cast_sum(int dtype, double v, double terms, int round) {
+    const double m = fmax(fabs(v), terms);
+    if (!round) { ival r = {v, v, v, m}; return r; }
+    if (dtype != DT_BF16) { const double f = cast_to(dtype, v); ival r = {f, f, f, m}; return r; }
+    const double d = m * MUSE_ORACLE_AMBIG_REL;
+    ival r = {bf16_round(v - d), bf16_round(v + d), bf16_round(v), 0.0};
+    r.m = fmax(fabs(r.lo), fabs(r.hi));
     return r;
 }
 
@@ -479,11 +496,12 @@ static ival iv_scale(ival a, double s) {
     const double p = a.lo * s, q = a.hi * s;
     r.lo = fmin(p, q);
     r.hi = fmax(p, q);
+    r.m = a.m * fabs(s);
     return r;
 }
 
 static ival iv_add(ival a, ival b) {
-    ival r = {a.lo + b.lo, a.hi + b.hi, a.rn + b.rn};
+    ival r = {a.lo + b.lo, a.hi + b.hi, a.rn + b.rn, a.m + b.m};
     return r;
 }
 
@@ -512,13 +530,13 @@ static void norm_row_bwd(int mode, int64_t H, const double* x, const double* w, 
     for (int64_t j = 0; j < H; ++j) {
         const double f = mode ? x[j] * w[j] : w[j] * x[j];
         C = iv_add(C, iv_scale(g[j], f));
-        Cabs += iv_absmax(g[j]) * fabs(f);
+        Cabs += g[j].m * fabs(f);
     }
     for (int64_t k = 0; k < H; ++k) {
         const double u = mode ? x[k] * w[k] : x[k];
         const double a = mode ? r : r * w[k];
         ival d = iv_add(iv_scale(g[k], a), iv_scale(C, -r3 * u / (double)H));
-        double m = iv_absmax(g[k]) * fabs(a) + r3 * fabs(u) * Cabs / (double)H;
+        double m = g[k].m * fabs(a) + r3 * fabs(u) * Cabs / (double)H;
         if (mode) {
             if (dw_term) {
                 dw_term[k] = iv_scale(d, x[k]);
@@ -528,7 +546,7 @@ static void norm_row_bwd(int mode, int64_t H, const double* x, const double* w, 
             m *= fabs(w[k]);
         } else if (dw_term) {
             dw_term[k] = iv_scale(g[k], x[k] * r);
-            dw_mag[k] = iv_absmax(g[k]) * fabs(x[k] * r);
+            dw_mag[k] = g[k].m * fabs(x[k] * r);
         }
         dx[k] = d;
         dx_mag[k] = m;
@@ -736,8 +754,16 @@ static void qk_head_bwd(int dtype, const void* x, const void* dy, int64_t base, 
             m1 = y1;
         }
         const double m[2] = {m0, m1};
+        /* magnitudes of the two products forming each component */
+        double t[2] = {fabs(y0), fabs(y1)};
+        if (use_rope) {
+            const float phi = (float)pos * inv_freq[i];
+            const double c = cos((double)phi), s = sin((double)phi);
+            t[0] = fabs(c * y0) + fabs(s * y1);
+            t[1] = fabs(s * y0) + fabs(c * y1);
+        }
         for (int e = 0; e < 2; ++e) {
-            const ival n2 = iv_cast(dtype, m[e], round_grads);
+            const ival n2 = iv_cast_sum(dtype, m[e], t[e], round_grads);
             ival n1 = n2;
             if (is_query) {
                 /* each admissible dn2 scaled, then cast again */
@@ -747,6 +773,7 @@ static void qk_head_bwd(int dtype, const void* x, const void* dy, int64_t base, 
                 n1.lo = fmin(fmin(a.lo, b.lo), fmin(a.hi, b.hi));
                 n1.hi = fmax(fmax(a.lo, b.lo), fmax(a.hi, b.hi));
                 n1.rn = p.rn;
+                n1.m = fmax(n2.m * fabs((double)query_scale), fmax(fabs(n1.lo), fabs(n1.hi)));
             }
             gr[2 * i + e] = n1;
         }

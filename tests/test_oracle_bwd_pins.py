@@ -17,7 +17,6 @@ import torch
 
 import oracle
 
-torch.set_default_dtype(torch.float64)
 REL = 1e-12
 
 
