@@ -57,6 +57,19 @@ def algo_bytes(wl, core: str, tokens: int) -> int:
     return per_tok * tokens + fixed
 
 
+def algo_bytes_bwd(wl, core: str, tokens: int) -> int:
+    """Minimum HBM bytes of one backward launch (bf16 activations, FP32 stream):
+    the forward inputs and the incoming gradient read once, every gradient
+    written once; gains / angles and their gradients once per launch."""
+    H, D = wl.hidden, wl.head_dim
+    per_tok = {"rms_norm": 6 * H, "input_scale_norm": 6 * H,
+               "qk_norm_rope": 6 * (wl.hq + wl.hkv) * D + (4 if wl.positions == "uniform" else 0),
+               "output_norm_gate": 10 * wl.hq * D, "norm_residual": 16 * H}[core]
+    fixed = {"rms_norm": 8 * H, "input_scale_norm": 8 * H, "qk_norm_rope": 0,
+             "output_norm_gate": 0, "norm_residual": 16 * H}[core]
+    return per_tok * tokens + fixed
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -203,8 +216,74 @@ class Step:
         return list(self.out.values())
 
 
-def per_core_isolated(st: "Step", peak: float, flush: torch.Tensor | None, warmup: int = 10,
-                      reps: int = 50):
+class BwdStep:
+    """Device-resident inputs, incoming gradients, gradient outputs and the
+    parameter-gradient workspace of the five backward calls for one batch;
+    launch() calls the C ABI directly on preallocated buffers."""
+
+    def __init__(self, st: "Step", seed: int):
+        from gate_cores_b200 import _lib
+        self.lib = _lib
+        self.wl, self.T, self.st = st.wl, st.T, st
+        wl, d = st.wl, st.dev
+        g = lambda tag, like: inputs.upstream_grad(wl, seed, tag, tuple(like.shape), like.dtype).cuda()
+        self.dy = {
+            "rms_norm": g("rms_norm", d["rms_norm"]["x"]),
+            "input_scale_norm": g("input_scale_norm", d["input_scale_norm"]["x"]),
+            "qk_q": g("qk_q", d["qk_norm_rope"]["q"]),
+            "qk_k": g("qk_k", d["qk_norm_rope"]["k"]),
+            "output_norm_gate": g("output_norm_gate", d["output_norm_gate"]["o"]),
+            "norm_residual": g("norm_residual", d["norm_residual"]["stream"]),
+        }
+        self.out = {
+            "rms_norm": torch.empty_like(d["rms_norm"]["x"]),
+            "input_scale_norm": torch.empty_like(d["input_scale_norm"]["x"]),
+            "dq": torch.empty_like(d["qk_norm_rope"]["q"]),
+            "dk": torch.empty_like(d["qk_norm_rope"]["k"]),
+            "do": torch.empty_like(d["output_norm_gate"]["o"]),
+            "dg": torch.empty_like(d["output_norm_gate"]["o"]),
+            "dstream": torch.empty_like(d["norm_residual"]["stream"]),
+            "dbranch": torch.empty_like(d["norm_residual"]["branch"]),
+        }
+        H = wl.hidden
+        self.dparam = {c: torch.empty(H, dtype=torch.float32, device="cuda")
+                       for c in ("rms_norm", "input_scale_norm", "gain_res", "theta_res")}
+        self.ws_bytes = _lib.muse_norm_backward_workspace_bytes(self.T, H)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
+
+    def launch(self, core: str):
+        L, wl, T, H = self.lib, self.wl, self.T, self.wl.hidden
+        d, sc = self.st.dev[core], self.st.host[core].scalars
+        stream = torch.cuda.current_stream().cuda_stream
+        bf = L.MUSE_DTYPE_BF16
+        if core in ("rms_norm", "input_scale_norm"):
+            fn = L.muse_rms_norm_backward if core == "rms_norm" else L.muse_input_scale_norm_backward
+            fn(d["x"].data_ptr(), self.dy[core].data_ptr(), self.out[core].data_ptr(), bf, T, H, H, H, H,
+               d["gain"].data_ptr(), sc["gain_offset"], sc["eps"], self.dparam[core].data_ptr(),
+               self.ws.data_ptr(), self.ws_bytes, stream)
+        elif core == "qk_norm_rope":
+            qw, kw = wl.hq * wl.head_dim, wl.hkv * wl.head_dim
+            pos = d["positions"]
+            L.muse_qk_norm_rope_backward(
+                d["q"].data_ptr(), d["k"].data_ptr(), self.dy["qk_q"].data_ptr(), self.dy["qk_k"].data_ptr(),
+                self.out["dq"].data_ptr(), self.out["dk"].data_ptr(), bf, L.MUSE_LAYOUT_BSHD, wl.batch,
+                wl.seqlen, None, 0, T, None if pos is None else pos.data_ptr(), wl.hq, wl.hkv,
+                wl.head_dim, qw, kw, qw, kw, qw, kw, sc["eps"], 1.0, True, sc["rope_base"], stream)
+        elif core == "output_norm_gate":
+            L.muse_output_norm_gate_backward(
+                d["o"].data_ptr(), d["g"].data_ptr(), self.dy[core].data_ptr(), self.out["do"].data_ptr(),
+                self.out["dg"].data_ptr(), bf, T, wl.hq, wl.head_dim, wl.head_dim, sc["eps"], stream)
+        else:
+            L.muse_norm_residual_backward(
+                d["stream"].data_ptr(), d["branch"].data_ptr(), self.dy[core].data_ptr(),
+                self.out["dstream"].data_ptr(), self.out["dbranch"].data_ptr(), bf, T, H,
+                d["gain"].data_ptr(), sc["gain_offset"], d["theta"].data_ptr(), False, sc["norm_eps"],
+                self.dparam["gain_res"].data_ptr(), self.dparam["theta_res"].data_ptr(),
+                self.ws.data_ptr(), self.ws_bytes, stream)
+
+
+def per_core_isolated(st, peak: float, flush: torch.Tensor | None, warmup: int = 10,
+                      reps: int = 50, nbytes=None):
     """Each core launched alone: `warmup` launches, then the median of `reps`
     launches timed with CUDA events around each one on the launching stream.
     With `flush`, a read pass over that buffer (> L2, reading leaves no dirty
@@ -229,7 +308,7 @@ def per_core_isolated(st: "Step", peak: float, flush: torch.Tensor | None, warmu
                 ev.append((e0, e1))
         torch.cuda.synchronize()
         us = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
-        nb = algo_bytes(st.wl, c, st.T)
+        nb = (nbytes or algo_bytes)(st.wl, c, st.T)
         gbs = nb / (us * 1e-6) / 1e9
         out[c] = {"us": round(us, 3), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
     return out
@@ -425,7 +504,36 @@ def run_ours(args, world, rank, local):
     decode_warm = per_core_isolated(dec, peak, None)
     decode = {c: {"us_cold_l2": decode_cold[c]["us"], "us_warm_l2": decode_warm[c]["us"]}
               for c in CORE_ORDER}
-    del flush, dec
+    del dec
+    # Backward of the five cores on the same batch: each call alone (L2
+    # read-flushed, median of 50) and the five back to back (K steps timed
+    # with two events, as the forward step).
+    bst = BwdStep(st, seed=rank)
+    bwd_iso = per_core_isolated(bst, peak, flush, nbytes=algo_bytes_bwd)
+    for _ in range(3):
+        for c in CORE_ORDER:
+            bst.launch(c)
+    barrier(world)
+    torch.cuda.synchronize()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0.record(stream)
+    for _ in range(args.steps):
+        for c in CORE_ORDER:
+            bst.launch(c)
+    b1.record(stream)
+    torch.cuda.synchronize()
+    bwd_el = allreduce_max(b0.elapsed_time(b1) / 1e3, world)
+    bwd_bytes = sum(algo_bytes_bwd(wl, c, T) for c in CORE_ORDER)
+    backward = {"tokens_per_s": round(world * T * args.steps / bwd_el, 1),
+                "ms_per_step": round(bwd_el / args.steps * 1e3, 5),
+                "gbs": round(bwd_bytes * args.steps / bwd_el / 1e9, 1),
+                "frac": round(bwd_bytes * args.steps / bwd_el / 1e9 / peak, 4),
+                "algo_bytes_per_step": bwd_bytes,
+                "gpu_launches_per_step": 9,
+                "per_core_isolated": bwd_iso,
+                "note": "gradients of the five cores (the Q/K call with the FP32 rotation); gain and "
+                        "theta gradients reduced through the caller's workspace"}
+    del bst, flush
     torch.cuda.empty_cache()
 
     e2e = run_e2e(st, args, world) if args.e2e else None
@@ -449,6 +557,7 @@ def run_ours(args, world, rank, local):
             "per_core": per_core,
             "per_core_isolated": isolated,
             "decode_t128_h4096_latency": decode,
+            "backward": backward,
             "roofline": roofline,
             "copy_kernel_gbs": None if copy_gbs is None else round(copy_gbs, 1),
             "e2e": e2e,
