@@ -31,6 +31,8 @@ EXPORTS = (
     "muse_norm_residual", "muse_device_error", "muse_stream_copy",
     "muse_norm_backward_workspace_bytes", "muse_rms_norm_backward",
     "muse_input_scale_norm_backward", "muse_norm_residual_backward",
+    "muse_output_norm_gate_backward", "muse_qk_norm_rope_backward",
+    "muse_rms_norm_backward_noalloc",
 )
 
 
@@ -81,6 +83,13 @@ def load() -> ctypes.CDLL:
         lib.muse_input_scale_norm_backward.argtypes = rbwd
         lib.muse_norm_residual_backward.argtypes = [P, P, P, P, P, c_int, i64, i64, P, f32, P,
                                                     c_int, f32, P, P, P, sz, P]
+        lib.muse_rms_norm_backward_noalloc.argtypes = [P, P, P, c_int, i64, i64, i64, i64, i64, P,
+                                                       f32, f32, P, P]
+        lib.muse_output_norm_gate_backward.argtypes = [P, P, P, P, P, c_int, i64, i32, i32, i32,
+                                                       f32, P]
+        lib.muse_qk_norm_rope_backward.argtypes = [P, P, P, P, P, P, c_int, c_int, i64, i64, P,
+                                                   i32, i64, P, i32, i32, i32, i64, i64, i64, i64,
+                                                   i64, i64, f32, f32, c_int, f32, P]
         for name in EXPORTS[3:]:
             getattr(lib, name).restype = c_int
         lib.muse_norm_backward_workspace_bytes.restype = sz
@@ -178,3 +187,26 @@ def muse_norm_residual_backward(stream_in, branch, dstream_out, dstream_in, dbra
     _call("muse_norm_residual_backward", stream_in, branch, dstream_out, dstream_in, dbranch,
           branch_dtype, rows, hidden, gain, gain_offset, theta, int(input_scale), norm_eps, dgain,
           dtheta, workspace, workspace_bytes, stream)
+
+
+def muse_output_norm_gate_backward(o, gate, dy, d_o, dgate, dtype, tokens, heads, head_dim,
+                                   norm_group, eps, stream) -> None:
+    _call("muse_output_norm_gate_backward", o, gate, dy, d_o, dgate, dtype, tokens, heads, head_dim,
+          norm_group, eps, stream)
+
+
+def muse_qk_norm_rope_backward(q, k, dq_out, dk_out, dq, dk, dtype, layout, batch, seqlen,
+                               cu_seqlens, num_seqs, total_tokens, positions, hq, hkv, head_dim,
+                               q_tok_stride, k_tok_stride, dq_out_tok_stride, dk_out_tok_stride,
+                               dq_tok_stride, dk_tok_stride, eps, query_scale, use_rope, rope_base,
+                               stream) -> None:
+    _call("muse_qk_norm_rope_backward", q, k, dq_out, dk_out, dq, dk, dtype, layout, batch, seqlen,
+          cu_seqlens, num_seqs, total_tokens, positions, hq, hkv, head_dim, q_tok_stride,
+          k_tok_stride, dq_out_tok_stride, dk_out_tok_stride, dq_tok_stride, dk_tok_stride, eps,
+          query_scale, int(use_rope), rope_base, stream)
+
+
+def muse_rms_norm_backward_noalloc(x, dy, dx, dtype, rows, hidden, x_row_stride, dy_row_stride,
+                                   dx_row_stride, gain, gain_offset, eps, dgain, stream) -> None:
+    _call("muse_rms_norm_backward_noalloc", x, dy, dx, dtype, rows, hidden, x_row_stride,
+          dy_row_stride, dx_row_stride, gain, gain_offset, eps, dgain, stream)

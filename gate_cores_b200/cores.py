@@ -269,3 +269,58 @@ def norm_residual_backward(stream_in, branch, dstream_out, theta, gain=None,
         theta.contiguous().data_ptr(), input_scale, norm_eps, _ptr(dgain), _ptr(dtheta), _ptr(ws),
         0 if ws is None else ws.numel(), _stream(stream))
     return dsi, db, dgain, dtheta
+
+
+def output_norm_gate_backward(o, gate, dy, norm_group=None, eps: float = 1e-6, stream=None):
+    """Backward of core 4: returns (d_o, dgate)."""
+    _cuda(o, gate, dy)
+    if gate.shape != o.shape or dy.shape != o.shape or gate.dtype != o.dtype or dy.dtype != o.dtype:
+        raise ValueError("gate and dy must match o")
+    if not (o.is_contiguous() and gate.is_contiguous() and dy.is_contiguous()):
+        raise ValueError("o, gate and dy must be contiguous")
+    heads, d = o.shape[-2], o.shape[-1]
+    tokens = o.numel() // (heads * d)
+    d_o = torch.empty_like(o)
+    dg = torch.empty_like(o)
+    ng = d if norm_group is None else norm_group
+    _lib.muse_output_norm_gate_backward(o.data_ptr(), gate.data_ptr(), dy.data_ptr(), d_o.data_ptr(),
+                                        dg.data_ptr(), _dtype(o), tokens, heads, d, ng, eps,
+                                        _stream(stream))
+    return d_o, dg
+
+
+def qk_norm_rope_backward(q, k, dq_out, dk_out, positions=None, cu_seqlens=None, eps: float = 1e-6,
+                          query_scale: float = 1.0, use_rope: bool = True,
+                          rope_base: float = 10000.0, stream=None):
+    """Backward of core 3 (FP32 rotation): returns (dq, dk) shaped like q, k.
+    Layout and positions as in qk_norm_rope."""
+    _cuda(q, k, dq_out, dk_out, positions, cu_seqlens)
+    if q.dim() == 4:
+        layout, batch, seqlen, T = _lib.MUSE_LAYOUT_BSHD, q.shape[0], q.shape[1], q.shape[0] * q.shape[1]
+    elif q.dim() == 3:
+        T = q.shape[0]
+        if cu_seqlens is not None:
+            layout, batch, seqlen = _lib.MUSE_LAYOUT_THD, 0, 0
+        else:
+            layout, batch, seqlen = _lib.MUSE_LAYOUT_BSHD, 1, T
+    else:
+        raise ValueError("q must be [B,S,Hq,D] or [T,Hq,D]")
+    hq, d = q.shape[-2], q.shape[-1]
+    hkv = k.shape[-2]
+    if dq_out.shape != q.shape or dk_out.shape != k.shape:
+        raise ValueError("incoming gradients must match q and k")
+    dq = torch.empty_like(q, memory_format=torch.contiguous_format)
+    dk = torch.empty_like(k, memory_format=torch.contiguous_format)
+    if positions is not None:
+        positions = positions.contiguous()
+    num_seqs = 0
+    if cu_seqlens is not None:
+        cu_seqlens = cu_seqlens.contiguous()
+        num_seqs = cu_seqlens.numel() - 1
+    _lib.muse_qk_norm_rope_backward(
+        q.data_ptr(), k.data_ptr(), dq_out.data_ptr(), dk_out.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+        _dtype(q), layout, batch, seqlen, _ptr(cu_seqlens), num_seqs, T, _ptr(positions), hq, hkv, d,
+        _tok_stride(q, hq, d), _tok_stride(k, hkv, d), _tok_stride(dq_out, hq, d),
+        _tok_stride(dk_out, hkv, d), _tok_stride(dq, hq, d), _tok_stride(dk, hkv, d), eps,
+        query_scale, use_rope, rope_base, _stream(stream))
+    return dq, dk

@@ -120,10 +120,9 @@ muse_status row_entry(muse::RowOp op, const void* x, void* y, muse_dtype dtype, 
 
 // Shared checks of the row backward entry points: the workspace and the
 // parameter-gradient outputs must not overlap each other or any tensor.
-muse_status bwd_workspace_check(const char* name, int64_t rows, int64_t hidden, void* ws,
-                                size_t ws_bytes, bool needed) {
+muse_status bwd_workspace_check(const char* name, size_t need, void* ws, size_t ws_bytes,
+                                bool needed) {
     if (!needed) return MUSE_OK;
-    const size_t need = muse::row_bwd_workspace_bytes(rows, (int32_t)hidden);
     if (!ws || ws_bytes < need)
         return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: workspace of %zu bytes needed, %zu given", name, need,
                     ws ? ws_bytes : (size_t)0);
@@ -163,7 +162,9 @@ muse_status row_bwd_entry(bool input_scale, const void* x, const void* dy, void*
         return fail(MUSE_ERR_UNSUPPORTED, "%s: gain / dgain not 16-byte aligned", name);
     if (hidden / vec_elems(dtype) > muse::kBwdMaxVectors)
         return fail(MUSE_ERR_UNSUPPORTED, "%s: rows of more than %d 16-byte vectors", name, muse::kBwdMaxVectors);
-    muse_status st = bwd_workspace_check(name, rows, hidden, ws, ws_bytes, dgain != nullptr);
+    // cores 1 and 2 use the gain half of the workspace only
+    muse_status st = bwd_workspace_check(name, muse::row_bwd_gain_scratch_bytes(rows, (int32_t)hidden),
+                                         ws, ws_bytes, dgain != nullptr);
     if (st != MUSE_OK) return st;
     const Span sx = span(x, rows, hidden, xs, es), sdy = span(dy, rows, hidden, dys, es);
     const Span sdx = span(dx, rows, hidden, dxs, es);
@@ -449,6 +450,26 @@ muse_status muse_rms_norm_backward(const void* x, const void* dy, void* dx, muse
                          stream, "muse_rms_norm_backward");
 }
 
+muse_status muse_rms_norm_backward_noalloc(const void* x, const void* dy, void* dx, muse_dtype dtype,
+                                           int64_t rows, int64_t hidden, int64_t x_row_stride,
+                                           int64_t dy_row_stride, int64_t dx_row_stride,
+                                           const float* gain, float gain_offset, float eps,
+                                           float* dgain, cudaStream_t stream) {
+    const char* name = "muse_rms_norm_backward_noalloc";
+    void* scratch = nullptr;
+    if (dgain && gain && rows > 0 && hidden > 0 && hidden <= ((int64_t)1 << 30)) {
+        const size_t need = muse::row_bwd_gain_scratch_bytes(rows, (int32_t)hidden);
+        if (need > muse::kNoAllocScratchBytes)
+            return fail(MUSE_ERR_UNSUPPORTED, "%s: gain partials need %zu bytes, the fixed scratch holds %zu",
+                        name, need, muse::kNoAllocScratchBytes);
+        const muse_status st = from_cuda(muse::noalloc_scratch(&scratch), name);
+        if (st != MUSE_OK) return st;
+    }
+    return row_bwd_entry(false, x, dy, dx, dtype, rows, hidden, x_row_stride, dy_row_stride,
+                         dx_row_stride, gain, gain_offset, eps, dgain, scratch,
+                         scratch ? muse::kNoAllocScratchBytes : 0, stream, name);
+}
+
 muse_status muse_input_scale_norm_backward(const void* x, const void* dy, void* dx,
                                            muse_dtype dtype, int64_t rows, int64_t hidden,
                                            int64_t x_row_stride, int64_t dy_row_stride,
@@ -492,7 +513,8 @@ muse_status muse_norm_residual_backward(const float* stream_in, const void* bran
         return fail(MUSE_ERR_UNSUPPORTED, "%s: theta / gain / dgain / dtheta not 16-byte aligned", name);
     if (hidden / vec_elems(branch_dtype) > muse::kBwdMaxVectors)
         return fail(MUSE_ERR_UNSUPPORTED, "%s: rows of more than %d 16-byte vectors", name, muse::kBwdMaxVectors);
-    muse_status st = bwd_workspace_check(name, rows, hidden, workspace, workspace_bytes, dgain || dtheta);
+    muse_status st = bwd_workspace_check(name, muse::row_bwd_workspace_bytes(rows, (int32_t)hidden),
+                                         workspace, workspace_bytes, dgain || dtheta);
     if (st != MUSE_OK) return st;
     const Span sh = span(stream_in, rows, hidden, hidden, 4), sdo = span(dstream_out, rows, hidden, hidden, 4);
     const Span sb = span(branch, rows, hidden, hidden, es), sdb = span(dbranch, rows, hidden, hidden, es);
@@ -527,14 +549,154 @@ muse_status muse_norm_residual_backward(const float* stream_in, const void* bran
     return from_cuda(muse::launch_row_bwd(branch_dtype, op, a, dgain, dtheta, stream), name);
 }
 
+muse_status muse_output_norm_gate_backward(const void* o, const void* gate, const void* dy, void* d_o,
+                                           void* dgate, muse_dtype dtype, int64_t tokens,
+                                           int32_t heads, int32_t head_dim, int32_t norm_group,
+                                           float eps, cudaStream_t stream) {
+    const char* name = "muse_output_norm_gate_backward";
+    if (!valid_dtype(dtype)) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, (int)dtype);
+    if (tokens < 0 || heads <= 0 || head_dim <= 0)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: tokens=%lld heads=%d head_dim=%d", name, (long long)tokens, heads, head_dim);
+    const int64_t width = (int64_t)heads * head_dim;
+    if (norm_group != head_dim && norm_group != width)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: norm_group=%d must be head_dim or heads*head_dim", name, norm_group);
+    if (!finite(eps) || eps < 0.0f) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: eps must be finite and >= 0", name);
+    if (tokens == 0) return MUSE_OK;
+    if (!o || !gate || !dy || !d_o || !dgate) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null tensor", name);
+    const int64_t es = elem_size(dtype);
+    if (!aligned(o, 16) || !aligned(gate, 16) || !aligned(dy, 16) || !aligned(d_o, 16) || !aligned(dgate, 16) ||
+        (head_dim * es) % 16)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: pointers and head_dim must be 16-byte multiples", name);
+    if (norm_group * es > MUSE_MAX_ROW_BYTES)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: norm group of %lld bytes exceeds %d", name, (long long)(norm_group * es), MUSE_MAX_ROW_BYTES);
+    const Span so = span(o, tokens, width, width, es), sg = span(gate, tokens, width, width, es);
+    const Span sdy = span(dy, tokens, width, width, es), sdo = span(d_o, tokens, width, width, es);
+    const Span sdg = span(dgate, tokens, width, width, es);
+    // do may coincide with o or dy, dgate with gate or dy; never with each other
+    bool bad = (!same_span(sdo, so) && !same_span(sdo, sdy) && any_overlap(sdo, {so, sdy})) || overlap(sdo, sg);
+    bad = bad || (!same_span(sdg, sg) && !same_span(sdg, sdy) && any_overlap(sdg, {sg, sdy})) || overlap(sdg, so);
+    bad = bad || overlap(sdo, sdg);
+    if (bad) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: an output partially overlaps an input", name);
+    muse::GateBwdArgs a{};
+    a.o = o;
+    a.gate = gate;
+    a.dy = dy;
+    a.d_o = d_o;
+    a.dgate = dgate;
+    a.rows = tokens * (width / norm_group);
+    a.width = norm_group;
+    a.eps = eps;
+    return from_cuda(muse::launch_gate_bwd(dtype, a, stream), name);
+}
+
+muse_status muse_qk_norm_rope_backward(const void* q, const void* k, const void* dq_out,
+                                       const void* dk_out, void* dq, void* dk, muse_dtype dtype,
+                                       muse_layout layout, int64_t batch, int64_t seqlen,
+                                       const int32_t* cu_seqlens, int32_t num_seqs,
+                                       int64_t total_tokens, const int32_t* positions, int32_t hq,
+                                       int32_t hkv, int32_t head_dim, int64_t q_tok_stride,
+                                       int64_t k_tok_stride, int64_t dq_out_tok_stride,
+                                       int64_t dk_out_tok_stride, int64_t dq_tok_stride,
+                                       int64_t dk_tok_stride, float eps, float query_scale,
+                                       int use_rope, float rope_base, cudaStream_t stream) {
+    const char* name = "muse_qk_norm_rope_backward";
+    if (!valid_dtype(dtype)) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, (int)dtype);
+    if (layout != MUSE_LAYOUT_BSHD && layout != MUSE_LAYOUT_THD)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown layout %d", name, (int)layout);
+    int64_t tokens;
+    if (layout == MUSE_LAYOUT_BSHD) {
+        if (batch < 0 || seqlen <= 0)
+            return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: batch=%lld seqlen=%lld", name, (long long)batch, (long long)seqlen);
+        tokens = batch * seqlen;
+    } else {
+        if (total_tokens < 0) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: total_tokens < 0", name);
+        tokens = total_tokens;
+    }
+    if (hkv <= 0 || hq <= 0 || hq % hkv)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: hq=%d must be a positive multiple of hkv=%d", name, hq, hkv);
+    if (head_dim <= 0 || (head_dim & 1))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: head_dim=%d must be positive and even", name, head_dim);
+    if (!finite(eps) || eps < 0.0f || !finite(query_scale))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: eps must be finite and >= 0, query_scale finite", name);
+    if (use_rope && !(finite(rope_base) && rope_base > 0.0f))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: rope_base must be finite and > 0", name);
+    const int64_t qw = (int64_t)hq * head_dim, kw = (int64_t)hkv * head_dim;
+    if (q_tok_stride < qw || dq_out_tok_stride < qw || dq_tok_stride < qw || k_tok_stride < kw ||
+        dk_out_tok_stride < kw || dk_tok_stride < kw)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: token strides must cover all heads", name);
+    const bool derive = use_rope && !positions;
+    if (tokens > 0 && derive && layout == MUSE_LAYOUT_THD && (!cu_seqlens || num_seqs < 1))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: THD without positions needs cu_seqlens and num_seqs >= 1", name);
+    if (tokens == 0) return MUSE_OK;
+    if (!q || !k || !dq_out || !dk_out || !dq || !dk) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null tensor", name);
+    const int64_t es = elem_size(dtype);
+    const void* ptrs[6] = {q, k, dq_out, dk_out, dq, dk};
+    for (const void* p : ptrs)
+        if (!aligned(p, 16)) return fail(MUSE_ERR_UNSUPPORTED, "%s: pointers must be 16-byte aligned", name);
+    const int64_t strides[6] = {q_tok_stride, k_tok_stride, dq_out_tok_stride, dk_out_tok_stride, dq_tok_stride, dk_tok_stride};
+    for (int64_t st : strides)
+        if ((st * es) % 16) return fail(MUSE_ERR_UNSUPPORTED, "%s: strides must be 16-byte multiples", name);
+    if ((head_dim * es) % 16 || head_dim / vec_elems(dtype) > 32 || head_dim / 2 > muse::kMaxHalfDim)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: head_dim=%d must be 16-byte multiple of at most 512 bytes", name, head_dim);
+    if ((positions && !aligned(positions, 4)) || (cu_seqlens && !aligned(cu_seqlens, 4)))
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: positions / cu_seqlens not 4-byte aligned", name);
+    const Span sq = span(q, tokens, qw, q_tok_stride, es), sk = span(k, tokens, kw, k_tok_stride, es);
+    const Span sgq = span(dq_out, tokens, qw, dq_out_tok_stride, es), sgk = span(dk_out, tokens, kw, dk_out_tok_stride, es);
+    const Span sdq = span(dq, tokens, qw, dq_tok_stride, es), sdk = span(dk, tokens, kw, dk_tok_stride, es);
+    // dq may coincide with q or dq_out, dk with k or dk_out
+    bool bad = (!same_span(sdq, sq) && !same_span(sdq, sgq) && any_overlap(sdq, {sq, sgq})) || any_overlap(sdq, {sk, sgk, sdk});
+    bad = bad || (!same_span(sdk, sk) && !same_span(sdk, sgk) && any_overlap(sdk, {sk, sgk})) || any_overlap(sdk, {sq, sgq});
+    if (use_rope && positions) {
+        const Span sp = span(positions, 1, tokens, tokens, 4);
+        bad = bad || overlap(sdq, sp) || overlap(sdk, sp);
+    }
+    if (derive && layout == MUSE_LAYOUT_THD) {
+        const Span sc = span(cu_seqlens, 1, (int64_t)num_seqs + 1, (int64_t)num_seqs + 1, 4);
+        bad = bad || overlap(sdq, sc) || overlap(sdk, sc);
+    }
+    if (bad) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: an output partially overlaps an input", name);
+    muse::QkBwdArgs A{};
+    muse::QkArgs& a = A.f;
+    a.q = q;
+    a.k = k;
+    a.q_out = dq;
+    a.k_out = dk;
+    a.positions = positions;
+    a.cu_seqlens = cu_seqlens;
+    a.tokens = tokens;
+    a.seqlen = layout == MUSE_LAYOUT_BSHD ? seqlen : 1;
+    a.q_stride = q_tok_stride;
+    a.k_stride = k_tok_stride;
+    a.q_out_stride = dq_tok_stride;
+    a.k_out_stride = dk_tok_stride;
+    a.num_seqs = num_seqs;
+    a.hq = hq;
+    a.hkv = hkv;
+    a.head_dim = head_dim;
+    a.split = 1;
+    a.pos_mode = positions ? 0 : (layout == MUSE_LAYOUT_BSHD ? 1 : 2);
+    a.eps = eps;
+    a.query_scale = query_scale;
+    if (use_rope)
+        for (int i = 0; i < head_dim / 2; ++i)
+            a.inv_freq[i] = (float)std::pow((double)rope_base, -(2.0 * i) / (double)head_dim);
+    A.gq = dq_out;
+    A.gk = dk_out;
+    A.gq_stride = dq_out_tok_stride;
+    A.gk_stride = dk_out_tok_stride;
+    return from_cuda(muse::launch_qk_bwd(dtype, use_rope, A, stream), name);
+}
+
 muse_status muse_device_error(unsigned int* flags, int clear) {
     if (!flags) return fail(MUSE_ERR_INVALID_ARGUMENT, "muse_device_error: null flags");
-    // bit 0: the row pipeline's word, bit 1: the Q/K ring's, bit 2: the row backward's
-    unsigned int row = 0, qk = 0, bwd = 0;
+    // bit 0: the row pipeline's word, bit 1: the Q/K ring's, bit 2: the row
+    // backward's, bit 3: the Q/K backward ring's
+    unsigned int row = 0, qk = 0, bwd = 0, qkb = 0;
     cudaError_t e = muse::read_device_error(&row, clear != 0);
     if (e == cudaSuccess) e = muse::read_qk_device_error(&qk, clear != 0);
     if (e == cudaSuccess) e = muse::read_bwd_device_error(&bwd, clear != 0);
-    *flags = (row ? 1u : 0u) | (qk ? 2u : 0u) | (bwd ? 4u : 0u);
+    if (e == cudaSuccess) e = muse::read_qk_bwd_device_error(&qkb, clear != 0);
+    *flags = (row ? 1u : 0u) | (qk ? 2u : 0u) | (bwd ? 4u : 0u) | (qkb ? 8u : 0u);
     return from_cuda(e, "muse_device_error");
 }
 

@@ -72,6 +72,12 @@ struct RowBwdArgs {
 // workspace it needs for `rows` rows of `width` elements.
 constexpr int kBwdMaxVectors = 1024;
 size_t row_bwd_workspace_bytes(int64_t rows, int32_t width);
+// Scratch of the allocation-free core 1 backward: bytes its gain partials need,
+// the fixed capacity, and the device address of the fixed array (looked up
+// once per device, then cached).
+size_t row_bwd_gain_scratch_bytes(int64_t rows, int32_t width);
+constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;
+cudaError_t noalloc_scratch(void** ptr);
 
 constexpr int kMaxHalfDim = 128;  // head_dim <= 256
 
@@ -93,6 +99,33 @@ struct QkArgs {
     float query_scale;
     float inv_freq[kMaxHalfDim];
 };
+
+// Backward of core 4 over contiguous groups of `width` elements (one head or
+// one token each): do and dgate from o, gate and dy.
+struct GateBwdArgs {
+    const void* o;
+    const void* gate;
+    const void* dy;
+    void* d_o;
+    void* dgate;
+    int64_t rows;     // groups
+    int32_t width;    // elements per group
+    float eps;
+};
+cudaError_t launch_gate_bwd(int dtype, const GateBwdArgs& a, cudaStream_t s);
+
+// Backward of core 3 (FP32 rotation or none): f holds the forward's inputs
+// (q, k, positions, layout, sizes, eps, query_scale, inv_freq) and, as
+// q_out / k_out, the gradient outputs dq / dk with their token strides; gq /
+// gk are the incoming gradients dL/dq_out, dL/dk_out.
+struct QkBwdArgs {
+    QkArgs f;
+    const void* gq;
+    const void* gk;
+    int64_t gq_stride, gk_stride;
+};
+cudaError_t launch_qk_bwd(int dtype, int use_rope, const QkBwdArgs& a, cudaStream_t s);
+cudaError_t read_qk_bwd_device_error(unsigned int* out, bool clear);
 
 // Returns cudaSuccess or the launch error.
 // launch_row: TMA-pipelined kernels (row_tma.cu), falling back to

@@ -23,6 +23,8 @@
 // columns in every row, so it accumulates its columns' gain / theta
 // gradients in registers and writes one partial row per CTA into the
 // caller's workspace, which a second kernel sums in a fixed order.
+#include <map>
+#include <mutex>
 #include <type_traits>
 
 #include "common.cuh"
@@ -410,6 +412,34 @@ cudaError_t launch_bwd_t(BwdOp op, const RowBwdArgs& a, float* dgain, float* dth
 }
 
 }  // namespace
+
+// Fixed scratch of the allocation-free gain-gradient call: one partial row
+// per CTA of the core 1 backward, kNoAllocScratchBytes at most (16 MiB: 1024
+// partial rows of 4096 FP32 columns).
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+cudaError_t noalloc_scratch(void** ptr) {
+    static std::mutex mu;
+    static std::map<int, void*> addr;  // per device, taken once
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = addr.find(dev);
+    if (it == addr.end()) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        it = addr.emplace(dev, p).first;
+    }
+    *ptr = it->second;
+    return cudaSuccess;
+}
+
+size_t row_bwd_gain_scratch_bytes(int64_t rows, int32_t width) {
+    const int64_t grid = min(rows, (int64_t)bwd_grid_cap());
+    return (size_t)(grid < 1 ? 1 : grid) * (size_t)width * sizeof(float);
+}
 
 size_t row_bwd_workspace_bytes(int64_t rows, int32_t width) {
     const int64_t grid = min(rows, (int64_t)bwd_grid_cap());

@@ -202,6 +202,29 @@ muse_status muse_rms_norm_backward(const void* x, const void* dy, void* dx, muse
                                    void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Allocation-free variant of muse_rms_norm_backward (an addition of this
+ * library; the API reference pages have no counterpart).  Same arguments and
+ * results, without the workspace: the gain partials (one row of `hidden` FP32
+ * values per CTA) go to a fixed 16 MiB device array of the library, whose
+ * address is looked up once per device on the first call that needs it.
+ *   - Allocates nothing and never calls cudaMalloc / cudaFree.
+ *   - Rejects with MUSE_ERR_UNSUPPORTED a call whose partials exceed the
+ *     fixed array (with hidden = 4096, up to 1024 partial rows: any row
+ *     count on a GPU whose backward grid stays at or below 1024 CTAs).
+ *   - The array is shared by every call on a device: two calls with dgain
+ *     must not run concurrently (issue them on one stream, or order their
+ *     streams); calls without dgain do not touch it.
+ *   - The first call with dgain on each device performs the address lookup,
+ *     which must not happen inside a stream capture: make that first call
+ *     outside any capture; later calls are capture-safe.
+ */
+muse_status muse_rms_norm_backward_noalloc(const void* x, const void* dy, void* dx, muse_dtype dtype,
+                                           int64_t rows, int64_t hidden, int64_t x_row_stride,
+                                           int64_t dy_row_stride, int64_t dx_row_stride,
+                                           const float* gain, float gain_offset, float eps,
+                                           float* dgain, cudaStream_t stream);
+
+/*
  * Backward of core 2 (_input_scale_norm_core).  z = x w, r = r(z):
  *   dz = r dy - r^3 z (sum_j dy_j z_j) / hidden;  dx = dz w;
  *   dgain[j] = sum over rows of dz[j] x[j].
@@ -235,12 +258,49 @@ muse_status muse_norm_residual_backward(const float* stream_in, const void* bran
                                         size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Backward of core 4 (_output_norm_gate_core).  Per norm group of G
+ * elements (norm_group = head_dim or heads*head_dim, as in the forward):
+ *   s = sigmoid(gate), n = o r(o), dn = dy s;
+ *   d_o = r dn - r^3 o (sum_j dn_j o_j) / G;   dgate = dy n s (1 - s).
+ * o, gate, dy, d_o, dgate contiguous [tokens, heads, head_dim] in dtype.
+ * d_o may be the very memory of o or dy, dgate of gate or dy.
+ */
+muse_status muse_output_norm_gate_backward(const void* o, const void* gate, const void* dy, void* d_o,
+                                           void* dgate, muse_dtype dtype, int64_t tokens,
+                                           int32_t heads, int32_t head_dim, int32_t norm_group,
+                                           float eps, cudaStream_t stream);
+
+/*
+ * Backward of core 3 (_qk_norm_rope_core) with the FP32 (legacy, upcast)
+ * rotation or none.  Per token and head, with phi the forward's FP32 angle
+ * (same positions rule and layouts as muse_qk_norm_rope):
+ *   dm = R(phi)^T dy, i.e. per pair (c dy0 + s dy1, -s dy0 + c dy1), FP32;
+ *   dn = cast(dm); query heads: dn = cast(dn * query_scale);
+ *   dx = r dn - r^3 x (sum_j dn_j x_j) / head_dim, cast to dtype.
+ * q, k are the forward's inputs; dq_out, dk_out the incoming gradients; dq,
+ * dk the results, each with its own token stride (elements).  dq may be the
+ * very memory of q or dq_out, dk of k or dk_out.  The v2 (bf16-product)
+ * rotation has no backward here.
+ */
+muse_status muse_qk_norm_rope_backward(const void* q, const void* k, const void* dq_out,
+                                       const void* dk_out, void* dq, void* dk, muse_dtype dtype,
+                                       muse_layout layout, int64_t batch, int64_t seqlen,
+                                       const int32_t* cu_seqlens, int32_t num_seqs,
+                                       int64_t total_tokens, const int32_t* positions, int32_t hq,
+                                       int32_t hkv, int32_t head_dim, int64_t q_tok_stride,
+                                       int64_t k_tok_stride, int64_t dq_out_tok_stride,
+                                       int64_t dk_out_tok_stride, int64_t dq_tok_stride,
+                                       int64_t dk_tok_stride, float eps, float query_scale,
+                                       int use_rope, float rope_base, cudaStream_t stream);
+
+/*
  * Device-side error flags of the current device, for diagnostics.  The row
  * kernels (cores 1, 2, 5, core 4 per token), the Q/K kernel (core 3) and the
- * row backward kernels stream their inputs through shared memory with bulk
+ * row and Q/K backward kernels stream their inputs through shared memory with bulk
  * copies tracked by mbarriers; every wait on one is bounded, and a wait that
- * gives up sets bit 0 (row kernels), bit 1 (Q/K kernel) or bit 2 (row
- * backward) of the flags (and the affected warps stop writing).  *flags receives them; clear != 0 resets them.  Synchronous: it
+ * gives up sets bit 0 (row kernels), bit 1 (Q/K kernel), bit 2 (row
+ * backward) or bit 3 (Q/K backward) of the flags (and the affected warps
+ * stop writing).  *flags receives them; clear != 0 resets them.  Synchronous: it
  * waits for the device.  Returns MUSE_ERR_INVALID_ARGUMENT for a NULL flags
  * pointer, MUSE_ERR_CUDA if the copy fails.
  */
