@@ -167,20 +167,35 @@ __device__ __forceinline__ void row_bwd_body(const RowBwdArgs& a) {
         valid[i] = tid + i * ncons < nvec;
         col[i] = valid[i] ? (tid + i * ncons) * V : 0;
     }
-    float w[VPT][V], cth[RES ? VPT : 1][V], sth[RES ? VPT : 1][V];
-    float acc_g[G ? VPT : 1][V], acc_t[RES ? VPT : 1][V];
+    // Element arithmetic on packed FP32 pairs (f32x2: two IEEE round-to-nearest
+    // operations per instruction); per-slot constants in registers.
+    constexpr int P = V / 2;
+    constexpr int SV = V / 4;  // 16-byte FP32 pieces per slot
+    f32x2 w[VPT][P], cth[RES ? VPT : 1][P], sth[RES ? VPT : 1][P], nsth[RES ? VPT : 1][P];
+    f32x2 acc_g[G ? VPT : 1][P], acc_t[RES ? VPT : 1][P];
+    {
+        const f32x2 off2 = f2_make(a.gain_offset, a.gain_offset);
+        const f32x2 zero = f2_make(0.0f, 0.0f);
 #pragma unroll
-    for (int i = 0; i < VPT; ++i) {
+        for (int i = 0; i < VPT; ++i) {
 #pragma unroll
-        for (int e = 0; e < V; ++e) {
-            w[i][e] = G ? __ldg(a.gain + col[i] + e) + a.gain_offset : 1.0f;  // FP32 sum
-            if constexpr (G) acc_g[i][e] = 0.0f;
-            if constexpr (RES) {
-                float sv, cv;
-                sincosf(__ldg(a.theta + col[i] + e), &sv, &cv);
-                cth[i][e] = cv;
-                sth[i][e] = sv;
-                acc_t[i][e] = 0.0f;
+            for (int q = 0; q < P; ++q) {
+                w[i][q] = f2_make(1.0f, 1.0f);
+                if constexpr (G) {
+                    const float2 g2 = __ldg(reinterpret_cast<const float2*>(a.gain + col[i]) + q);
+                    w[i][q] = f2_add(f2_make(g2.x, g2.y), off2);  // FP32 sums
+                    acc_g[i][q] = zero;
+                }
+                if constexpr (RES) {
+                    const float2 t2 = __ldg(reinterpret_cast<const float2*>(a.theta + col[i]) + q);
+                    float s0, c0, s1, c1;
+                    sincosf(t2.x, &s0, &c0);
+                    sincosf(t2.y, &s1, &c1);
+                    cth[i][q] = f2_make(c0, c1);
+                    sth[i][q] = f2_make(s0, s1);
+                    nsth[i][q] = f2_make(-s0, -s1);
+                    acc_t[i][q] = zero;
+                }
             }
         }
     }
@@ -198,26 +213,26 @@ __device__ __forceinline__ void row_bwd_body(const RowBwdArgs& a) {
         if (alive) alive = mbar_wait(&full_bar[s], phase);
         alive = __all_sync(0xffffffffu, alive);
         const unsigned char* st = smem + s * L.stage_bytes;
-        float x[VPT][V], g[VPT][V], h[RES ? VPT : 1][V];
+        f32x2 x[VPT][P], g[VPT][P], h[RES ? VPT : 1][P];
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
-            if (alive && valid[i]) {
-                ld_stage<T>(st + (uint32_t)col[i] * sizeof(T), x[i]);
-                if constexpr (RES) {
-                    ld_stage_f32<V>(st + L.dy_off + (uint32_t)col[i] * 4u, g[i]);
-                    ld_stage_f32<V>(st + L.h_off + (uint32_t)col[i] * 4u, h[i]);
-                } else {
-                    ld_stage<T>(st + L.dy_off + (uint32_t)col[i] * sizeof(T), g[i]);
+            const bool rd = alive && valid[i];
+            const uint32_t xo = (uint32_t)col[i] * sizeof(T);
+            to_pairs<T>(rd ? *reinterpret_cast<const uint4*>(st + xo) : make_uint4(0, 0, 0, 0), x[i]);
+            if constexpr (RES) {
+#pragma unroll
+                for (int q = 0; q < SV; ++q) {
+                    const uint32_t fo = (uint32_t)col[i] * 4u + 16u * q;
+                    to_pairs<float>(rd ? *reinterpret_cast<const uint4*>(st + L.dy_off + fo) : make_uint4(0, 0, 0, 0),
+                                    g[i] + 2 * q);
+                    to_pairs<float>(rd ? *reinterpret_cast<const uint4*>(st + L.h_off + fo) : make_uint4(0, 0, 0, 0),
+                                    h[i] + 2 * q);
                 }
             } else {
-#pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    x[i][e] = 0.0f;
-                    g[i][e] = 0.0f;
-                    if constexpr (RES) h[i][e] = 0.0f;
-                }
+                to_pairs<T>(rd ? *reinterpret_cast<const uint4*>(st + L.dy_off + xo) : make_uint4(0, 0, 0, 0), g[i]);
             }
         }
+        // this warp is done with the stage
         __syncwarp();
         if (lane == 0 && alive) mbar_arrive(&empty_bar[s]);
         if (++s == S) {
@@ -226,56 +241,61 @@ __device__ __forceinline__ void row_bwd_body(const RowBwdArgs& a) {
         }
 
         // core 5: the blend's gradient reaching the cast branch, rounded to it
-        float dh[RES ? VPT : 1][V];
+        f32x2 dh[RES ? VPT : 1][P];
         if constexpr (RES) {
 #pragma unroll
             for (int i = 0; i < VPT; ++i)
 #pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    dh[i][e] = g[i][e];
-                    g[i][e] = round_to<T>(sth[i][e] * dh[i][e]);
+                for (int q = 0; q < P; ++q) {
+                    dh[i][q] = g[i][q];
+                    g[i][q] = round_pair<T>(f2_mul(sth[i][q], dh[i][q]));
                 }
         }
         // row sums: mean square of the normalised input, gradient dot product
-        float ss = 0.0f, cd = 0.0f;
+        f32x2 ss2 = f2_make(0.0f, 0.0f), cd2 = f2_make(0.0f, 0.0f);
 #pragma unroll
         for (int i = 0; i < VPT; ++i)
 #pragma unroll
-            for (int e = 0; e < V; ++e) {
-                const float u = FIRST ? x[i][e] * w[i][e] : x[i][e];
-                ss = fmaf(u, u, ss);
-                cd = fmaf(FIRST ? g[i][e] : g[i][e] * w[i][e], u, cd);
+            for (int q = 0; q < P; ++q) {
+                const f32x2 u = FIRST ? f2_mul(x[i][q], w[i][q]) : x[i][q];
+                ss2 = f2_fma(u, u, ss2);
+                cd2 = f2_fma(FIRST ? g[i][q] : f2_mul(g[i][q], w[i][q]), u, cd2);
             }
-        const float2 tot = consumer_sum2(ss, cd, red, bank, ncons);
+        const float2 tot = consumer_sum2(f2_sum(ss2), f2_sum(cd2), red, bank, ncons);
         const float r = inv_rms_fast(tot.x, inv_width, a.eps);
         const float cr = r * r * r * tot.y * inv_width;
+        const f32x2 r2 = f2_make(r, r), ncr2 = f2_make(-cr, -cr);
 
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
-            float dx[V];
+            f32x2 d[P];
 #pragma unroll
-            for (int e = 0; e < V; ++e) {
+            for (int q = 0; q < P; ++q) {
                 if constexpr (FIRST) {
-                    const float u = x[i][e] * w[i][e];
-                    const float dz = r * g[i][e] - cr * u;
-                    dx[e] = dz * w[i][e];
-                    if constexpr (G) acc_g[i][e] = fmaf(dz, x[i][e], acc_g[i][e]);
+                    const f32x2 u = f2_mul(x[i][q], w[i][q]);
+                    const f32x2 dz = f2_fma(u, ncr2, f2_mul(r2, g[i][q]));
+                    d[q] = f2_mul(dz, w[i][q]);
+                    if constexpr (G) acc_g[i][q] = f2_fma(dz, x[i][q], acc_g[i][q]);
                 } else {
-                    dx[e] = (r * w[i][e]) * g[i][e] - cr * x[i][e];
-                    if constexpr (G) acc_g[i][e] = fmaf(g[i][e], x[i][e] * r, acc_g[i][e]);
+                    d[q] = f2_fma(x[i][q], ncr2, f2_mul(f2_mul(r2, w[i][q]), g[i][q]));
+                    if constexpr (G) acc_g[i][q] = f2_fma(g[i][q], f2_mul(x[i][q], r2), acc_g[i][q]);
                 }
             }
-            if (alive && valid[i]) st_vec(dx_row + (uint32_t)col[i] * sizeof(T), pack<T>(dx));
+            if (alive && valid[i]) st_vec(dx_row + (uint32_t)col[i] * sizeof(T), from_pairs<T>(d));
             if constexpr (RES) {
-                float dhs[V];
+                f32x2 dhs[P];
 #pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    dhs[e] = cth[i][e] * dh[i][e];
-                    const float v = FIRST ? (x[i][e] * w[i][e]) * r : (x[i][e] * r) * w[i][e];
-                    const float nb = round_to<T>(v);  // the forward's cast branch
-                    acc_t[i][e] = fmaf(dh[i][e], fmaf(-sth[i][e], h[i][e], cth[i][e] * nb), acc_t[i][e]);
+                for (int q = 0; q < P; ++q) {
+                    dhs[q] = f2_mul(cth[i][q], dh[i][q]);
+                    const f32x2 v = FIRST ? f2_mul(f2_mul(x[i][q], w[i][q]), r2) : f2_mul(f2_mul(x[i][q], r2), w[i][q]);
+                    const f32x2 nb = round_pair<T>(v);  // the forward's cast branch
+                    acc_t[i][q] = f2_fma(dh[i][q], f2_fma(nsth[i][q], h[i][q], f2_mul(cth[i][q], nb)), acc_t[i][q]);
                 }
-                if (alive && valid[i]) st_f32<V>(dh_row + col[i], dhs);
+                if (alive && valid[i]) {
+#pragma unroll
+                    for (int q = 0; q < SV; ++q)
+                        st_vec(dh_row + col[i] + 4 * q, from_pairs<float>(dhs + 2 * q));
+                }
             }
         }
         dx_row += dx_step;
@@ -287,20 +307,26 @@ __device__ __forceinline__ void row_bwd_body(const RowBwdArgs& a) {
     for (int i = 0; i < VPT; ++i) {
         if (!valid[i]) continue;
         if constexpr (G)
-            if (a.part_gain) st_f32<V>(a.part_gain + (int64_t)blockIdx.x * a.width + col[i], acc_g[i]);
+            if (a.part_gain)
+#pragma unroll
+                for (int q = 0; q < SV; ++q)
+                    st_vec(a.part_gain + (int64_t)blockIdx.x * a.width + col[i] + 4 * q, from_pairs<float>(acc_g[i] + 2 * q));
         if constexpr (RES)
-            if (a.part_theta) st_f32<V>(a.part_theta + (int64_t)blockIdx.x * a.width + col[i], acc_t[i]);
+            if (a.part_theta)
+#pragma unroll
+                for (int q = 0; q < SV; ++q)
+                    st_vec(a.part_theta + (int64_t)blockIdx.x * a.width + col[i] + 4 * q, from_pairs<float>(acc_t[i] + 2 * q));
     }
 }
 
 // One entry symbol per core.
 template <typename T, int VPT, bool G, int S>
-__global__ void __launch_bounds__(512 + 32) rms_norm_bwd_kernel(const __grid_constant__ RowBwdArgs a) {
+__global__ void __launch_bounds__(VPT == 1 ? 544 : 288, VPT == 2 ? 2 : 1) rms_norm_bwd_kernel(const __grid_constant__ RowBwdArgs a) {
     pdl_begin();
     row_bwd_body<T, BwdOp::kRms, VPT, G, S>(a);
 }
 template <typename T, int VPT, bool G, int S>
-__global__ void __launch_bounds__(512 + 32) input_scale_norm_bwd_kernel(const __grid_constant__ RowBwdArgs a) {
+__global__ void __launch_bounds__(VPT == 1 ? 544 : 288, VPT == 2 ? 2 : 1) input_scale_norm_bwd_kernel(const __grid_constant__ RowBwdArgs a) {
     pdl_begin();
     row_bwd_body<T, BwdOp::kInputScale, VPT, G, S>(a);
 }
@@ -323,24 +349,31 @@ constexpr auto row_bwd_kernel() {
     else return norm_residual_input_scale_bwd_kernel<T, VPT, G, S>;
 }
 
-// out[c] = sum over parts of part[p][c], in a fixed order: 8 interleaved
-// partial sums per column, combined in order.
-__global__ void __launch_bounds__(256) param_grad_reduce_kernel(const float* __restrict__ part, int nparts,
-                                                                int width, float* __restrict__ out) {
+// out[c] = sum over parts of part[p][c], in a fixed order: 32 thread groups
+// each sum the parts p = grp (mod 32) in order, then one warp adds the 32
+// results in a fixed tree (many short runs keep many loads in flight).
+constexpr int kReduceGroups = 32;
+__global__ void __launch_bounds__(32 * kReduceGroups) param_grad_reduce_kernel(const float* __restrict__ part,
+                                                                               int nparts, int width,
+                                                                               float* __restrict__ out) {
     pdl_begin();
-    __shared__ float sm[8][33];
+    __shared__ float sm[kReduceGroups][33];
     const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
     const int c = blockIdx.x * 32 + lane;
     float acc = 0.0f;
     if (c < width)
-        for (int p = grp; p < nparts; p += 8) acc += part[(int64_t)p * width + c];
+        for (int p = grp; p < nparts; p += kReduceGroups) acc += part[(int64_t)p * width + c];
     sm[grp][lane] = acc;
     __syncthreads();
-    if (grp == 0 && c < width) {
-        float t = sm[0][lane];
+    if (grp == 0) {
+        float v[kReduceGroups];
 #pragma unroll
-        for (int q = 1; q < 8; ++q) t += sm[q][lane];
-        out[c] = t;
+        for (int q = 0; q < kReduceGroups; ++q) v[q] = sm[q][lane];
+#pragma unroll
+        for (int n = kReduceGroups / 2; n > 0; n >>= 1)
+#pragma unroll
+            for (int q = 0; q < n; ++q) v[q] += v[q + n];
+        if (c < width) out[c] = v[0];
     }
 }
 
@@ -365,12 +398,12 @@ cudaError_t launch_bwd_s(RowBwdArgs a, int nvec, float* dgain, float* dtheta, cu
     if (e != cudaSuccess) return e;
     const unsigned rgrid = (unsigned)((a.width + 31) / 32);
     if (a.part_gain) {
-        e = launch_pdl(param_grad_reduce_kernel, rgrid, 256u, 0, s, (const float*)a.part_gain, (int)grid, (int)a.width, dgain);
+        e = launch_pdl(param_grad_reduce_kernel, rgrid, 32u * kReduceGroups, 0, s, (const float*)a.part_gain, (int)grid, (int)a.width, dgain);
         if (e != cudaSuccess) return e;
     }
     if constexpr (b_is_res(OP)) {
         if (a.part_theta)
-            e = launch_pdl(param_grad_reduce_kernel, rgrid, 256u, 0, s, (const float*)a.part_theta, (int)grid, (int)a.width, dtheta);
+            e = launch_pdl(param_grad_reduce_kernel, rgrid, 32u * kReduceGroups, 0, s, (const float*)a.part_theta, (int)grid, (int)a.width, dtheta);
     }
     return e;
 }
