@@ -57,6 +57,8 @@ def _load():
             lib.muse_oracle_positions.argtypes = [c_int, i64, i64, P, i32, i64, P]
             lib.muse_oracle_rms_norm.argtypes = [c_int, P, i64, i64, P, f32, f32, P, P, P, P]
             lib.muse_oracle_input_scale_norm.argtypes = lib.muse_oracle_rms_norm.argtypes
+            lib.muse_oracle_rms_norm_to.argtypes = [c_int, c_int, P, i64, i64, P, f32, f32, P, P, P, P]
+            lib.muse_oracle_rms_norm_to.restype = c_int
             lib.muse_oracle_qk_norm_rope.argtypes = [
                 c_int, P, P, i64, i32, i32, i32, P, f32, f32, c_int, c_int, f32,
                 P, P, P, P, P, P, P, P]
@@ -155,6 +157,20 @@ def rms_norm(x, gain=None, gain_offset=0.0, eps=1e-6):
     rows = x.size // hidden
     _check(_load().muse_oracle_rms_norm(_dt(x), _ptr(x), rows, hidden, _ptr(gain), gain_offset,
                                         eps, _ptr(out), _ptr(lo), _ptr(hi), _ptr(mag)), "rms_norm")
+    return out, lo, hi, mag
+
+
+def rms_norm_to(x, out_dtype, gain=None, gain_offset=0.0, eps=1e-6):
+    """Core 1 with the output in out_dtype (BF16 or F32) whatever x's dtype."""
+    x = _c(x)
+    gain = _c(gain)
+    out = np.empty(x.shape, dtype=np.uint16 if out_dtype == BF16 else np.float32)
+    lo, hi, mag = _checks(x.shape)
+    hidden = x.shape[-1]
+    rows = x.size // hidden
+    _check(_load().muse_oracle_rms_norm_to(_dt(x), out_dtype, _ptr(x), rows, hidden, _ptr(gain),
+                                           gain_offset, eps, _ptr(out), _ptr(lo), _ptr(hi),
+                                           _ptr(mag)), "rms_norm_to")
     return out, lo, hi, mag
 
 

@@ -158,19 +158,30 @@ static int valid_dtype(int dt) { return dt == DT_BF16 || dt == DT_F32; }
 int muse_oracle_rms_norm(int dtype, const void* x, int64_t rows, int64_t hidden,
                          const float* gain, float gain_offset, float eps,
                          void* out, double* lo, double* hi, double* mag) {
-    if (!valid_dtype(dtype) || rows < 0 || hidden <= 0 || (rows && (!x || !out))) return -1;
+    return muse_oracle_rms_norm_to(dtype, dtype, x, rows, hidden, gain, gain_offset, eps, out, lo,
+                                   hi, mag);
+}
+
+/* Core 1 with the output cast to out_dtype (the pre-norm of the FP32 stream
+ * feeding a projection may be asked for in the activation dtype). */
+int muse_oracle_rms_norm_to(int in_dtype, int out_dtype, const void* x, int64_t rows,
+                            int64_t hidden, const float* gain, float gain_offset, float eps,
+                            void* out, double* lo, double* hi, double* mag) {
+    if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype) || rows < 0 || hidden <= 0 ||
+        (rows && (!x || !out)))
+        return -1;
     for (int64_t r = 0; r < rows; ++r) {
         const int64_t base = r * hidden;
         double ss = 0.0;
         for (int64_t j = 0; j < hidden; ++j) {
-            double xj = load_elem(dtype, x, base + j);
+            double xj = load_elem(in_dtype, x, base + j);
             ss += xj * xj;
         }
         const double inv = inv_rms(ss, hidden, eps);
         for (int64_t j = 0; j < hidden; ++j) {
-            double y = load_elem(dtype, x, base + j) * inv;
+            double y = load_elem(in_dtype, x, base + j) * inv;
             if (gain) y *= eff_gain(gain, gain_offset, j);
-            store_elem(dtype, out, base + j, y);
+            store_elem(out_dtype, out, base + j, y);
             put_check(lo, hi, mag, base + j, y, y, fabs(y));
         }
     }

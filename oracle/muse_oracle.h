@@ -78,6 +78,12 @@ int muse_oracle_rms_norm(int dtype, const void* x, int64_t rows, int64_t hidden,
                          const float* gain, float gain_offset, float eps,
                          void* out, double* lo, double* hi, double* mag);
 
+/* Core 1 with separate input and output dtypes (y = cast_out((x r(x)) w_eff));
+ * muse_oracle_rms_norm is the case in_dtype == out_dtype. */
+int muse_oracle_rms_norm_to(int in_dtype, int out_dtype, const void* x, int64_t rows,
+                            int64_t hidden, const float* gain, float gain_offset, float eps,
+                            void* out, double* lo, double* hi, double* mag);
+
 /* Core 2, _input_scale_norm_core: z = x * w_eff, y = cast(z * r(z)). */
 int muse_oracle_input_scale_norm(int dtype, const void* x, int64_t rows, int64_t hidden,
                                  const float* gain, float gain_offset, float eps,

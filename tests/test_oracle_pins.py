@@ -451,3 +451,20 @@ def test_qk_query_scale_applies_to_the_cast_query():
     _, lo1, _, _ = oracle.rms_norm(q.reshape(-1, 64), None, 0, 1e-6)
     once = oracle.round_bf16(lo1.reshape(q.shape) * qs)
     assert np.mean(once != want) > 0.01  # the two orders are distinguishable
+
+
+def test_rms_norm_to_output_cast():
+    # FP32 input, bf16 output: a constant row normalises to sign * w exactly
+    # (eps = 0), so the output is the bf16 rounding of the effective gain.
+    H = 64
+    rng = np.random.default_rng(12)
+    gain = rng.uniform(0.5, 1.5, H).astype(np.float32)
+    x = np.vstack([np.full(H, 3.25, np.float32), np.full(H, -0.125, np.float32)])
+    out, lo, hi, _ = oracle.rms_norm_to(x, oracle.BF16, gain, 0.0, 0.0)
+    assert out.dtype == np.uint16
+    assert np.array_equal(out[0], oracle.round_bf16(gain.astype(np.float64)))
+    assert np.array_equal(out[1], oracle.round_bf16(-gain.astype(np.float64)))
+    assert np.array_equal(lo, hi)
+    # same arithmetic as the FP32-output call; only the final cast differs
+    o32, lo32, _, _ = oracle.rms_norm_to(x, oracle.F32, gain, 0.0, 0.0)
+    assert np.array_equal(lo, lo32) and np.array_equal(o32, lo32.astype(np.float32))
