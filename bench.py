@@ -282,6 +282,52 @@ class BwdStep:
                 self.ws.data_ptr(), self.ws_bytes, stream)
 
 
+def fused_vs_unfused(st: "Step", peak: float, flush: torch.Tensor, warmup: int = 10, reps: int = 50):
+    """Core 5 fused with the next sublayer's pre-norm (FP32 y) against core 5
+    followed by core 1 on the new FP32 stream: median of `reps`, each call
+    pair timed with events around both launches, L2 read-flushed before each."""
+    wl, T, H = st.wl, st.T, st.wl.hidden
+    d, sc = st.dev["norm_residual"], st.host["norm_residual"].scalars
+    g2, off2 = inputs.gain(wl, 0, "gain_next", True)
+    g2 = g2.cuda()
+    h = torch.empty_like(d["stream"])
+    y = torch.empty_like(d["stream"])
+    res = (d["stream"], d["branch"], d["theta"], d["gain"], sc["gain_offset"], False, sc["norm_eps"])
+
+    def fused():
+        cores.norm_residual_rms_norm(*res, next_gain=g2, next_gain_offset=off2, next_eps=1e-6,
+                                     out=h, y=y)
+
+    def unfused():
+        cores.norm_residual(*res, out=h)
+        cores.rms_norm(h, g2, off2, 1e-6, out=y)
+
+    stream = torch.cuda.current_stream()
+    out = {}
+    for name, fn in (("fused", fused), ("unfused", unfused)):
+        torch.cuda.synchronize()
+        torch.cuda._sleep(20_000_000)
+        ev = []
+        for i in range(warmup + reps):
+            flush.amax()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            if i >= warmup:
+                ev.append((e0, e1))
+        torch.cuda.synchronize()
+        out[name + "_us"] = round(statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3, 3)
+    nb = 14 * H * T + 12 * H  # branch + stream in, stream + FP32 y out; gains and angles once
+    out["fused_gbs"] = round(nb / (out["fused_us"] * 1e-6) / 1e9, 1)
+    out["fused_frac"] = round(out["fused_gbs"] / peak, 4)
+    out["algo_bytes_fused"] = nb
+    out["algo_bytes_unfused"] = 18 * H * T + 16 * H
+    out["note"] = ("core 5 + the next sublayer's RMS pre-norm of the new FP32 stream (FP32 y) in one "
+                   "pass, against muse_norm_residual then muse_rms_norm on its output")
+    return out
+
+
 def per_core_isolated(st, peak: float, flush: torch.Tensor | None, warmup: int = 10,
                       reps: int = 50, nbytes=None):
     """Each core launched alone: `warmup` launches, then the median of `reps`
@@ -533,7 +579,9 @@ def run_ours(args, world, rank, local):
                 "per_core_isolated": bwd_iso,
                 "note": "gradients of the five cores (the Q/K call with the FP32 rotation); gain and "
                         "theta gradients reduced through the caller's workspace"}
-    del bst, flush
+    del bst
+    fused = fused_vs_unfused(st, peak, flush)
+    del flush
     torch.cuda.empty_cache()
 
     e2e = run_e2e(st, args, world) if args.e2e else None
@@ -558,6 +606,7 @@ def run_ours(args, world, rank, local):
             "per_core_isolated": isolated,
             "decode_t128_h4096_latency": decode,
             "backward": backward,
+            "fused_residual_prenorm": fused,
             "roofline": roofline,
             "copy_kernel_gbs": None if copy_gbs is None else round(copy_gbs, 1),
             "e2e": e2e,

@@ -187,6 +187,32 @@ def norm_residual(stream_in: torch.Tensor, branch: torch.Tensor, theta: torch.Te
     return h_out
 
 
+def norm_residual_rms_norm(stream_in: torch.Tensor, branch: torch.Tensor, theta: torch.Tensor,
+                           gain: torch.Tensor | None = None, gain_offset: float = 0.0,
+                           input_scale: bool = False, norm_eps: float = 1e-6,
+                           next_gain: torch.Tensor | None = None, next_gain_offset: float = 0.0,
+                           next_eps: float = 1e-6, y_dtype=torch.float32, out=None, y=None,
+                           stream=None):
+    """Core 5 fused with the next sublayer's RMS pre-norm of the new stream:
+    returns (stream_out, y), y = rms_norm(stream_out) in y_dtype."""
+    _cuda(stream_in, branch, theta, gain, next_gain, out, y)
+    if stream_in.dtype != torch.float32 or theta.dtype != torch.float32:
+        raise TypeError("stream and theta must be float32")
+    if branch.shape != stream_in.shape or not (stream_in.is_contiguous() and branch.is_contiguous()):
+        raise ValueError("stream and branch must be contiguous and of one shape")
+    h_out = _out_like(stream_in, out)
+    if y is None:
+        y = torch.empty(stream_in.shape, dtype=y_dtype, device=stream_in.device)
+    hidden = stream_in.shape[-1]
+    rows = stream_in.numel() // hidden
+    g, g2 = _gain(gain), _gain(next_gain)
+    _lib.muse_norm_residual_rms_norm(
+        stream_in.data_ptr(), branch.data_ptr(), h_out.data_ptr(), y.data_ptr(), _dtype(branch),
+        _dtype(y), rows, hidden, _ptr(g), gain_offset, theta.contiguous().data_ptr(), input_scale,
+        norm_eps, _ptr(g2), next_gain_offset, next_eps, _stream(stream))
+    return h_out, y
+
+
 def stream_copy(src: torch.Tensor, dst: torch.Tensor, stream=None) -> torch.Tensor:
     """16-byte vector copy of src into dst (same byte size) - the HBM reference kernel."""
     _cuda(src, dst)

@@ -687,6 +687,63 @@ muse_status muse_qk_norm_rope_backward(const void* q, const void* k, const void*
     return from_cuda(muse::launch_qk_bwd(dtype, use_rope, A, stream), name);
 }
 
+muse_status muse_norm_residual_rms_norm(const float* stream_in, const void* branch, float* stream_out,
+                                        void* y, muse_dtype branch_dtype, muse_dtype y_dtype,
+                                        int64_t rows, int64_t hidden, const float* gain,
+                                        float gain_offset, const float* theta, int input_scale,
+                                        float norm_eps, const float* next_gain,
+                                        float next_gain_offset, float next_eps,
+                                        cudaStream_t stream) {
+    const char* name = "muse_norm_residual_rms_norm";
+    if (!valid_dtype(branch_dtype) || !valid_dtype(y_dtype))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype", name);
+    if (rows < 0 || hidden <= 0)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: rows=%lld hidden=%lld", name, (long long)rows, (long long)hidden);
+    if (!finite(norm_eps) || norm_eps < 0.0f || !finite(gain_offset) || !finite(next_eps) || next_eps < 0.0f ||
+        !finite(next_gain_offset))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: eps values must be finite and >= 0, offsets finite", name);
+    if (rows == 0) return MUSE_OK;
+    if (!stream_in || !branch || !stream_out || !theta || !y)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null stream_in/branch/stream_out/theta/y", name);
+    const int64_t es = elem_size(branch_dtype), ys = elem_size(y_dtype);
+    if (!aligned(stream_in, 16) || !aligned(stream_out, 16) || !aligned(branch, 16) || !aligned(y, 16) ||
+        (hidden * es) % 16 || (hidden * ys) % 16)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: pointers and row widths must be 16-byte multiples", name);
+    if (!aligned(theta, 16) || (gain && !aligned(gain, 16)) || (next_gain && !aligned(next_gain, 16)))
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: theta / gains not 16-byte aligned", name);
+    if (hidden / vec_elems(branch_dtype) > 1024)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: rows of more than 1024 16-byte branch vectors", name);
+    if (y_dtype != MUSE_DTYPE_F32 && y_dtype != branch_dtype)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: y must be FP32 or in the branch dtype", name);
+    const Span sin_ = span(stream_in, rows, hidden, hidden, 4), sout = span(stream_out, rows, hidden, hidden, 4);
+    const Span sb = span(branch, rows, hidden, hidden, es), st = span(theta, 1, hidden, hidden, 4);
+    const Span sy = span(y, rows, hidden, hidden, ys);
+    const Span sg = span(gain, gain ? 1 : 0, hidden, hidden, 4), sg2 = span(next_gain, next_gain ? 1 : 0, hidden, hidden, 4);
+    bool bad = bad_alias(sout, sin_, true) || any_overlap(sout, {sb, st, sg, sg2, sy});
+    bad = bad || (!same_span(sy, sb) && overlap(sy, sb)) || any_overlap(sy, {sin_, st, sg, sg2});
+    if (bad) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: an output partially overlaps an input", name);
+    muse::RowArgs a{};
+    a.x = branch;
+    a.y = y;
+    a.stream_in = stream_in;
+    a.stream_out = stream_out;
+    a.gain = gain;
+    a.theta = theta;
+    a.rows = rows;
+    a.x_stride = hidden;
+    a.y_stride = hidden;
+    a.s_in_stride = a.s_out_stride = hidden;
+    a.width = (int32_t)hidden;
+    a.gain_offset = gain_offset;
+    a.eps = norm_eps;
+    a.gain2 = next_gain;
+    a.gain2_offset = next_gain_offset;
+    a.eps2 = next_eps;
+    a.y_f32 = y_dtype == MUSE_DTYPE_F32 ? 1 : 0;
+    const muse::RowOp op = input_scale ? muse::RowOp::kResidualISPre : muse::RowOp::kResidualPre;
+    return from_cuda(muse::launch_row(branch_dtype, op, a, stream), name);
+}
+
 muse_status muse_device_error(unsigned int* flags, int clear) {
     if (!flags) return fail(MUSE_ERR_INVALID_ARGUMENT, "muse_device_error: null flags");
     // bit 0: the row pipeline's word, bit 1: the Q/K ring's, bit 2: the row

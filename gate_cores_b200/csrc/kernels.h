@@ -13,6 +13,8 @@ enum class RowOp : int {
     kNormGate = 2,     // core 4, one norm per token row: y = cast(o r sigmoid(g))
     kResidual = 3,     // core 5, gain after the norm
     kResidualIS = 4,   // core 5, gain before the norm
+    kResidualPre = 5,    // core 5 (gain after) + the next sublayer's RMS pre-norm of the new stream
+    kResidualISPre = 6,  // core 5 (gain before) + the next sublayer's RMS pre-norm
 };
 
 // One row = one token's `width` elements.  Strides in elements.
@@ -31,6 +33,12 @@ struct RowArgs {
     int32_t rows_per_cta;   // set by the launcher (register-staged row kernels)
     float gain_offset;
     float eps;
+    // kResidualPre / kResidualISPre: y = cast((h' r(h')) (gain2 + gain2_offset))
+    // into `y` (row stride y_stride), FP32 when y_f32 else the branch dtype
+    const float* gain2;     // may be null
+    float gain2_offset;
+    float eps2;
+    int32_t y_f32;
 };
 
 // Many short rows (one attention head each), contiguous: core 4 per head.

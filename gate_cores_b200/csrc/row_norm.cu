@@ -318,6 +318,7 @@ cudaError_t launch_row_dt(RowOp op, const RowArgs& a, cudaStream_t s) {
         case RowOp::kNormGate: return launch_row_t<T, RowOp::kNormGate>(a, s);
         case RowOp::kResidual: return launch_row_t<T, RowOp::kResidual>(a, s);
         case RowOp::kResidualIS: return launch_row_t<T, RowOp::kResidualIS>(a, s);
+        default: break;  // the fused residual + pre-norm has no register-staged form
     }
     return cudaErrorInvalidValue;
 }

@@ -32,8 +32,13 @@ namespace {
 
 using namespace pipe;
 
-__host__ __device__ constexpr bool t_is_residual(RowOp op) { return op == RowOp::kResidual || op == RowOp::kResidualIS; }
-__host__ __device__ constexpr bool t_scales_first(RowOp op) { return op == RowOp::kInputScale || op == RowOp::kResidualIS; }
+__host__ __device__ constexpr bool t_is_residual(RowOp op) {
+    return op == RowOp::kResidual || op == RowOp::kResidualIS || op == RowOp::kResidualPre || op == RowOp::kResidualISPre;
+}
+__host__ __device__ constexpr bool t_scales_first(RowOp op) {
+    return op == RowOp::kInputScale || op == RowOp::kResidualIS || op == RowOp::kResidualISPre;
+}
+__host__ __device__ constexpr bool t_prenorm(RowOp op) { return op == RowOp::kResidualPre || op == RowOp::kResidualISPre; }
 
 template <typename T, RowOp OP>
 struct TmaShape {
@@ -180,6 +185,17 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
         : static_cast<char*>(a.y) + r0 * a.y_stride * (int64_t)sizeof(T);
     const int64_t out_step = step * (t_is_residual(OP) ? a.s_out_stride * (int64_t)sizeof(float)
                                                       : a.y_stride * (int64_t)sizeof(T));
+    // fused ops: the next sublayer's effective gain in shared memory, after the
+    // ring (written here, first read after the row's first consumer barrier)
+    float* w2s = reinterpret_cast<float*>(smem + (size_t)S * L.stage_bytes);
+    if constexpr (t_prenorm(OP)) {
+        if (a.gain2)
+            for (int j = tid; j < a.width; j += ncons) w2s[j] = __ldg(a.gain2 + j) + a.gain2_offset;  // FP32 sum
+    }
+    // pre-norm output rows (fused ops only)
+    const int64_t y_es = a.y_f32 ? 4 : (int64_t)sizeof(T);
+    char* y_row = t_prenorm(OP) ? static_cast<char*>(a.y) + r0 * a.y_stride * y_es : nullptr;
+    const int64_t y_step = step * a.y_stride * y_es;
 
     // After a timed-out wait a warp stops touching the ring and the outputs but
     // keeps joining the consumer barrier, so no other warp is left waiting.
@@ -250,6 +266,8 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
                 if (alive && valid[i]) st_vec(out_row + voff[i], from_pairs<T>(o));
             }
         } else {
+            f32x2 hs[t_prenorm(OP) ? VPT : 1][P];  // the new stream, for the pre-norm
+            f32x2 hss = f2_make(0.0f, 0.0f);
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
                 f32x2 h[P], o[P];
@@ -258,14 +276,43 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
 #pragma unroll
                 for (int q = 0; q < P; ++q) {
                     f32x2 t = f2_mul(x[i][q], r2);  // z r when the gain came first
-                    if constexpr (OP == RowOp::kResidual && HAS_GAIN) t = f2_mul(t, w[i][q]);
+                    if constexpr (!t_scales_first(OP) && HAS_GAIN) t = f2_mul(t, w[i][q]);
                     const f32x2 nb = round_pair<T>(t);  // cast back to the branch dtype
                     o[q] = f2_fma(cth[i][q], h[q], f2_mul(sth[i][q], nb));
+                    if constexpr (t_prenorm(OP)) {
+                        hs[i][q] = o[q];
+                        hss = f2_fma(o[q], o[q], hss);
+                    }
                 }
                 if (alive && valid[i]) {
 #pragma unroll
                     for (int q = 0; q < SV; ++q) st_vec(out_row + voff[i] * SV + 16u * q, from_pairs<float>(o + 2 * q));
                 }
+            }
+            if constexpr (t_prenorm(OP)) {
+                // next sublayer's pre-norm of the new FP32 stream: y = (h' r(h')) w2,
+                // cast once; w2 from shared memory (filled once per CTA)
+                const float rr = inv_rms_fast(consumer_sum(f2_sum(hss), red, bank, ncons), inv_width, a.eps2);
+                const f32x2 rr2 = f2_make(rr, rr);
+#pragma unroll
+                for (int i = 0; i < VPT; ++i) {
+                    f32x2 y[P];
+                    const int wi = valid[i] ? (int)(voff[i] >> 4) * V : 0;  // idle slots read column 0
+#pragma unroll
+                    for (int q = 0; q < P; ++q) {
+                        y[q] = f2_mul(hs[i][q], rr2);
+                        if (a.gain2) y[q] = f2_mul(y[q], *reinterpret_cast<const f32x2*>(w2s + wi + 2 * q));
+                    }
+                    if (alive && valid[i]) {
+                        if (a.y_f32) {
+#pragma unroll
+                            for (int q = 0; q < SV; ++q) st_vec(y_row + voff[i] * SV + 16u * q, from_pairs<float>(y + 2 * q));
+                        } else {
+                            st_vec(y_row + voff[i], from_pairs<T>(y));
+                        }
+                    }
+                }
+                y_row += y_step;
             }
         }
         out_row += out_step;
@@ -298,6 +345,16 @@ __global__ void __launch_bounds__(512 + 32) norm_residual_input_scale_kernel(con
     pdl_begin();
     row_tma_body<T, RowOp::kResidualIS, VPT, G, S>(a);
 }
+template <typename T, int VPT, bool G, int S>
+__global__ void __launch_bounds__(512 + 32) norm_residual_prenorm_kernel(const __grid_constant__ RowArgs a) {
+    pdl_begin();
+    row_tma_body<T, RowOp::kResidualPre, VPT, G, S>(a);
+}
+template <typename T, int VPT, bool G, int S>
+__global__ void __launch_bounds__(512 + 32) norm_residual_input_scale_prenorm_kernel(const __grid_constant__ RowArgs a) {
+    pdl_begin();
+    row_tma_body<T, RowOp::kResidualISPre, VPT, G, S>(a);
+}
 
 template <typename T, RowOp OP, int VPT, bool G, int S>
 constexpr auto row_tma_kernel() {
@@ -305,7 +362,9 @@ constexpr auto row_tma_kernel() {
     else if constexpr (OP == RowOp::kInputScale) return input_scale_norm_kernel<T, VPT, G, S>;
     else if constexpr (OP == RowOp::kNormGate) return output_norm_gate_row_kernel<T, VPT, G, S>;
     else if constexpr (OP == RowOp::kResidual) return norm_residual_kernel<T, VPT, G, S>;
-    else return norm_residual_input_scale_kernel<T, VPT, G, S>;
+    else if constexpr (OP == RowOp::kResidualIS) return norm_residual_input_scale_kernel<T, VPT, G, S>;
+    else if constexpr (OP == RowOp::kResidualPre) return norm_residual_prenorm_kernel<T, VPT, G, S>;
+    else return norm_residual_input_scale_prenorm_kernel<T, VPT, G, S>;
 }
 
 }  // namespace
@@ -317,7 +376,7 @@ cudaError_t launch_row_tma_s(const RowArgs& a0, int nvec, cudaStream_t s) {
     const int ncons = ((nvec + VPT - 1) / VPT + 31) / 32 * 32;
     const int threads = ncons + 32;
     const StageLayout L = stage_layout<T, OP>(a.width);
-    const size_t smem = (size_t)S * L.stage_bytes;
+    const size_t smem = (size_t)S * L.stage_bytes + (t_prenorm(OP) ? (size_t)a.width * 4 : 0);
     auto kern = row_tma_kernel<T, OP, VPT, G, S>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -348,7 +407,10 @@ cudaError_t launch_row_op(const RowArgs& a, cudaStream_t s) {
     const int nvec = a.width / Vec<T>::N;
     const StageLayout L = stage_layout<T, OP>(a.width);
     const int dt = std::is_same<T, float>::value ? 1 : 0;
-    if (2 * L.stage_bytes > kRingMaxBytes) return launch_row_regs(dt, OP, a, s);
+    if (2 * L.stage_bytes > kRingMaxBytes) {
+        if constexpr (t_prenorm(OP)) return cudaErrorInvalidValue;  // the API keeps fused rows in range
+        return launch_row_regs(dt, OP, a, s);
+    }
     const int stages = L.stage_bytes >= 16 * 1024 ? 2 : 3;
     const bool g = a.gain != nullptr;
     // slots per consumer thread: the fewest that fit a row into kConsumers
@@ -361,6 +423,7 @@ cudaError_t launch_row_op(const RowArgs& a, cudaStream_t s) {
         if (nvec <= 4 * kConsumers)
             return g ? launch_row_tma_v<T, OP, 4, true>(a, nvec, stages, s) : launch_row_tma_v<T, OP, 4, false>(a, nvec, stages, s);
     }
+    if constexpr (t_prenorm(OP)) return cudaErrorInvalidValue;
     return launch_row_regs(dt, OP, a, s);
 }
 
@@ -372,6 +435,8 @@ cudaError_t launch_row_t2(RowOp op, const RowArgs& a, cudaStream_t s) {
         case RowOp::kNormGate: return launch_row_op<T, RowOp::kNormGate>(a, s);
         case RowOp::kResidual: return launch_row_op<T, RowOp::kResidual>(a, s);
         case RowOp::kResidualIS: return launch_row_op<T, RowOp::kResidualIS>(a, s);
+        case RowOp::kResidualPre: return launch_row_op<T, RowOp::kResidualPre>(a, s);
+        case RowOp::kResidualISPre: return launch_row_op<T, RowOp::kResidualISPre>(a, s);
     }
     return cudaErrorInvalidValue;
 }

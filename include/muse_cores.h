@@ -160,6 +160,29 @@ muse_status muse_norm_residual(const float* stream_in, const void* branch, float
                                const float* gain, float gain_offset, const float* theta,
                                int input_scale, float norm_eps, cudaStream_t stream);
 
+/*
+ * Core 5 fused with the next sublayer's pre-norm.  The decoder layer updates
+ * the FP32 stream with core 5 and then normalises that stream for the next
+ * sublayer (MuseSparkDecoderLayer: add_attn, then pre_ffn_norm; add_ffn, then
+ * the next layer's input norm).  This call does both in one pass, so the new
+ * stream is not read back:
+ *   stream_out = core 5 (as muse_norm_residual);
+ *   y = cast_y((stream_out r(stream_out)) w2),  w2 = next_gain + next_gain_offset
+ *       (no multiply when next_gain is NULL), r with next_eps, FP32 arithmetic
+ *       on the FP32 values written to stream_out;
+ * y [rows, hidden] contiguous in y_dtype: FP32, or the branch (activation)
+ * dtype for a projection input; any other y_dtype is MUSE_ERR_UNSUPPORTED.  y may be the very memory of branch when the dtypes
+ * match; stream_out may be stream_in.  Rows up to 1024 16-byte branch vectors
+ * (8192 bf16 / 4096 f32 elements), else MUSE_ERR_UNSUPPORTED.
+ */
+muse_status muse_norm_residual_rms_norm(const float* stream_in, const void* branch, float* stream_out,
+                                        void* y, muse_dtype branch_dtype, muse_dtype y_dtype,
+                                        int64_t rows, int64_t hidden, const float* gain,
+                                        float gain_offset, const float* theta, int input_scale,
+                                        float norm_eps, const float* next_gain,
+                                        float next_gain_offset, float next_eps,
+                                        cudaStream_t stream);
+
 /* ------------------------------------------------------------------ backward
  *
  * The cores run under autograd: the layers page keeps them outside
