@@ -59,6 +59,9 @@ def _load():
             lib.muse_oracle_input_scale_norm.argtypes = lib.muse_oracle_rms_norm.argtypes
             lib.muse_oracle_rms_norm_to.argtypes = [c_int, c_int, P, i64, i64, P, f32, f32, P, P, P, P]
             lib.muse_oracle_rms_norm_to.restype = c_int
+            lib.muse_oracle_rms_norm_grouped.argtypes = [c_int, P, i64, i64, P, f32, P, i32, f32,
+                                                         P, P, P, P]
+            lib.muse_oracle_rms_norm_grouped.restype = c_int
             lib.muse_oracle_qk_norm_rope.argtypes = [
                 c_int, P, P, i64, i32, i32, i32, P, f32, f32, c_int, c_int, f32,
                 P, P, P, P, P, P, P, P]
@@ -171,6 +174,22 @@ def rms_norm_to(x, out_dtype, gain=None, gain_offset=0.0, eps=1e-6):
     _check(_load().muse_oracle_rms_norm_to(_dt(x), out_dtype, _ptr(x), rows, hidden, _ptr(gain),
                                            gain_offset, eps, _ptr(out), _ptr(lo), _ptr(hi),
                                            _ptr(mag)), "rms_norm_to")
+    return out, lo, hi, mag
+
+
+def rms_norm_grouped(x, gains, offsets, gain_offset=0.0, eps=1e-6):
+    """Per-expert core 1: rows offsets[g]..offsets[g+1]-1 use gains[g]."""
+    x = _c(x)
+    gains = np.ascontiguousarray(gains, dtype=np.float32)
+    offsets = np.ascontiguousarray(offsets, dtype=np.int32)
+    out = np.empty_like(x)
+    lo, hi, mag = _checks(x.shape)
+    hidden = x.shape[-1]
+    rows = x.size // hidden
+    _check(_load().muse_oracle_rms_norm_grouped(_dt(x), _ptr(x), rows, hidden, _ptr(gains),
+                                                gain_offset, _ptr(offsets), offsets.size - 1, eps,
+                                                _ptr(out), _ptr(lo), _ptr(hi), _ptr(mag)),
+           "rms_norm_grouped")
     return out, lo, hi, mag
 
 

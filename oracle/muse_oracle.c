@@ -188,6 +188,33 @@ int muse_oracle_rms_norm_to(int in_dtype, int out_dtype, const void* x, int64_t 
     return 0;
 }
 
+/* Per-expert form of core 1 (MuseSparkMoE.pre_expert_norm /
+ * post_expert_norm: per-expert norms over the tokens routed to each expert).
+ * Rows [offsets[g], offsets[g+1]) are normalised with the gain row g of
+ * gains [num_groups, hidden]; offsets has num_groups + 1 entries, starts at
+ * 0, does not decrease and ends at rows. */
+int muse_oracle_rms_norm_grouped(int dtype, const void* x, int64_t rows, int64_t hidden,
+                                 const float* gains, float gain_offset, const int32_t* offsets,
+                                 int32_t num_groups, float eps, void* out, double* lo, double* hi,
+                                 double* mag) {
+    if (!valid_dtype(dtype) || rows < 0 || hidden <= 0 || num_groups < 1 || !offsets || !gains)
+        return -1;
+    if (offsets[0] != 0 || offsets[num_groups] != rows) return -1;
+    const size_t es = dtype == DT_BF16 ? 2 : 4;
+    for (int32_t g = 0; g < num_groups; ++g) {
+        const int64_t r0 = offsets[g], r1 = offsets[g + 1];
+        if (r1 < r0) return -1;
+        if (r1 == r0) continue;
+        const int64_t e0 = r0 * hidden;
+        const int rc = muse_oracle_rms_norm(
+            dtype, (const char*)x + (size_t)e0 * es, r1 - r0, hidden, gains + (int64_t)g * hidden,
+            gain_offset, eps, (char*)out + (size_t)e0 * es, lo ? lo + e0 : NULL, hi ? hi + e0 : NULL,
+            mag ? mag + e0 : NULL);
+        if (rc != 0) return rc;
+    }
+    return 0;
+}
+
 /* ------------------------------------------------------------------ core 2 */
 
 /* _input_scale_norm_core: apply the effective gain first, then a

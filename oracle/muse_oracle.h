@@ -78,6 +78,13 @@ int muse_oracle_rms_norm(int dtype, const void* x, int64_t rows, int64_t hidden,
                          const float* gain, float gain_offset, float eps,
                          void* out, double* lo, double* hi, double* mag);
 
+/* Per-expert core 1 (MuseSparkMoE pre_expert_norm / post_expert_norm): rows
+ * [offsets[g], offsets[g+1]) use gain row g of gains [num_groups, hidden]. */
+int muse_oracle_rms_norm_grouped(int dtype, const void* x, int64_t rows, int64_t hidden,
+                                 const float* gains, float gain_offset, const int32_t* offsets,
+                                 int32_t num_groups, float eps, void* out, double* lo, double* hi,
+                                 double* mag);
+
 /* Core 1 with separate input and output dtypes (y = cast_out((x r(x)) w_eff));
  * muse_oracle_rms_norm is the case in_dtype == out_dtype. */
 int muse_oracle_rms_norm_to(int in_dtype, int out_dtype, const void* x, int64_t rows,

@@ -468,3 +468,25 @@ def test_rms_norm_to_output_cast():
     # same arithmetic as the FP32-output call; only the final cast differs
     o32, lo32, _, _ = oracle.rms_norm_to(x, oracle.F32, gain, 0.0, 0.0)
     assert np.array_equal(lo, lo32) and np.array_equal(o32, lo32.astype(np.float32))
+
+
+def test_rms_norm_grouped_pins():
+    # per-expert gains: a group whose gain is twice another's gives exactly
+    # twice the outputs (power-of-two scaling is exact through every rounding);
+    # an empty group shifts nothing; a single group is core 1
+    rng = np.random.default_rng(13)
+    H, rows = 32, 9
+    x = oracle.round_bf16(rng.standard_normal((rows, H)))
+    g = rng.uniform(0.5, 1.5, H).astype(np.float32)
+    gains = np.stack([g, 0.5 * g, 2 * g])     # distinct rows: a shifted group index shows
+    offs = np.array([0, 4, 4, 9], np.int32)   # groups of 4, 0 and 5 rows
+    out, lo, hi, _ = oracle.rms_norm_grouped(x, gains, offs, 0.0, 1e-6)
+    a = oracle.rms_norm(x[:4], g, 0.0, 1e-6)
+    b = oracle.rms_norm(x[4:], 2 * g, 0.0, 1e-6)
+    assert np.array_equal(out[:4], a[0]) and np.array_equal(out[4:], b[0])
+    b1 = oracle.rms_norm(x[4:], g, 0.0, 1e-6)
+    np.testing.assert_array_equal(lo[4:], 2 * b1[1])
+    one, *_ = oracle.rms_norm_grouped(x, g[None, :], np.array([0, rows], np.int32), 0.0, 1e-6)
+    assert np.array_equal(one, oracle.rms_norm(x, g, 0.0, 1e-6)[0])
+    with pytest.raises(ValueError):
+        oracle.rms_norm_grouped(x, gains, np.array([0, 3, 2, 9], np.int32))
