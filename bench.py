@@ -328,6 +328,37 @@ def fused_vs_unfused(st: "Step", peak: float, flush: torch.Tensor, warmup: int =
     return out
 
 
+def grouped_norm(st: "Step", peak: float, flush: torch.Tensor, experts: int = 64, warmup: int = 10,
+                 reps: int = 50):
+    """Per-expert core 1 (MoE pre/post expert norm) on the batch's activations
+    routed to `experts` groups of skewed sizes: median of `reps` launches,
+    L2 read-flushed before each, against core 1 with one gain."""
+    wl, T, H = st.wl, st.T, st.wl.hidden
+    x = st.dev["rms_norm"]["x"]
+    gains, off = inputs.expert_gains(wl, 0, experts, True)
+    gains = gains.cuda()
+    offs = inputs.expert_groups(wl, 0, experts, T).cuda()
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    torch.cuda._sleep(20_000_000)
+    ev = []
+    for i in range(warmup + reps):
+        flush.amax()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        cores.rms_norm_grouped(x, gains, offs, off, 1e-6, out=y)
+        e1.record(stream)
+        if i >= warmup:
+            ev.append((e0, e1))
+    torch.cuda.synchronize()
+    us = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+    nb = 4 * H * T + 4 * H * experts + 4 * (experts + 1)
+    return {"us": round(us, 3), "gbs": round(nb / (us * 1e-6) / 1e9, 1),
+            "frac": round(nb / (us * 1e-6) / 1e9 / peak, 4), "experts": experts, "algo_bytes": nb,
+            "note": "muse_rms_norm_grouped: rows grouped by expert, each group with its own FP32 gain row"}
+
+
 def per_core_isolated(st, peak: float, flush: torch.Tensor | None, warmup: int = 10,
                       reps: int = 50, nbytes=None):
     """Each core launched alone: `warmup` launches, then the median of `reps`
@@ -581,6 +612,7 @@ def run_ours(args, world, rank, local):
                         "theta gradients reduced through the caller's workspace"}
     del bst
     fused = fused_vs_unfused(st, peak, flush)
+    grouped = grouped_norm(st, peak, flush)
     del flush
     torch.cuda.empty_cache()
 
@@ -607,6 +639,7 @@ def run_ours(args, world, rank, local):
             "decode_t128_h4096_latency": decode,
             "backward": backward,
             "fused_residual_prenorm": fused,
+            "per_expert_norm": grouped,
             "roofline": roofline,
             "copy_kernel_gbs": None if copy_gbs is None else round(copy_gbs, 1),
             "e2e": e2e,

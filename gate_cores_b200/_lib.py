@@ -32,7 +32,7 @@ EXPORTS = (
     "muse_norm_backward_workspace_bytes", "muse_rms_norm_backward",
     "muse_input_scale_norm_backward", "muse_norm_residual_backward",
     "muse_output_norm_gate_backward", "muse_qk_norm_rope_backward",
-    "muse_rms_norm_backward_noalloc", "muse_norm_residual_rms_norm",
+    "muse_rms_norm_backward_noalloc", "muse_norm_residual_rms_norm", "muse_rms_norm_grouped",
 )
 
 
@@ -83,6 +83,7 @@ def load() -> ctypes.CDLL:
         lib.muse_input_scale_norm_backward.argtypes = rbwd
         lib.muse_norm_residual_backward.argtypes = [P, P, P, P, P, c_int, i64, i64, P, f32, P,
                                                     c_int, f32, P, P, P, sz, P]
+        lib.muse_rms_norm_grouped.argtypes = [P, P, c_int, i64, i64, i64, i64, P, f32, P, i32, f32, P]
         lib.muse_norm_residual_rms_norm.argtypes = [P, P, P, P, c_int, c_int, i64, i64, P, f32, P,
                                                     c_int, f32, P, f32, f32, P]
         lib.muse_rms_norm_backward_noalloc.argtypes = [P, P, P, c_int, i64, i64, i64, i64, i64, P,
@@ -220,3 +221,9 @@ def muse_norm_residual_rms_norm(stream_in, branch, stream_out, y, branch_dtype, 
     _call("muse_norm_residual_rms_norm", stream_in, branch, stream_out, y, branch_dtype, y_dtype, rows,
           hidden, gain, gain_offset, theta, int(input_scale), norm_eps, next_gain, next_gain_offset,
           next_eps, stream)
+
+
+def muse_rms_norm_grouped(x, y, dtype, rows, hidden, x_row_stride, y_row_stride, gains, gain_offset,
+                          group_offsets, num_groups, eps, stream) -> None:
+    _call("muse_rms_norm_grouped", x, y, dtype, rows, hidden, x_row_stride, y_row_stride, gains,
+          gain_offset, group_offsets, num_groups, eps, stream)

@@ -187,6 +187,27 @@ def norm_residual(stream_in: torch.Tensor, branch: torch.Tensor, theta: torch.Te
     return h_out
 
 
+def rms_norm_grouped(x: torch.Tensor, gains: torch.Tensor, group_offsets: torch.Tensor,
+                     gain_offset: float = 0.0, eps: float = 1e-6, out: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """Per-expert core 1: rows group_offsets[g]..group_offsets[g+1]-1 of x use
+    gains[g] (gains FP32 [E, H]; group_offsets int32 [E+1] on the device)."""
+    _cuda(x, gains, group_offsets, out)
+    if gains.dtype != torch.float32 or group_offsets.dtype != torch.int32:
+        raise TypeError("gains must be float32 and group_offsets int32")
+    y = _out_like(x, out)
+    rows, hidden, xs = _rows(x)
+    _, _, ys = _rows(y)
+    gains = gains.contiguous()
+    group_offsets = group_offsets.contiguous()
+    if gains.shape[-1] != hidden or gains.numel() != hidden * (group_offsets.numel() - 1):
+        raise ValueError("gains must be [num_groups, hidden] with num_groups + 1 offsets")
+    _lib.muse_rms_norm_grouped(x.data_ptr(), y.data_ptr(), _dtype(x), rows, hidden, xs, ys,
+                               gains.data_ptr(), gain_offset, group_offsets.data_ptr(),
+                               group_offsets.numel() - 1, eps, _stream(stream))
+    return y
+
+
 def norm_residual_rms_norm(stream_in: torch.Tensor, branch: torch.Tensor, theta: torch.Tensor,
                            gain: torch.Tensor | None = None, gain_offset: float = 0.0,
                            input_scale: bool = False, norm_eps: float = 1e-6,

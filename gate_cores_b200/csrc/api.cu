@@ -687,6 +687,49 @@ muse_status muse_qk_norm_rope_backward(const void* q, const void* k, const void*
     return from_cuda(muse::launch_qk_bwd(dtype, use_rope, A, stream), name);
 }
 
+muse_status muse_rms_norm_grouped(const void* x, void* y, muse_dtype dtype, int64_t rows, int64_t hidden,
+                                  int64_t x_row_stride, int64_t y_row_stride, const float* gains,
+                                  float gain_offset, const int32_t* group_offsets, int32_t num_groups,
+                                  float eps, cudaStream_t stream) {
+    const char* name = "muse_rms_norm_grouped";
+    if (!valid_dtype(dtype)) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, (int)dtype);
+    if (rows < 0 || hidden <= 0 || num_groups < 1)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: rows=%lld hidden=%lld num_groups=%d", name, (long long)rows,
+                    (long long)hidden, num_groups);
+    if (!finite(eps) || eps < 0.0f || !finite(gain_offset))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: eps must be finite and >= 0, gain_offset finite", name);
+    if (x_row_stride < hidden || y_row_stride < hidden)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: row strides must be >= hidden", name);
+    if (rows == 0) return MUSE_OK;
+    if (!x || !y || !gains || !group_offsets)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null x, y, gains or group_offsets", name);
+    const int64_t es = elem_size(dtype);
+    if (!aligned(x, 16) || !aligned(y, 16) || !aligned(gains, 16) || (hidden * es) % 16 ||
+        (x_row_stride * es) % 16 || (y_row_stride * es) % 16)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: pointers, row widths and strides must be 16-byte multiples", name);
+    if (!aligned(group_offsets, 4)) return fail(MUSE_ERR_UNSUPPORTED, "%s: group_offsets not 4-byte aligned", name);
+    if (hidden / vec_elems(dtype) > 1024)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: rows of more than 1024 16-byte vectors", name);
+    const Span sx = span(x, rows, hidden, x_row_stride, es), sy = span(y, rows, hidden, y_row_stride, es);
+    const Span sg = span(gains, num_groups, hidden, hidden, 4);
+    const Span so = span(group_offsets, 1, (int64_t)num_groups + 1, (int64_t)num_groups + 1, 4);
+    if (bad_alias(sy, sx, true) || any_overlap(sy, {sg, so}))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: output partially overlaps an input", name);
+    muse::RowArgs a{};
+    a.x = x;
+    a.y = y;
+    a.gain = gains;
+    a.rows = rows;
+    a.x_stride = x_row_stride;
+    a.y_stride = y_row_stride;
+    a.width = (int32_t)hidden;
+    a.gain_offset = gain_offset;
+    a.eps = eps;
+    a.group_offsets = group_offsets;
+    a.num_groups = num_groups;
+    return from_cuda(muse::launch_row(dtype, muse::RowOp::kRmsGrouped, a, stream), name);
+}
+
 muse_status muse_norm_residual_rms_norm(const float* stream_in, const void* branch, float* stream_out,
                                         void* y, muse_dtype branch_dtype, muse_dtype y_dtype,
                                         int64_t rows, int64_t hidden, const float* gain,

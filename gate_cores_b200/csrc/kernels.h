@@ -15,6 +15,7 @@ enum class RowOp : int {
     kResidualIS = 4,   // core 5, gain before the norm
     kResidualPre = 5,    // core 5 (gain after) + the next sublayer's RMS pre-norm of the new stream
     kResidualISPre = 6,  // core 5 (gain before) + the next sublayer's RMS pre-norm
+    kRmsGrouped = 7,     // core 1 with per-expert gains: rows of group g use gain row g
 };
 
 // One row = one token's `width` elements.  Strides in elements.
@@ -39,6 +40,9 @@ struct RowArgs {
     float gain2_offset;
     float eps2;
     int32_t y_f32;
+    // kRmsGrouped: gain is [num_groups, width]; rows [offsets[g], offsets[g+1]) use row g
+    const int32_t* group_offsets;
+    int32_t num_groups;
 };
 
 // Many short rows (one attention head each), contiguous: core 4 per head.

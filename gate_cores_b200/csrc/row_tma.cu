@@ -39,6 +39,9 @@ __host__ __device__ constexpr bool t_scales_first(RowOp op) {
     return op == RowOp::kInputScale || op == RowOp::kResidualIS || op == RowOp::kResidualISPre;
 }
 __host__ __device__ constexpr bool t_prenorm(RowOp op) { return op == RowOp::kResidualPre || op == RowOp::kResidualISPre; }
+// Ops whose stage carries an FP32 row besides the activation row: the stream
+// (core 5) or the row's expert gain (per-expert core 1).
+__host__ __device__ constexpr bool t_f32_row(RowOp op) { return t_is_residual(op) || op == RowOp::kRmsGrouped; }
 
 template <typename T, RowOp OP>
 struct TmaShape {
@@ -63,7 +66,7 @@ __host__ __device__ inline StageLayout stage_layout(int width) {
     L.g_off = off;
     if (OP == RowOp::kNormGate) off += align128(L.x_bytes);
     L.h_off = off;
-    if (t_is_residual(OP)) off += align128((uint32_t)width * 4u);
+    if (t_f32_row(OP)) off += align128((uint32_t)width * 4u);
     L.stage_bytes = off;
     return L;
 }
@@ -105,7 +108,7 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
         if (lane == 0) {
             uint32_t bytes = L.x_bytes;
             if (OP == RowOp::kNormGate) bytes += L.x_bytes;
-            if (t_is_residual(OP)) bytes += (uint32_t)a.width * 4u;
+            if (t_f32_row(OP)) bytes += (uint32_t)a.width * 4u;
             int issued = 0;
             bool ok = true;
             for (int k = 0; k < n && ok; ++k) {
@@ -122,6 +125,16 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
                              L.x_bytes, &full_bar[s]);
                 if constexpr (t_is_residual(OP))
                     bulk_g2s(st + L.h_off, a.stream_in + row * a.s_in_stride, (uint32_t)a.width * 4u, &full_bar[s]);
+                if constexpr (OP == RowOp::kRmsGrouped) {
+                    // the row's group: offsets[g] <= row < offsets[g+1]; every index
+                    // read stays in [0, num_groups - 1] whatever the table holds
+                    int lo = 0, hi = a.num_groups;
+                    while (hi - lo > 1) {
+                        const int mid = (lo + hi) >> 1;
+                        if ((int64_t)__ldg(a.group_offsets + mid) <= row) lo = mid; else hi = mid;
+                    }
+                    bulk_g2s(st + L.h_off, a.gain + (int64_t)lo * a.width, (uint32_t)a.width * 4u, &full_bar[s]);
+                }
                 ++issued;
             }
             // Before exiting, every copy this CTA issued must have landed: in
@@ -157,7 +170,7 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
             const int v = valid[i] ? tid + i * ncons : 0;
 #pragma unroll
             for (int k = 0; k < SV; ++k) {
-                if constexpr (HAS_GAIN) {
+                if constexpr (HAS_GAIN && OP != RowOp::kRmsGrouped) {
                     const float4 g4 = __ldg(reinterpret_cast<const float4*>(a.gain) + v * SV + k);
                     w[i][2 * k] = f2_add(f2_make(g4.x, g4.y), off2);  // FP32 sums
                     w[i][2 * k + 1] = f2_add(f2_make(g4.z, g4.w), off2);
@@ -207,14 +220,14 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
         if (alive) alive = mbar_wait(&full_bar[s], phase);
         alive = __all_sync(0xffffffffu, alive);
         const unsigned char* st = smem + s * L.stage_bytes;
-        uint4 xv[VPT], gv[OP == RowOp::kNormGate ? VPT : 1], hv[t_is_residual(OP) ? VPT * SV : 1];
+        uint4 xv[VPT], gv[OP == RowOp::kNormGate ? VPT : 1], hv[t_f32_row(OP) ? VPT * SV : 1];
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
             const bool rd = alive && valid[i];
             xv[i] = rd ? *reinterpret_cast<const uint4*>(st + L.x_off + voff[i]) : make_uint4(0, 0, 0, 0);
             if constexpr (OP == RowOp::kNormGate)
                 gv[i] = rd ? *reinterpret_cast<const uint4*>(st + L.g_off + voff[i]) : make_uint4(0, 0, 0, 0);
-            if constexpr (t_is_residual(OP)) {
+            if constexpr (t_f32_row(OP)) {
 #pragma unroll
                 for (int q = 0; q < SV; ++q)
                     hv[i * SV + q] = rd ? *reinterpret_cast<const uint4*>(st + L.h_off + voff[i] * SV + 16u * q)
@@ -244,14 +257,22 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
         const float r = inv_rms_fast(consumer_sum(part, red, bank, ncons), inv_width, a.eps);
         const f32x2 r2 = f2_make(r, r);
 
-        if constexpr (OP == RowOp::kRms || OP == RowOp::kInputScale || OP == RowOp::kNormGate) {
+        if constexpr (OP == RowOp::kRms || OP == RowOp::kInputScale || OP == RowOp::kNormGate ||
+                      OP == RowOp::kRmsGrouped) {
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
                 f32x2 o[P];
+                f32x2 wg[OP == RowOp::kRmsGrouped ? P : 1];  // the row's expert gain, from the stage
+                if constexpr (OP == RowOp::kRmsGrouped) {
+#pragma unroll
+                    for (int q = 0; q < SV; ++q) to_pairs<float>(hv[i * SV + q], wg + 2 * q);
+                }
 #pragma unroll
                 for (int q = 0; q < P; ++q) {
                     o[q] = f2_mul(x[i][q], r2);
                     if constexpr (OP == RowOp::kRms && HAS_GAIN) o[q] = f2_mul(o[q], w[i][q]);
+                    if constexpr (OP == RowOp::kRmsGrouped)
+                        o[q] = f2_mul(o[q], f2_add(wg[q], f2_make(a.gain_offset, a.gain_offset)));  // FP32 sum
                 }
                 if constexpr (OP == RowOp::kNormGate) {
                     float gf[V];
@@ -346,6 +367,11 @@ __global__ void __launch_bounds__(512 + 32) norm_residual_input_scale_kernel(con
     row_tma_body<T, RowOp::kResidualIS, VPT, G, S>(a);
 }
 template <typename T, int VPT, bool G, int S>
+__global__ void __launch_bounds__(512 + 32) rms_norm_grouped_kernel(const __grid_constant__ RowArgs a) {
+    pdl_begin();
+    row_tma_body<T, RowOp::kRmsGrouped, VPT, G, S>(a);
+}
+template <typename T, int VPT, bool G, int S>
 __global__ void __launch_bounds__(512 + 32) norm_residual_prenorm_kernel(const __grid_constant__ RowArgs a) {
     pdl_begin();
     row_tma_body<T, RowOp::kResidualPre, VPT, G, S>(a);
@@ -364,6 +390,7 @@ constexpr auto row_tma_kernel() {
     else if constexpr (OP == RowOp::kResidual) return norm_residual_kernel<T, VPT, G, S>;
     else if constexpr (OP == RowOp::kResidualIS) return norm_residual_input_scale_kernel<T, VPT, G, S>;
     else if constexpr (OP == RowOp::kResidualPre) return norm_residual_prenorm_kernel<T, VPT, G, S>;
+    else if constexpr (OP == RowOp::kRmsGrouped) return rms_norm_grouped_kernel<T, VPT, G, S>;
     else return norm_residual_input_scale_prenorm_kernel<T, VPT, G, S>;
 }
 
@@ -408,7 +435,7 @@ cudaError_t launch_row_op(const RowArgs& a, cudaStream_t s) {
     const StageLayout L = stage_layout<T, OP>(a.width);
     const int dt = std::is_same<T, float>::value ? 1 : 0;
     if (2 * L.stage_bytes > kRingMaxBytes) {
-        if constexpr (t_prenorm(OP)) return cudaErrorInvalidValue;  // the API keeps fused rows in range
+        if constexpr (t_prenorm(OP) || OP == RowOp::kRmsGrouped) return cudaErrorInvalidValue;  // the API keeps these rows in range
         return launch_row_regs(dt, OP, a, s);
     }
     const int stages = L.stage_bytes >= 16 * 1024 ? 2 : 3;
@@ -423,7 +450,7 @@ cudaError_t launch_row_op(const RowArgs& a, cudaStream_t s) {
         if (nvec <= 4 * kConsumers)
             return g ? launch_row_tma_v<T, OP, 4, true>(a, nvec, stages, s) : launch_row_tma_v<T, OP, 4, false>(a, nvec, stages, s);
     }
-    if constexpr (t_prenorm(OP)) return cudaErrorInvalidValue;
+    if constexpr (t_prenorm(OP) || OP == RowOp::kRmsGrouped) return cudaErrorInvalidValue;
     return launch_row_regs(dt, OP, a, s);
 }
 
@@ -437,6 +464,7 @@ cudaError_t launch_row_t2(RowOp op, const RowArgs& a, cudaStream_t s) {
         case RowOp::kResidualIS: return launch_row_op<T, RowOp::kResidualIS>(a, s);
         case RowOp::kResidualPre: return launch_row_op<T, RowOp::kResidualPre>(a, s);
         case RowOp::kResidualISPre: return launch_row_op<T, RowOp::kResidualISPre>(a, s);
+        case RowOp::kRmsGrouped: return launch_row_op<T, RowOp::kRmsGrouped>(a, s);
     }
     return cudaErrorInvalidValue;
 }

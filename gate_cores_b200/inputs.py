@@ -139,6 +139,32 @@ def theta(wl: Workload, seed: int, tag: str = "theta") -> torch.Tensor:
     return u * float(math.pi / 2)
 
 
+def expert_groups(wl: Workload, seed: int, num_groups: int, tokens: int | None = None) -> torch.Tensor:
+    """Routed-token group boundaries for per-expert norms: int32 [num_groups + 1],
+    0 .. tokens, group sizes drawn from a seeded Dirichlet-like split (some
+    groups empty)."""
+    T = num_tokens(wl, seed) if tokens is None else tokens
+    g = _gen(seed, wl.name, "expert_groups", num_groups)
+    w = torch.rand(num_groups, generator=g, dtype=torch.float64) ** 3  # skewed loads
+    w[torch.randperm(num_groups, generator=g)[: max(1, num_groups // 8)]] = 0.0  # idle experts
+    if float(w.sum()) == 0.0:
+        w[0] = 1.0
+    cuts = torch.floor(torch.cumsum(w, 0) / w.sum() * T).to(torch.int64)
+    cuts[-1] = T
+    off = torch.zeros(num_groups + 1, dtype=torch.int64)
+    off[1:] = cuts
+    return off.to(torch.int32)
+
+
+def expert_gains(wl: Workload, seed: int, num_groups: int, zero_centered: bool) -> tuple[torch.Tensor, float]:
+    """(gains [num_groups, H] f32, offset), each row drawn like gain()."""
+    rows, off = [], 0.0
+    for e in range(num_groups):
+        gr, off = gain(wl, seed, f"gain_expert_{e}", zero_centered)
+        rows.append(gr)
+    return torch.stack(rows), off
+
+
 def upstream_grad(wl: Workload, seed: int, tag: str, shape, dtype=torch.bfloat16) -> torch.Tensor:
     """Incoming gradient dL/d(output) for the backward calls: N(0, 1) drawn in
     FP32 and rounded to dtype (no outlier channels)."""

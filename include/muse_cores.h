@@ -161,6 +161,23 @@ muse_status muse_norm_residual(const float* stream_in, const void* branch, float
                                int input_scale, float norm_eps, cudaStream_t stream);
 
 /*
+ * Per-expert form of core 1 (MuseSparkMoE pre_expert_norm / post_expert_norm:
+ * per-expert norms over the tokens routed to each expert).  The rows arrive
+ * grouped by expert, as a grouped-GEMM dispatch lays them out: rows
+ * [group_offsets[g], group_offsets[g+1]) are normalised like
+ * muse_rms_norm with the gain row g of gains [num_groups, hidden] (FP32,
+ * contiguous) plus gain_offset.  group_offsets is a DEVICE int32 array of
+ * num_groups + 1 entries starting at 0, non-decreasing, ending at rows; the
+ * library does not read it on the host (a row outside the table uses the
+ * nearest group, no access leaves the table).  Rows up to 1024 16-byte
+ * vectors, else MUSE_ERR_UNSUPPORTED.
+ */
+muse_status muse_rms_norm_grouped(const void* x, void* y, muse_dtype dtype, int64_t rows, int64_t hidden,
+                                  int64_t x_row_stride, int64_t y_row_stride, const float* gains,
+                                  float gain_offset, const int32_t* group_offsets, int32_t num_groups,
+                                  float eps, cudaStream_t stream);
+
+/*
  * Core 5 fused with the next sublayer's pre-norm.  The decoder layer updates
  * the FP32 stream with core 5 and then normalises that stream for the next
  * sublayer (MuseSparkDecoderLayer: add_attn, then pre_ffn_norm; add_ffn, then
