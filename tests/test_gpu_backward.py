@@ -1,4 +1,4 @@
-"""GPU parity of the backward calls (cores 1, 2, 5) against the oracle.
+"""GPU parity of the backward calls (all five cores) against the oracle.
 
 Forward inputs come from the same seeded generators as the forward parity
 tests, the incoming gradient from inputs.upstream_grad.  Every output is
@@ -120,4 +120,70 @@ def test_backward_workspace_checked(cuda_ok):
     with pytest.raises((_lib.MuseError, ValueError)):
         cores.rms_norm_backward(x, x, g, 0.0, 1e-6, workspace=small)
     assert _lib.muse_norm_backward_workspace_bytes(64, 256) >= 256 * 4
+    assert _lib.muse_device_error() == 0
+
+
+HEAD_WLS = [
+    inputs.WORKLOADS["tiny_t64_h256"],
+    Workload("ragged_t37_h264", hidden=264, hq=6, hkv=2, head_dim=80, rope_base=1.0e4, batch=1, seqlen=37),
+    Workload("ragged_b3s5_h40", hidden=40, hq=3, hkv=1, head_dim=16, rope_base=1.0e4, batch=3, seqlen=5),
+    Workload("ragged_thd_h512", hidden=512, hq=8, hkv=4, head_dim=64, rope_base=5.0e5, layout="thd",
+             positions="restart", num_seqs=7, seq_len_range=(0, 40)),
+    Workload("ragged_t1_h4096", hidden=4096, hq=32, hkv=8, head_dim=128, rope_base=5.0e5, batch=1, seqlen=1),
+    Workload("ragged_t300_h8192", hidden=8192, hq=64, hkv=8, head_dim=256, rope_base=5.0e5, batch=3,
+             seqlen=100, outlier_frac=0.01),
+    inputs.WORKLOADS["decode_t128_h4096"],
+    inputs.WORKLOADS["prefill_t8192_h4096"],
+]
+GATE_CASES = ["per_head", "per_token", "f32"]
+QK_CASES = ["upcast", "qscale", "no_rope", "explicit_pos", "f32"]
+
+
+@pytest.mark.parametrize("wl", HEAD_WLS, ids=lambda w: w.name)
+@pytest.mark.parametrize("variant", GATE_CASES)
+def test_output_norm_gate_backward(cuda_ok, wl, variant):
+    ci = harness.make(wl, "output_norm_gate", variant)
+    t, s = ci.tensors, ci.scalars
+    o, g = t["o"], t["g"]
+    dy = inputs.upstream_grad(wl, 0, "output_norm_gate", tuple(o.shape), o.dtype)
+    ng = o.shape[-2] * o.shape[-1] if s.get("per_token") else None
+    if ng is not None and ng * o.element_size() > 65536:
+        pytest.skip("norm group above the documented 64 KB")
+    d_o, dg = cores.output_norm_gate_backward(o.cuda(), g.cuda(), dy.cuda(), ng, s["eps"])
+    torch.cuda.synchronize()
+    r_o, r_g = oracle.output_norm_gate_bwd(_np(o), _np(g), _np(dy), ng, s["eps"])
+    what = f"{wl.name}/output_norm_gate/{variant}"
+    check(_np(d_o), r_o, what + "/do", backward=True)
+    check(_np(dg), r_g, what + "/dgate", backward=True)
+
+
+@pytest.mark.parametrize("wl", HEAD_WLS, ids=lambda w: w.name)
+@pytest.mark.parametrize("variant", QK_CASES)
+def test_qk_norm_rope_backward(cuda_ok, wl, variant):
+    ci = harness.make(wl, "qk_norm_rope", variant)
+    t, s = ci.tensors, ci.scalars
+    q, k = t["q"], t["k"]
+    if q.dtype == torch.float32 and wl.head_dim * 4 > 512:
+        pytest.skip("f32 heads above 512 bytes are outside the documented limit")
+    gq = inputs.upstream_grad(wl, 0, "qk_q", tuple(q.shape), q.dtype)
+    gk = inputs.upstream_grad(wl, 0, "qk_k", tuple(k.shape), k.dtype)
+    qd, kd, gqd, gkd = q.cuda(), k.cuda(), gq.cuda(), gk.cuda()
+    if s["layout"] == "bshd":
+        B, S = s["batch"], s["seqlen"]
+        qd, kd, gqd, gkd = (x.view(B, S, *x.shape[1:]) for x in (qd, kd, gqd, gkd))
+    pos = t["positions"]
+    dq, dk = cores.qk_norm_rope_backward(
+        qd, kd, gqd, gkd, positions=None if pos is None else pos.cuda(),
+        cu_seqlens=t["cu_seqlens"].cuda() if s["layout"] == "thd" else None, eps=s["eps"],
+        query_scale=s.get("query_scale", 1.0), use_rope=s.get("use_rope", True), rope_base=s["rope_base"])
+    torch.cuda.synchronize()
+    rq, rk = oracle.qk_norm_rope_bwd(_np(q), _np(k), _np(gq), _np(gk), harness.all_positions(wl, ci),
+                                     s["eps"], s.get("query_scale", 1.0), s.get("use_rope", True),
+                                     s["rope_base"])
+    what = f"{wl.name}/qk_norm_rope/{variant}"
+    check(_np(dq.reshape(q.shape)), rq, what + "/dq", backward=True)
+    check(_np(dk.reshape(k.shape)), rk, what + "/dk", backward=True)
+
+
+def test_no_device_error_after_backward_runs(cuda_ok):
     assert _lib.muse_device_error() == 0
