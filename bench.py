@@ -282,11 +282,10 @@ class BwdStep:
                 self.ws.data_ptr(), self.ws_bytes, stream)
 
 
-def fused_vs_unfused(st: "Step", peak: float, flush: torch.Tensor, warmup: int = 10, reps: int = 50):
-    """Core 5 fused with the next sublayer's pre-norm (FP32 y) against core 5
-    followed by core 1 on the new FP32 stream: median of `reps`, each call
-    pair timed with events around both launches, L2 read-flushed before each."""
-    wl, T, H = st.wl, st.T, st.wl.hidden
+def fused_calls(st: "Step"):
+    """(fused, unfused): core 5 with the next sublayer's pre-norm in one call,
+    and core 5 then core 1 on its output, on the batch's core 5 inputs."""
+    wl = st.wl
     d, sc = st.dev["norm_residual"], st.host["norm_residual"].scalars
     g2, off2 = inputs.gain(wl, 0, "gain_next", True)
     g2 = g2.cuda()
@@ -302,6 +301,15 @@ def fused_vs_unfused(st: "Step", peak: float, flush: torch.Tensor, warmup: int =
         cores.norm_residual(*res, out=h)
         cores.rms_norm(h, g2, off2, 1e-6, out=y)
 
+    return fused, unfused
+
+
+def fused_vs_unfused(st: "Step", peak: float, flush: torch.Tensor, warmup: int = 10, reps: int = 50):
+    """Core 5 fused with the next sublayer's pre-norm (FP32 y) against core 5
+    followed by core 1 on the new FP32 stream: median of `reps`, each call
+    pair timed with events around both launches, L2 read-flushed before each."""
+    T, H = st.T, st.wl.hidden
+    fused, unfused = fused_calls(st)
     stream = torch.cuda.current_stream()
     out = {}
     for name, fn in (("fused", fused), ("unfused", unfused)):
@@ -328,17 +336,29 @@ def fused_vs_unfused(st: "Step", peak: float, flush: torch.Tensor, warmup: int =
     return out
 
 
-def grouped_norm(st: "Step", peak: float, flush: torch.Tensor, experts: int = 64, warmup: int = 10,
-                 reps: int = 50):
-    """Per-expert core 1 (MoE pre/post expert norm) on the batch's activations
-    routed to `experts` groups of skewed sizes: median of `reps` launches,
-    L2 read-flushed before each, against core 1 with one gain."""
-    wl, T, H = st.wl, st.T, st.wl.hidden
+def grouped_call(st: "Step", experts: int = 64):
+    """Per-expert core 1 on the batch's core 1 activations routed to `experts`
+    groups of skewed sizes."""
+    wl, T = st.wl, st.T
     x = st.dev["rms_norm"]["x"]
     gains, off = inputs.expert_gains(wl, 0, experts, True)
     gains = gains.cuda()
     offs = inputs.expert_groups(wl, 0, experts, T).cuda()
     y = torch.empty_like(x)
+
+    def call():
+        cores.rms_norm_grouped(x, gains, offs, off, 1e-6, out=y)
+
+    return call
+
+
+def grouped_norm(st: "Step", peak: float, flush: torch.Tensor, experts: int = 64, warmup: int = 10,
+                 reps: int = 50):
+    """Per-expert core 1 (MoE pre/post expert norm) on the batch's activations
+    routed to `experts` groups of skewed sizes: median of `reps` launches,
+    L2 read-flushed before each."""
+    T, H = st.T, st.wl.hidden
+    call = grouped_call(st, experts)
     stream = torch.cuda.current_stream()
     torch.cuda.synchronize()
     torch.cuda._sleep(20_000_000)
@@ -347,7 +367,7 @@ def grouped_norm(st: "Step", peak: float, flush: torch.Tensor, experts: int = 64
         flush.amax()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        cores.rms_norm_grouped(x, gains, offs, off, 1e-6, out=y)
+        call()
         e1.record(stream)
         if i >= warmup:
             ev.append((e0, e1))
@@ -739,19 +759,25 @@ def run_reference(args, world, rank):
 
 
 def profile_pass(args):
-    """Each forward core, then each backward core, launched twice in that
-    order on the workload's batch: a short, fixed launch sequence for an
-    ncu capture (skip the first ten matching launches to capture warm ones)."""
+    """Each forward core, each backward core, then core 5 fused with the next
+    pre-norm and the per-expert core 1, the sequence launched twice on the
+    workload's batch: a short, fixed launch sequence for an ncu capture (16
+    kernel launches per pass; skip the first pass to capture warm ones)."""
     wl = WORKLOADS[args.workload]
     st = Step(wl, seed=0)
     bst = BwdStep(st, seed=0)
+    fused, _ = fused_calls(st)
+    grouped = grouped_call(st)
     for _ in range(2):
         for c in CORE_ORDER:
             st.launch(c)
         for c in CORE_ORDER:
             bst.launch(c)
+        fused()
+        grouped()
     torch.cuda.synchronize()
-    print("profile pass: 2 x (5 forward + 5 backward calls) on " + wl.name, file=sys.stderr)
+    print("profile pass: 2 x (5 forward + 5 backward calls, fused core 5 + pre-norm, per-expert core 1) on "
+          + wl.name, file=sys.stderr)
 
 
 def main():

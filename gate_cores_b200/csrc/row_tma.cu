@@ -10,6 +10,13 @@
 // squares (named barrier among consumers only), and write the outputs.  Rows
 // in flight per SM are set by the stage count, not by registers.
 //
+// Per-expert core 1 (rows grouped by expert) deals each CTA a contiguous run
+// of rows instead, and stages expert gain rows through one or two shared slots
+// outside the ring: the producer loads a gain row once per change of expert
+// (after the consumers have released the slot), each stage carries the index
+// of the expert run its row belongs to, and the consumers copy a run's gain to
+// registers at its first row.
+//
 // Every mbarrier wait is bounded: after kSpinLimit polls the thread records a
 // timeout in a device-wide error word (read by muse_device_error), stops, and
 // the producer waits - again bounded - for its own copies still in flight
@@ -39,9 +46,20 @@ __host__ __device__ constexpr bool t_scales_first(RowOp op) {
     return op == RowOp::kInputScale || op == RowOp::kResidualIS || op == RowOp::kResidualISPre;
 }
 __host__ __device__ constexpr bool t_prenorm(RowOp op) { return op == RowOp::kResidualPre || op == RowOp::kResidualISPre; }
-// Ops whose stage carries an FP32 row besides the activation row: the stream
-// (core 5) or the row's expert gain (per-expert core 1).
-__host__ __device__ constexpr bool t_f32_row(RowOp op) { return t_is_residual(op) || op == RowOp::kRmsGrouped; }
+// Ops whose stage carries the FP32 stream row besides the activation row (core 5).
+__host__ __device__ constexpr bool t_f32_row(RowOp op) { return t_is_residual(op); }
+// Per-expert core 1: each CTA takes a contiguous run of rows, so consecutive
+// rows mostly share an expert, and stages expert gain rows through one or two
+// shared slots outside the ring, one load per change of expert; the consumers
+// keep the current expert's gain in registers, as core 1 keeps its gain.
+__host__ __device__ constexpr bool t_grouped(RowOp op) { return op == RowOp::kRmsGrouped; }
+constexpr int kGainSlots = 2;
+// Two slots (the next expert's gain can land before the consumers reach it)
+// while the CTA's shared memory stays within a quarter of an SM's; else one,
+// which keeps four CTAs per SM.
+__host__ __device__ inline int grouped_gain_slots(uint32_t ring_bytes, uint32_t gslot_bytes) {
+    return ring_bytes + 2u * gslot_bytes <= 48u * 1024u ? 2 : 1;
+}
 
 template <typename T, RowOp OP>
 struct TmaShape {
@@ -79,6 +97,13 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
     __shared__ float red[2][32];
     __shared__ __align__(8) uint64_t full_bar[S];
     __shared__ __align__(8) uint64_t empty_bar[S];
+    // per-expert core 1: with N slots, slot j holds expert runs j, j + N, ...
+    // of this CTA's rows; full completes when a run's gain row has landed,
+    // free when every consumer warp has copied it to registers; stage_run[s]
+    // is the run of the row in stage s (written before the stage's full arrive)
+    __shared__ __align__(8) uint64_t gain_full[t_grouped(OP) ? kGainSlots : 1];
+    __shared__ __align__(8) uint64_t gain_free[t_grouped(OP) ? kGainSlots : 1];
+    __shared__ int stage_run[t_grouped(OP) ? S : 1];
 
     const int ncons = blockDim.x - 32;  // consumer threads; the last warp produces
     const int tid = threadIdx.x;
@@ -89,15 +114,26 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
     // This CTA's rows: r0, r0 + step, ... - rows interleaved across the grid,
     // so at any time the CTAs stream one compact window of the tensors
     // (measured slightly ahead of contiguous chunks per CTA when the previous
-    // kernel left dirty lines in L2).
-    const int64_t step = gridDim.x;
-    const int64_t r0 = blockIdx.x;
-    const int n = (int)max((int64_t)0, (a.rows - r0 + step - 1) / step);
+    // kernel left dirty lines in L2); per-expert core 1 takes a contiguous run.
+    const int64_t step = t_grouped(OP) ? 1 : gridDim.x;
+    const int64_t r0 = t_grouped(OP) ? (int64_t)blockIdx.x * a.rows / gridDim.x : (int64_t)blockIdx.x;
+    const int n = t_grouped(OP) ? (int)(((int64_t)blockIdx.x + 1) * a.rows / gridDim.x - r0)
+                                : (int)max((int64_t)0, (a.rows - r0 + step - 1) / step);
+    // the expert gain slots, after the ring
+    const uint32_t gslot_bytes = align128((uint32_t)a.width * 4u);
+    unsigned char* gslots = smem + (size_t)S * L.stage_bytes;
+    const int nslots = grouped_gain_slots((uint32_t)S * L.stage_bytes, gslot_bytes);
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], (uint32_t)(ncons >> 5));
+        }
+        if constexpr (t_grouped(OP)) {
+            for (int j = 0; j < kGainSlots; ++j) {
+                mbar_init(&gain_full[j], 1);
+                mbar_init(&gain_free[j], (uint32_t)(ncons >> 5));
+            }
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -105,18 +141,70 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
 
     if (warp == (ncons >> 5)) {
         // ---------------- producer warp: lane 0 issues whole-row bulk copies
+        // per-expert core 1: the first row's group (the last g with
+        // offsets[g] <= row), found by the whole warp with 32 probes a round;
+        // every index read stays in [0, num_groups - 1] whatever the table holds
+        int g_first = 0;
+        if constexpr (t_grouped(OP)) {
+            if (n > 0) {
+                int lo = 0, hi = a.num_groups;
+                while (hi - lo > 1) {
+                    const int chunk = (hi - lo + 31) >> 5;
+                    const int probe = lo + lane * chunk;
+                    const bool le = probe < hi && (int64_t)__ldg(a.group_offsets + probe) <= r0;
+                    const unsigned m = __ballot_sync(0xffffffffu, le);
+                    const int last = m ? 31 - __clz(m) : 0;
+                    const int nlo = lo + last * chunk;
+                    hi = min(hi, nlo + chunk);
+                    lo = nlo;
+                }
+                g_first = lo;
+            }
+        }
         if (lane == 0) {
             uint32_t bytes = L.x_bytes;
             if (OP == RowOp::kNormGate) bytes += L.x_bytes;
             if (t_f32_row(OP)) bytes += (uint32_t)a.width * 4u;
             int issued = 0;
             bool ok = true;
+            int grp = -1, runs = 0;  // per-expert core 1: current group, runs started
             for (int k = 0; k < n && ok; ++k) {
                 const int s = k % S;
                 if (k >= S) ok = mbar_wait(&empty_bar[s], (uint32_t)((k / S - 1) & 1));
                 if (!ok) break;
                 unsigned char* st = smem + (size_t)s * L.stage_bytes;
                 const int64_t row = r0 + k * step;
+                if constexpr (t_grouped(OP)) {
+                    // the activation copy first; the stage's run index is written
+                    // before the producer's arrival, which completes the phase
+                    mbar_expect_tx(&full_bar[s], bytes);
+                    bulk_g2s(st + L.x_off, static_cast<const char*>(a.x) + row * a.x_stride * (int64_t)sizeof(T),
+                             L.x_bytes, &full_bar[s]);
+                    // the row's group: the first row's, then a forward walk
+                    int g = g_first;
+                    if (grp >= 0) {
+                        g = grp;
+                        while (g + 1 < a.num_groups && (int64_t)__ldg(a.group_offsets + g + 1) <= row) ++g;
+                    }
+                    if (g != grp) {
+                        // a new run: its slot's previous run must be released first
+                        const int j = runs % nslots;
+                        if (runs >= nslots) ok = mbar_wait(&gain_free[j], (uint32_t)((runs / nslots - 1) & 1));
+                        if (ok) {
+                            mbar_arrive_expect_tx(&gain_full[j], (uint32_t)a.width * 4u);
+                            bulk_g2s(gslots + (size_t)j * gslot_bytes, a.gain + (int64_t)g * a.width,
+                                     (uint32_t)a.width * 4u, &gain_full[j]);
+                            grp = g;
+                            ++runs;
+                        }
+                    }
+                    stage_run[s] = runs - 1;
+                    // arrive even after a timed-out wait: the activation copy is
+                    // in flight and the exit waits below must see it land
+                    mbar_arrive(&full_bar[s]);
+                    ++issued;
+                    continue;
+                }
                 mbar_arrive_expect_tx(&full_bar[s], bytes);
                 bulk_g2s(st + L.x_off, static_cast<const char*>(a.x) + row * a.x_stride * (int64_t)sizeof(T),
                          L.x_bytes, &full_bar[s]);
@@ -125,16 +213,6 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
                              L.x_bytes, &full_bar[s]);
                 if constexpr (t_is_residual(OP))
                     bulk_g2s(st + L.h_off, a.stream_in + row * a.s_in_stride, (uint32_t)a.width * 4u, &full_bar[s]);
-                if constexpr (OP == RowOp::kRmsGrouped) {
-                    // the row's group: offsets[g] <= row < offsets[g+1]; every index
-                    // read stays in [0, num_groups - 1] whatever the table holds
-                    int lo = 0, hi = a.num_groups;
-                    while (hi - lo > 1) {
-                        const int mid = (lo + hi) >> 1;
-                        if ((int64_t)__ldg(a.group_offsets + mid) <= row) lo = mid; else hi = mid;
-                    }
-                    bulk_g2s(st + L.h_off, a.gain + (int64_t)lo * a.width, (uint32_t)a.width * 4u, &full_bar[s]);
-                }
                 ++issued;
             }
             // Before exiting, every copy this CTA issued must have landed: in
@@ -142,6 +220,10 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
             // waits return at once.
             for (int k = max(0, issued - S); k < issued; ++k)
                 if (!mbar_wait(&full_bar[k % S], (uint32_t)((k / S) & 1))) break;
+            if constexpr (t_grouped(OP)) {
+                for (int r = max(0, runs - nslots); r < runs; ++r)
+                    if (!mbar_wait(&gain_full[r % nslots], (uint32_t)((r / nslots) & 1))) break;
+            }
         }
         return;
     }
@@ -216,10 +298,39 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
     int bank = 0;
     int s = 0;
     uint32_t phase = 0;
+    int run = -1;  // per-expert core 1: the expert run whose gain slot this warp holds
     for (int k = 0; k < n; ++k) {
         if (alive) alive = mbar_wait(&full_bar[s], phase);
         alive = __all_sync(0xffffffffu, alive);
         const unsigned char* st = smem + s * L.stage_bytes;
+        if constexpr (t_grouped(OP)) {
+            const int r = alive ? stage_run[s] : run;
+            if (r != run && alive) {
+                // the first row of the next expert run: wait for its gain row,
+                // copy it (plus the offset, an FP32 sum) to registers, release the slot
+                run = r;
+                alive = mbar_wait(&gain_full[run % nslots], (uint32_t)((run / nslots) & 1));
+                alive = __all_sync(0xffffffffu, alive);
+                if (alive) {
+                    if constexpr (HAS_GAIN) {
+                        const unsigned char* gs = gslots + (size_t)(run % nslots) * gslot_bytes;
+                        const f32x2 off2 = f2_make(a.gain_offset, a.gain_offset);
+#pragma unroll
+                        for (int i = 0; i < VPT; ++i) {
+                            if (!valid[i]) continue;
+#pragma unroll
+                            for (int q = 0; q < SV; ++q) {
+                                const float4 g4 = *reinterpret_cast<const float4*>(gs + voff[i] * SV + 16u * q);
+                                w[i][2 * q] = f2_add(f2_make(g4.x, g4.y), off2);
+                                w[i][2 * q + 1] = f2_add(f2_make(g4.z, g4.w), off2);
+                            }
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&gain_free[run % nslots]);
+                }
+            }
+        }
         uint4 xv[VPT], gv[OP == RowOp::kNormGate ? VPT : 1], hv[t_f32_row(OP) ? VPT * SV : 1];
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
@@ -262,17 +373,11 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
                 f32x2 o[P];
-                f32x2 wg[OP == RowOp::kRmsGrouped ? P : 1];  // the row's expert gain, from the stage
-                if constexpr (OP == RowOp::kRmsGrouped) {
-#pragma unroll
-                    for (int q = 0; q < SV; ++q) to_pairs<float>(hv[i * SV + q], wg + 2 * q);
-                }
 #pragma unroll
                 for (int q = 0; q < P; ++q) {
                     o[q] = f2_mul(x[i][q], r2);
-                    if constexpr (OP == RowOp::kRms && HAS_GAIN) o[q] = f2_mul(o[q], w[i][q]);
-                    if constexpr (OP == RowOp::kRmsGrouped)
-                        o[q] = f2_mul(o[q], f2_add(wg[q], f2_make(a.gain_offset, a.gain_offset)));  // FP32 sum
+                    if constexpr ((OP == RowOp::kRms || OP == RowOp::kRmsGrouped) && HAS_GAIN)
+                        o[q] = f2_mul(o[q], w[i][q]);
                 }
                 if constexpr (OP == RowOp::kNormGate) {
                     float gf[V];
@@ -403,7 +508,9 @@ cudaError_t launch_row_tma_s(const RowArgs& a0, int nvec, cudaStream_t s) {
     const int ncons = ((nvec + VPT - 1) / VPT + 31) / 32 * 32;
     const int threads = ncons + 32;
     const StageLayout L = stage_layout<T, OP>(a.width);
-    const size_t smem = (size_t)S * L.stage_bytes + (t_prenorm(OP) ? (size_t)a.width * 4 : 0);
+    const uint32_t gslot = align128((uint32_t)a.width * 4u);
+    const size_t smem = (size_t)S * L.stage_bytes + (t_prenorm(OP) ? (size_t)a.width * 4 : 0) +
+                        (t_grouped(OP) ? (size_t)grouped_gain_slots((uint32_t)S * L.stage_bytes, gslot) * gslot : 0);
     auto kern = row_tma_kernel<T, OP, VPT, G, S>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

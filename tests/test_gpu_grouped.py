@@ -46,3 +46,28 @@ def test_rms_norm_grouped_one_group_is_core1(cuda_ok):
     y2 = cores.rms_norm(x, g.cuda(), off)
     torch.cuda.synchronize()
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+@pytest.mark.parametrize("T,H,E,single", [(8192, 1024, 8192, True), (8192, 4096, 2000, False),
+                                          (1000, 8192, 997, False)],
+                         ids=["one_row_per_expert", "t8192_h4096_e2000", "t1000_h8192_e997"])
+def test_rms_norm_grouped_many_runs_per_cta(cuda_ok, T, H, E, single):
+    # each CTA's contiguous rows cross many expert boundaries, so the two
+    # gain slots are refilled again and again within one CTA
+    g = torch.Generator().manual_seed(1234 + E)
+    x = (torch.randn(T, H, generator=g) * 2.0).to(torch.bfloat16)
+    gains = torch.rand(E, H, generator=g) * 0.4 - 0.2
+    if single:
+        offs = torch.arange(E + 1, dtype=torch.int32)
+    else:
+        w = torch.rand(E, generator=g, dtype=torch.float64) ** 3
+        w[torch.randperm(E, generator=g)[: E // 8]] = 0.0
+        cuts = torch.floor(torch.cumsum(w, 0) / w.sum() * T).to(torch.int64)
+        cuts[-1] = T
+        offs = torch.cat([torch.zeros(1, dtype=torch.int64), cuts]).to(torch.int32)
+    y = cores.rms_norm_grouped(x.cuda(), gains.cuda(), offs.cuda(), 1.0, 1e-6)
+    torch.cuda.synchronize()
+    ref = oracle.rms_norm_grouped(to_numpy(x), gains.numpy(), offs.numpy(), 1.0, 1e-6)
+    check(to_numpy(y.cpu()), ref, f"grouped/T{T}/H{H}/E{E}")
+    from gate_cores_b200 import _lib
+    assert _lib.muse_device_error() == 0
