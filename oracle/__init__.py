@@ -73,7 +73,7 @@ def _load():
                                                      P, P, P, P, P, P, P]
             lib.muse_oracle_input_scale_norm_bwd.argtypes = lib.muse_oracle_rms_norm_bwd.argtypes
             lib.muse_oracle_qk_norm_rope_bwd.argtypes = [
-                c_int, P, P, P, P, i64, i32, i32, i32, P, f32, f32, c_int, f32, c_int,
+                c_int, P, P, P, P, i64, i32, i32, i32, P, f32, f32, c_int, c_int, f32, c_int,
                 P, P, P, P, P, P, P, P]
             lib.muse_oracle_output_norm_gate_bwd.argtypes = [
                 c_int, P, P, P, i64, i32, i32, i32, f32, P, P, P, P, P, P, P, P]
@@ -292,8 +292,8 @@ def input_scale_norm_bwd(x, dy, gain=None, gain_offset=0.0, eps=1e-6):
 
 
 def qk_norm_rope_bwd(q, k, dq_out, dk_out, pos, eps=1e-6, query_scale=1.0, use_rope=True,
-                     rope_base=10000.0, round_grads=True):
-    """Core 3 backward (FP32 rotation): (dq, dk)."""
+                     rope_base=10000.0, round_grads=True, upcast_rope=True):
+    """Core 3 backward, FP32 (legacy) or, upcast_rope=False on bf16, v2 rotation: (dq, dk)."""
     q, k, dq_out, dk_out = _c(q), _c(k), _c(dq_out), _c(dk_out)
     pos = None if pos is None else np.ascontiguousarray(pos, dtype=np.int32)
     T, hq, d = q.shape
@@ -305,7 +305,7 @@ def qk_norm_rope_bwd(q, k, dq_out, dk_out, pos, eps=1e-6, query_scale=1.0, use_r
     kl, kh, km = _checks(k.shape)
     _check(_load().muse_oracle_qk_norm_rope_bwd(
         _dt(q), _ptr(q), _ptr(k), _ptr(dq_out), _ptr(dk_out), T, hq, hkv, d, _ptr(pos), eps,
-        query_scale, int(use_rope), rope_base, int(round_grads), _ptr(dq), _ptr(ql), _ptr(qh),
+        query_scale, int(use_rope), int(upcast_rope), rope_base, int(round_grads), _ptr(dq), _ptr(ql), _ptr(qh),
         _ptr(qm), _ptr(dk), _ptr(kl), _ptr(kh), _ptr(km)), "qk_norm_rope_bwd")
     return (dq, ql, qh, qm), (dk, kl, kh, km)
 

@@ -767,18 +767,62 @@ int muse_oracle_norm_residual_bwd(const float* stream, int branch_dtype, const v
     return 0;
 }
 
-/* Core 3 backward, FP32 (legacy) rotation.  Per head:
+/* Gradient of one pair's rotated-in values under the v2 rotation (bf16):
+ * the forward's y0 = cast(cast(a C) - cast(b S)), y1 = cast(cast(a S) +
+ * cast(b C)) with C = cast(c), S = cast(s).  Backward through those bf16
+ * operations: each product's gradient is the incoming gradient times the
+ * other factor, rounded to bf16, and the two gradients reaching a (or b) are
+ * added in bf16:
+ *   da = cast(cast(dy0 C) + cast(dy1 S)),   db = cast(cast(dy1 C) - cast(dy0 S));
+ * then, for query heads, cast(. * query_scale).  Products of two bf16 values
+ * are exact; the sums and the scaling take cast_candidates' values; C and S
+ * each take theirs (an FP32 sine or cosine near a bf16 midpoint). */
+static void qk_pair_bwd_v2(int dtype, double y0, double y1, float phi, int is_query,
+                           float query_scale, ival out[2]) {
+    double C[2], S[2];
+    const int nC = cast_candidates(dtype, cos((double)phi), C);
+    const int nS = cast_candidates(dtype, sin((double)phi), S);
+    for (int e = 0; e < 2; ++e) {
+        double mn = INFINITY, mx = -INFINITY, prim = 0.0;
+        for (int ic = 0; ic < nC; ++ic)
+            for (int is = 0; is < nS; ++is) {
+                const double v = e == 0 ? cast_to(dtype, y0 * C[ic]) + cast_to(dtype, y1 * S[is])
+                                        : cast_to(dtype, y1 * C[ic]) - cast_to(dtype, y0 * S[is]);
+                double g[2];
+                const int ng = cast_candidates(dtype, v, g);
+                for (int ig = 0; ig < ng; ++ig) {
+                    double h[2] = {g[ig], g[ig]};
+                    int nh = 1;
+                    if (is_query) nh = cast_candidates(dtype, g[ig] * (double)query_scale, h);
+                    for (int ih = 0; ih < nh; ++ih) minmax_upd(h[ih], &mn, &mx);
+                    if (ic == 0 && is == 0 && ig == 0) prim = h[0];
+                }
+            }
+        out[e].lo = mn;
+        out[e].hi = mx;
+        out[e].rn = prim;
+        out[e].m = fmax(fabs(mn), fabs(mx));
+    }
+}
+
+/* Core 3 backward.  Per head, FP32 (legacy) rotation:
  *   dm = R(phi)^T dy                     (FP32: da = c dy0 + s dy1, db = -s dy0 + c dy1)
  *   dn2 = cast(dm)                       (gradient of the rotated-in value, Q/K dtype)
  *   query heads: dn1 = cast(dn2 * query_scale); key heads: dn1 = dn2
+ * or, v2 rotation on bf16 tensors, dn1 from qk_pair_bwd_v2; then
  *   dx = r dn1 - r^3 x (sum_j dn1_j x_j) / d, cast to the Q/K dtype. */
 static void qk_head_bwd(int dtype, const void* x, const void* dy, int64_t base, int32_t d,
-                        const float* inv_freq, int32_t pos, int use_rope, float eps,
+                        const float* inv_freq, int32_t pos, int use_rope, int v2, float eps,
                         int is_query, float query_scale, int round_grads, double* xv,
                         double* one, ival* gr, ival* dd, double* dm, void* dx, double* lo,
                         double* hi, double* mag) {
     for (int32_t j = 0; j < d; ++j) xv[j] = load_elem(dtype, x, base + j);
     for (int32_t i = 0; i < d / 2; ++i) {
+        if (v2) {
+            qk_pair_bwd_v2(dtype, load_elem(dtype, dy, base + 2 * i), load_elem(dtype, dy, base + 2 * i + 1),
+                           (float)pos * inv_freq[i], is_query, query_scale, gr + 2 * i);
+            continue;
+        }
         double m0, m1;
         const double y0 = load_elem(dtype, dy, base + 2 * i);
         const double y1 = load_elem(dtype, dy, base + 2 * i + 1);
@@ -826,7 +870,7 @@ static void qk_head_bwd(int dtype, const void* x, const void* dy, int64_t base, 
 int muse_oracle_qk_norm_rope_bwd(int dtype, const void* q, const void* k, const void* dq_out,
                                  const void* dk_out, int64_t tokens, int32_t hq, int32_t hkv,
                                  int32_t head_dim, const int32_t* pos, float eps,
-                                 float query_scale, int use_rope, float rope_base,
+                                 float query_scale, int use_rope, int upcast_rope, float rope_base,
                                  int round_grads, void* dq, double* dq_lo, double* dq_hi,
                                  double* dq_mag, void* dk, double* dk_lo, double* dk_hi,
                                  double* dk_mag) {
@@ -845,15 +889,18 @@ int muse_oracle_qk_norm_rope_bwd(int dtype, const void* q, const void* k, const 
     double* dm = xv + 2 * (int64_t)head_dim;
     ival* dd = gr + head_dim;
     for (int32_t j = 0; j < head_dim; ++j) one[j] = 1.0;
+    /* v2 applies to bf16 tensors (FP32 tensors rotate in FP32 in both modes);
+     * the exact derivative (round_grads = 0) is the legacy one */
+    const int v2 = use_rope && !upcast_rope && dtype == DT_BF16 && round_grads;
     for (int64_t t = 0; t < tokens; ++t) {
         const int32_t p = use_rope ? pos[t] : 0;
         for (int32_t h = 0; h < hq; ++h)
             qk_head_bwd(dtype, q, dq_out, (t * hq + h) * (int64_t)head_dim, head_dim, inv_freq, p,
-                        use_rope, eps, 1, query_scale, round_grads, xv, one, gr, dd, dm, dq,
+                        use_rope, v2, eps, 1, query_scale, round_grads, xv, one, gr, dd, dm, dq,
                         dq_lo, dq_hi, dq_mag);
         for (int32_t h = 0; h < hkv; ++h)
             qk_head_bwd(dtype, k, dk_out, (t * hkv + h) * (int64_t)head_dim, head_dim, inv_freq,
-                        p, use_rope, eps, 0, 1.0f, round_grads, xv, one, gr, dd, dm, dk, dk_lo,
+                        p, use_rope, v2, eps, 0, 1.0f, round_grads, xv, one, gr, dd, dm, dk, dk_lo,
                         dk_hi, dk_mag);
     }
     free(inv_freq);

@@ -155,12 +155,15 @@ int muse_oracle_input_scale_norm_bwd(int dtype, const void* x, const void* dy, i
                                      float eps, void* dx, double* lo, double* hi, double* mag,
                                      double* dgain_lo, double* dgain_hi, double* dgain_mag);
 
-/* Core 3, FP32 (legacy) rotation: dm = R(phi)^T dy; dn = cast(dm), query
- * heads dn = cast(dn * query_scale); dx = r dn - r^3 x (sum_j dn_j x_j) / d. */
+/* Core 3.  FP32 (legacy) rotation: dm = R(phi)^T dy; dn = cast(dm), query
+ * heads dn = cast(dn * query_scale).  v2 rotation (upcast_rope = 0, bf16
+ * tensors; C = cast(cos), S = cast(sin)): dn = cast(cast(dy0 C) + cast(dy1 S)),
+ * cast(cast(dy1 C) - cast(dy0 S)) per pair, query heads cast(dn * query_scale).
+ * Then dx = r dn - r^3 x (sum_j dn_j x_j) / d. */
 int muse_oracle_qk_norm_rope_bwd(int dtype, const void* q, const void* k, const void* dq_out,
                                  const void* dk_out, int64_t tokens, int32_t hq, int32_t hkv,
                                  int32_t head_dim, const int32_t* pos, float eps,
-                                 float query_scale, int use_rope, float rope_base,
+                                 float query_scale, int use_rope, int upcast_rope, float rope_base,
                                  int round_grads, void* dq, double* dq_lo, double* dq_hi,
                                  double* dq_mag, void* dk, double* dk_lo, double* dk_hi,
                                  double* dk_mag);

@@ -256,3 +256,76 @@ def test_qk_norm_rope_bwd_rounded_gradient_composes():
     (dx, lo, _, _), _ = oracle.rms_norm_bwd(qb[:, 0, :], dn, None, 0.0, eps)
     assert np.array_equal(dq[:, 0, :], dx)
     assert np.all(qlo[:, 0, :] <= lo) and np.all(lo <= qhi[:, 0, :])
+
+
+def _bf16_ok(gpu_bits, lo, hi, mag):
+    from .parity import bf16_ok, BWD_EVAL_ULPS
+    return bf16_ok(gpu_bits, lo, hi, mag, BWD_EVAL_ULPS)
+
+
+@pytest.mark.parametrize("qs", [1.0, 0.3])
+def test_qk_norm_rope_bwd_v2_matches_bf16_autograd(qs):
+    # The v2 rotation on bf16 tensors, written with torch's own bf16 CPU
+    # operations (each product and sum rounded to bf16, cos/sin cast to bf16);
+    # torch.autograd then derives the backward through those bf16 operations
+    # (a product's gradient rounded to bf16, the two gradients of a tensor used
+    # twice added in bf16).  The oracle's v2 backward must agree within the
+    # backward rule.
+    rng = np.random.default_rng(21)
+    T, hq, hkv, D, eps, base = 6, 4, 2, 64, 1e-6, 10000.0
+    qb, kb = rnd_bf16((T, hq, D), rng, 3.0), rnd_bf16((T, hkv, D), rng, 3.0)
+    dqb, dkb = rnd_bf16((T, hq, D), rng), rnd_bf16((T, hkv, D), rng)
+    pos = np.array([0, 1, 17, 999, 4096, 31000], np.int32)
+    (dq, qlo, qhi, qmag), (dk, klo, khi, kmag) = oracle.qk_norm_rope_bwd(
+        qb, kb, dqb, dkb, pos, eps, qs, True, base, upcast_rope=False)
+    inv = torch.tensor(oracle.inv_freq(D, base).astype(np.float32))
+    phi = torch.tensor(pos).float()[:, None] * inv[None, :]          # FP32 angle
+    C = torch.cos(phi).to(torch.bfloat16)[:, None, :]
+    S = torch.sin(phi).to(torch.bfloat16)[:, None, :]
+
+    def to_t(bits):
+        return torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16)
+
+    def fwd(x, scale):
+        xf = x.float()
+        n = (xf * torch.rsqrt((xf * xf).mean(-1, keepdim=True) + eps)).to(torch.bfloat16)
+        if scale is not None:
+            n = n * scale
+        a, b = n[..., 0::2], n[..., 1::2]
+        return torch.stack([a * C - b * S, a * S + b * C], dim=-1).reshape(n.shape)
+
+    q = to_t(qb).requires_grad_(True)
+    k = to_t(kb).requires_grad_(True)
+    fwd(q, qs if qs != 1.0 else None).backward(to_t(dqb))
+    fwd(k, None).backward(to_t(dkb))
+    gq = q.grad.view(torch.int16).numpy().view(np.uint16)
+    gk = k.grad.view(torch.int16).numpy().view(np.uint16)
+    assert _bf16_ok(gq, qlo, qhi, qmag).all()
+    assert _bf16_ok(gk, klo, khi, kmag).all()
+
+
+def test_qk_norm_rope_bwd_v2_rounded_gradient_composes():
+    # v2: the key gradient is the plain norm backward of the pairs
+    # (bf16(bf16(dy0 C) + bf16(dy1 S)), bf16(bf16(dy1 C) - bf16(dy0 S))),
+    # C, S the bf16 cos / sin of the FP32 angle; it differs from the FP32
+    # rotation's gradient
+    rng = np.random.default_rng(22)
+    T, D, eps, base = 4, 32, 1e-6, 5e5
+    kb = rnd_bf16((T, 1, D), rng)
+    dkb = rnd_bf16((T, 1, D), rng)
+    qb, dqb = kb.copy(), dkb.copy()
+    pos = np.array([3, 77, 4000, 12345], np.int32)
+    _, (dk, klo, khi, _) = oracle.qk_norm_rope_bwd(qb, kb, dqb, dkb, pos, eps, 1.0, True, base,
+                                                   upcast_rope=False)
+    _, (dk_legacy, *_) = oracle.qk_norm_rope_bwd(qb, kb, dqb, dkb, pos, eps, 1.0, True, base)
+    inv = oracle.inv_freq(D, base).astype(np.float32)
+    phi = (pos.astype(np.float32)[:, None] * inv[None, :]).astype(np.float32).astype(np.float64)
+    C, S = bf16_vals(oracle.round_bf16(np.cos(phi))), bf16_vals(oracle.round_bf16(np.sin(phi)))
+    r = lambda v: bf16_vals(oracle.round_bf16(v))
+    dy = bf16_vals(dkb)[:, 0, :]
+    a, b = dy[:, 0::2], dy[:, 1::2]
+    dn = np.stack([r(r(a * C) + r(b * S)), r(r(b * C) - r(a * S))], -1).reshape(T, D)
+    (dx, lo, _, _), _ = oracle.rms_norm_bwd(kb[:, 0, :], oracle.round_bf16(dn), None, 0.0, eps)
+    assert np.array_equal(dk[:, 0, :], dx)
+    assert np.all(klo[:, 0, :] <= lo) and np.all(lo <= khi[:, 0, :])
+    assert not np.array_equal(dk, dk_legacy)
