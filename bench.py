@@ -250,6 +250,7 @@ class BwdStep:
                        for c in ("rms_norm", "input_scale_norm", "gain_res", "theta_res")}
         self.ws_bytes = _lib.muse_norm_backward_workspace_bytes(self.T, H)
         self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
+        self.qk_upcast = True  # the Q/K backward's rotation: FP32 (legacy) or v2
 
     def launch(self, core: str):
         L, wl, T, H = self.lib, self.wl, self.T, self.wl.hidden
@@ -268,7 +269,8 @@ class BwdStep:
                 d["q"].data_ptr(), d["k"].data_ptr(), self.dy["qk_q"].data_ptr(), self.dy["qk_k"].data_ptr(),
                 self.out["dq"].data_ptr(), self.out["dk"].data_ptr(), bf, L.MUSE_LAYOUT_BSHD, wl.batch,
                 wl.seqlen, None, 0, T, None if pos is None else pos.data_ptr(), wl.hq, wl.hkv,
-                wl.head_dim, qw, kw, qw, kw, qw, kw, sc["eps"], 1.0, True, sc["rope_base"], stream)
+                wl.head_dim, qw, kw, qw, kw, qw, kw, sc["eps"], 1.0, True, self.qk_upcast, sc["rope_base"],
+                stream)
         elif core == "output_norm_gate":
             L.muse_output_norm_gate_backward(
                 d["o"].data_ptr(), d["g"].data_ptr(), self.dy[core].data_ptr(), self.out["do"].data_ptr(),
@@ -380,7 +382,7 @@ def grouped_norm(st: "Step", peak: float, flush: torch.Tensor, experts: int = 64
 
 
 def per_core_isolated(st, peak: float, flush: torch.Tensor | None, warmup: int = 10,
-                      reps: int = 50, nbytes=None):
+                      reps: int = 50, nbytes=None, which=CORE_ORDER):
     """Each core launched alone: `warmup` launches, then the median of `reps`
     launches timed with CUDA events around each one on the launching stream.
     With `flush`, a read pass over that buffer (> L2, reading leaves no dirty
@@ -388,7 +390,7 @@ def per_core_isolated(st, peak: float, flush: torch.Tensor | None, warmup: int =
     without it, L2 stays warm (the decode latency figures)."""
     stream = torch.cuda.current_stream()
     out = {}
-    for c in CORE_ORDER:
+    for c in which:
         ev = []
         torch.cuda.synchronize()
         # hold the GPU for a few ms so that the host queues every launch ahead
@@ -607,6 +609,10 @@ def run_ours(args, world, rank, local):
     # with two events, as the forward step).
     bst = BwdStep(st, seed=rank)
     bwd_iso = per_core_isolated(bst, peak, flush, nbytes=algo_bytes_bwd)
+    bst.qk_upcast = False  # the v2 (bf16) rotation's backward, alone
+    bwd_iso["qk_norm_rope_v2"] = per_core_isolated(bst, peak, flush, nbytes=algo_bytes_bwd,
+                                                   which=("qk_norm_rope",))["qk_norm_rope"]
+    bst.qk_upcast = True
     for _ in range(3):
         for c in CORE_ORDER:
             bst.launch(c)

@@ -92,7 +92,7 @@ def load() -> ctypes.CDLL:
                                                        f32, P]
         lib.muse_qk_norm_rope_backward.argtypes = [P, P, P, P, P, P, c_int, c_int, i64, i64, P,
                                                    i32, i64, P, i32, i32, i32, i64, i64, i64, i64,
-                                                   i64, i64, f32, f32, c_int, f32, P]
+                                                   i64, i64, f32, f32, c_int, c_int, f32, P]
         for name in EXPORTS[3:]:
             getattr(lib, name).restype = c_int
         lib.muse_norm_backward_workspace_bytes.restype = sz
@@ -201,12 +201,12 @@ def muse_output_norm_gate_backward(o, gate, dy, d_o, dgate, dtype, tokens, heads
 def muse_qk_norm_rope_backward(q, k, dq_out, dk_out, dq, dk, dtype, layout, batch, seqlen,
                                cu_seqlens, num_seqs, total_tokens, positions, hq, hkv, head_dim,
                                q_tok_stride, k_tok_stride, dq_out_tok_stride, dk_out_tok_stride,
-                               dq_tok_stride, dk_tok_stride, eps, query_scale, use_rope, rope_base,
-                               stream) -> None:
+                               dq_tok_stride, dk_tok_stride, eps, query_scale, use_rope, upcast_rope,
+                               rope_base, stream) -> None:
     _call("muse_qk_norm_rope_backward", q, k, dq_out, dk_out, dq, dk, dtype, layout, batch, seqlen,
           cu_seqlens, num_seqs, total_tokens, positions, hq, hkv, head_dim, q_tok_stride,
           k_tok_stride, dq_out_tok_stride, dk_out_tok_stride, dq_tok_stride, dk_tok_stride, eps,
-          query_scale, int(use_rope), rope_base, stream)
+          query_scale, int(use_rope), int(upcast_rope), rope_base, stream)
 
 
 def muse_rms_norm_backward_noalloc(x, dy, dx, dtype, rows, hidden, x_row_stride, dy_row_stride,

@@ -338,9 +338,10 @@ def output_norm_gate_backward(o, gate, dy, norm_group=None, eps: float = 1e-6, s
 
 def qk_norm_rope_backward(q, k, dq_out, dk_out, positions=None, cu_seqlens=None, eps: float = 1e-6,
                           query_scale: float = 1.0, use_rope: bool = True,
-                          rope_base: float = 10000.0, stream=None):
-    """Backward of core 3 (FP32 rotation): returns (dq, dk) shaped like q, k.
-    Layout and positions as in qk_norm_rope."""
+                          rope_base: float = 10000.0, upcast_rope: bool = True, stream=None):
+    """Backward of core 3 (FP32 rotation, or the v2 bf16 rotation with
+    upcast_rope=False): returns (dq, dk) shaped like q, k.  Layout and
+    positions as in qk_norm_rope."""
     _cuda(q, k, dq_out, dk_out, positions, cu_seqlens)
     if q.dim() == 4:
         layout, batch, seqlen, T = _lib.MUSE_LAYOUT_BSHD, q.shape[0], q.shape[1], q.shape[0] * q.shape[1]
@@ -369,5 +370,5 @@ def qk_norm_rope_backward(q, k, dq_out, dk_out, positions=None, cu_seqlens=None,
         _dtype(q), layout, batch, seqlen, _ptr(cu_seqlens), num_seqs, T, _ptr(positions), hq, hkv, d,
         _tok_stride(q, hq, d), _tok_stride(k, hkv, d), _tok_stride(dq_out, hq, d),
         _tok_stride(dk_out, hkv, d), _tok_stride(dq, hq, d), _tok_stride(dk, hkv, d), eps,
-        query_scale, use_rope, rope_base, _stream(stream))
+        query_scale, use_rope, upcast_rope, rope_base, _stream(stream))
     return dq, dk

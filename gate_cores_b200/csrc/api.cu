@@ -598,7 +598,8 @@ muse_status muse_qk_norm_rope_backward(const void* q, const void* k, const void*
                                        int64_t k_tok_stride, int64_t dq_out_tok_stride,
                                        int64_t dk_out_tok_stride, int64_t dq_tok_stride,
                                        int64_t dk_tok_stride, float eps, float query_scale,
-                                       int use_rope, float rope_base, cudaStream_t stream) {
+                                       int use_rope, int upcast_rope, float rope_base,
+                                       cudaStream_t stream) {
     const char* name = "muse_qk_norm_rope_backward";
     if (!valid_dtype(dtype)) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, (int)dtype);
     if (layout != MUSE_LAYOUT_BSHD && layout != MUSE_LAYOUT_THD)
@@ -684,7 +685,7 @@ muse_status muse_qk_norm_rope_backward(const void* q, const void* k, const void*
     A.gk = dk_out;
     A.gq_stride = dq_out_tok_stride;
     A.gk_stride = dk_out_tok_stride;
-    return from_cuda(muse::launch_qk_bwd(dtype, use_rope, A, stream), name);
+    return from_cuda(muse::launch_qk_bwd(dtype, use_rope, upcast_rope, A, stream), name);
 }
 
 muse_status muse_rms_norm_grouped(const void* x, void* y, muse_dtype dtype, int64_t rows, int64_t hidden,

@@ -1,5 +1,5 @@
 // Backward of the per-head cores: core 4 (_output_norm_gate_core) and core 3
-// (_qk_norm_rope_core, FP32 rotation).  Derivatives of the forward maps,
+// (_qk_norm_rope_core, FP32 or v2 rotation).  Derivatives of the forward maps,
 // evaluated in FP32 from the saved forward inputs, with every dtype boundary
 // the forward materialises rounding the gradient that flows back through it:
 //
@@ -10,6 +10,9 @@
 //     dm = R(phi)^T dy  (da = c dy0 + s dy1, db = -s dy0 + c dy1, FP32);
 //     dn = cast(dm);  query heads: dn = cast(dn * query_scale);
 //     dx = r dn - r^3 x (sum_j dn_j x_j) / D
+//   v2 rotation (bf16; C, S the bf16 cos and sin): the forward's bf16
+//   products and sums give dn = (cast(cast(dy0 C) + cast(dy1 S)),
+//   cast(cast(dy1 C) - cast(dy0 S))) per pair before the query scaling.
 //
 // Layouts, lanes per head and the Q/K ring (each warp streams its batches of
 // head steps through its own shared-memory slots with cp.async.bulk, here two
@@ -205,7 +208,7 @@ __global__ void __launch_bounds__(512) output_norm_gate_group_bwd_kernel(const _
 // token's head steps); a shared cos/sin table per tile; each warp streams its
 // batches (BATCH head steps of the forward input and of the incoming
 // gradient) through a ring of R slots, as the forward kernel does.
-template <typename T, int L, bool ROPE, bool TAIL, int BATCH, int R>
+template <typename T, int L, bool ROPE, bool V2, bool TAIL, int BATCH, int R>
 __global__ void __launch_bounds__(256, 3) qk_norm_rope_bwd_kernel(const __grid_constant__ QkBwdArgs A) {
     pdl_begin();
     const QkArgs& a = A.f;
@@ -283,6 +286,10 @@ __global__ void __launch_bounds__(256, 3) qk_norm_rope_bwd_kernel(const __grid_c
                 const float phi = pos * a.inv_freq[p];  // one FP32 rounding
                 float sv, cv;
                 sincosf(phi, &sv, &cv);
+                if constexpr (V2) {
+                    cv = round_to<T>(cv);
+                    sv = round_to<T>(sv);
+                }
                 cs[k * half + p] = cv;
                 sn[k * half + p] = sv;
             }
@@ -320,7 +327,10 @@ __global__ void __launch_bounds__(256, 3) qk_norm_rope_bwd_kernel(const __grid_c
 #pragma unroll
             for (int j = 0; j < H; ++j) {
                 f32x2 me = de[j], mo = dd[j];
-                if constexpr (ROPE) {  // R^T: (c dy0 + s dy1, -s dy0 + c dy1)
+                if constexpr (ROPE && V2) {  // bf16 products, their sums rounded below
+                    me = f2_add(round_pair<T>(f2_mul(de[j], c2[j])), round_pair<T>(f2_mul(dd[j], s2[j])));
+                    mo = f2_add(round_pair<T>(f2_mul(dd[j], c2[j])), round_pair<T>(f2_mul(de[j], n2[j])));
+                } else if constexpr (ROPE) {  // R^T: (c dy0 + s dy1, -s dy0 + c dy1)
                     me = f2_fma(dd[j], s2[j], f2_mul(de[j], c2[j]));
                     mo = f2_fma(de[j], n2[j], f2_mul(dd[j], c2[j]));
                 }
@@ -425,7 +435,7 @@ cudaError_t launch_gate_bwd_t(const GateBwdArgs& a, cudaStream_t s) {
     return launch_gate_head<T, 16, 1>(a, s);
 }
 
-template <typename T, int L, bool ROPE>
+template <typename T, int L, bool ROPE, bool V2>
 cudaError_t launch_qk_bwd_l(const QkBwdArgs& a0, cudaStream_t s) {
     constexpr int RW = 32 / L;
     constexpr int BATCH = kBwdBatch;
@@ -446,8 +456,8 @@ cudaError_t launch_qk_bwd_l(const QkBwdArgs& a0, cudaStream_t s) {
     const int64_t grid = (a.tokens + tt - 1) / tt;
     const bool exact = split == 1 && a.head_dim / Vec<T>::N == L && a.hq % RW == 0 &&
                        a.hkv % RW == 0 && nst_q % BATCH == 0 && nst_k % BATCH == 0;
-    auto kern = exact ? qk_norm_rope_bwd_kernel<T, L, ROPE, false, BATCH, kBwdRing>
-                      : qk_norm_rope_bwd_kernel<T, L, ROPE, true, BATCH, kBwdRing>;
+    auto kern = exact ? qk_norm_rope_bwd_kernel<T, L, ROPE, V2, false, BATCH, kBwdRing>
+                      : qk_norm_rope_bwd_kernel<T, L, ROPE, V2, true, BATCH, kBwdRing>;
     if (smem > 48 * 1024) {
         const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
@@ -456,19 +466,23 @@ cudaError_t launch_qk_bwd_l(const QkBwdArgs& a0, cudaStream_t s) {
 }
 
 template <typename T, int L>
-cudaError_t launch_qk_bwd_r(int use_rope, const QkBwdArgs& a, cudaStream_t s) {
-    return use_rope ? launch_qk_bwd_l<T, L, true>(a, s) : launch_qk_bwd_l<T, L, false>(a, s);
+cudaError_t launch_qk_bwd_r(int use_rope, int upcast, const QkBwdArgs& a, cudaStream_t s) {
+    if (!use_rope) return launch_qk_bwd_l<T, L, false, false>(a, s);
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        if (!upcast) return launch_qk_bwd_l<T, L, true, true>(a, s);
+    }
+    return launch_qk_bwd_l<T, L, true, false>(a, s);
 }
 
 template <typename T>
-cudaError_t launch_qk_bwd_t(int use_rope, const QkBwdArgs& a, cudaStream_t s) {
+cudaError_t launch_qk_bwd_t(int use_rope, int upcast, const QkBwdArgs& a, cudaStream_t s) {
     const int nv = a.f.head_dim / Vec<T>::N;
-    if (nv > 16) return launch_qk_bwd_r<T, 32>(use_rope, a, s);
-    if (nv <= 1) return launch_qk_bwd_r<T, 1>(use_rope, a, s);
-    if (nv <= 2) return launch_qk_bwd_r<T, 2>(use_rope, a, s);
-    if (nv <= 4) return launch_qk_bwd_r<T, 4>(use_rope, a, s);
-    if (nv <= 8) return launch_qk_bwd_r<T, 8>(use_rope, a, s);
-    return launch_qk_bwd_r<T, 16>(use_rope, a, s);
+    if (nv > 16) return launch_qk_bwd_r<T, 32>(use_rope, upcast, a, s);
+    if (nv <= 1) return launch_qk_bwd_r<T, 1>(use_rope, upcast, a, s);
+    if (nv <= 2) return launch_qk_bwd_r<T, 2>(use_rope, upcast, a, s);
+    if (nv <= 4) return launch_qk_bwd_r<T, 4>(use_rope, upcast, a, s);
+    if (nv <= 8) return launch_qk_bwd_r<T, 8>(use_rope, upcast, a, s);
+    return launch_qk_bwd_r<T, 16>(use_rope, upcast, a, s);
 }
 
 }  // namespace
@@ -477,8 +491,10 @@ cudaError_t launch_gate_bwd(int dtype, const GateBwdArgs& a, cudaStream_t s) {
     return dtype == 0 ? launch_gate_bwd_t<__nv_bfloat16>(a, s) : launch_gate_bwd_t<float>(a, s);
 }
 
-cudaError_t launch_qk_bwd(int dtype, int use_rope, const QkBwdArgs& a, cudaStream_t s) {
-    return dtype == 0 ? launch_qk_bwd_t<__nv_bfloat16>(use_rope, a, s) : launch_qk_bwd_t<float>(use_rope, a, s);
+cudaError_t launch_qk_bwd(int dtype, int use_rope, int upcast_rope, const QkBwdArgs& a, cudaStream_t s) {
+    // FP32 tensors rotate in FP32 in both modes.
+    return dtype == 0 ? launch_qk_bwd_t<__nv_bfloat16>(use_rope, upcast_rope, a, s)
+                      : launch_qk_bwd_t<float>(use_rope, 1, a, s);
 }
 
 cudaError_t read_qk_bwd_device_error(unsigned int* out, bool clear) {

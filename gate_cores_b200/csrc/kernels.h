@@ -136,7 +136,7 @@ struct QkBwdArgs {
     const void* gk;
     int64_t gq_stride, gk_stride;
 };
-cudaError_t launch_qk_bwd(int dtype, int use_rope, const QkBwdArgs& a, cudaStream_t s);
+cudaError_t launch_qk_bwd(int dtype, int use_rope, int upcast_rope, const QkBwdArgs& a, cudaStream_t s);
 cudaError_t read_qk_bwd_device_error(unsigned int* out, bool clear);
 
 // Returns cudaSuccess or the launch error.

@@ -311,16 +311,21 @@ muse_status muse_output_norm_gate_backward(const void* o, const void* gate, cons
                                            float eps, cudaStream_t stream);
 
 /*
- * Backward of core 3 (_qk_norm_rope_core) with the FP32 (legacy, upcast)
- * rotation or none.  Per token and head, with phi the forward's FP32 angle
- * (same positions rule and layouts as muse_qk_norm_rope):
- *   dm = R(phi)^T dy, i.e. per pair (c dy0 + s dy1, -s dy0 + c dy1), FP32;
- *   dn = cast(dm); query heads: dn = cast(dn * query_scale);
+ * Backward of core 3 (_qk_norm_rope_core; the rotation modes of
+ * MuseSparkAttention's upcast_rope and apply_rotary_embedding).  Per token
+ * and head, with phi the forward's FP32 angle (same positions rule and
+ * layouts as muse_qk_norm_rope):
+ *   upcast_rope != 0 (legacy, FP32 rotation), or FP32 tensors:
+ *     dm = R(phi)^T dy, i.e. per pair (c dy0 + s dy1, -s dy0 + c dy1), FP32;
+ *     dn = cast(dm);
+ *   upcast_rope == 0 on bf16 (v2: the forward's products and sums in bf16,
+ *   C, S = bf16 cos and sin of phi), the gradient through those operations:
+ *     dn = (cast(cast(dy0 C) + cast(dy1 S)), cast(cast(dy1 C) - cast(dy0 S)));
+ *   query heads: dn = cast(dn * query_scale);
  *   dx = r dn - r^3 x (sum_j dn_j x_j) / head_dim, cast to dtype.
  * q, k are the forward's inputs; dq_out, dk_out the incoming gradients; dq,
  * dk the results, each with its own token stride (elements).  dq may be the
- * very memory of q or dq_out, dk of k or dk_out.  The v2 (bf16-product)
- * rotation has no backward here.
+ * very memory of q or dq_out, dk of k or dk_out.
  */
 muse_status muse_qk_norm_rope_backward(const void* q, const void* k, const void* dq_out,
                                        const void* dk_out, void* dq, void* dk, muse_dtype dtype,
@@ -331,7 +336,8 @@ muse_status muse_qk_norm_rope_backward(const void* q, const void* k, const void*
                                        int64_t k_tok_stride, int64_t dq_out_tok_stride,
                                        int64_t dk_out_tok_stride, int64_t dq_tok_stride,
                                        int64_t dk_tok_stride, float eps, float query_scale,
-                                       int use_rope, float rope_base, cudaStream_t stream);
+                                       int use_rope, int upcast_rope, float rope_base,
+                                       cudaStream_t stream);
 
 /*
  * Device-side error flags of the current device, for diagnostics.  The row

@@ -136,7 +136,7 @@ HEAD_WLS = [
     inputs.WORKLOADS["prefill_t8192_h4096"],
 ]
 GATE_CASES = ["per_head", "per_token", "f32"]
-QK_CASES = ["upcast", "qscale", "no_rope", "explicit_pos", "f32"]
+QK_CASES = ["upcast", "qscale", "no_rope", "explicit_pos", "f32", "v2", "v2_qscale"]
 
 
 @pytest.mark.parametrize("wl", HEAD_WLS, ids=lambda w: w.name)
@@ -175,11 +175,12 @@ def test_qk_norm_rope_backward(cuda_ok, wl, variant):
     dq, dk = cores.qk_norm_rope_backward(
         qd, kd, gqd, gkd, positions=None if pos is None else pos.cuda(),
         cu_seqlens=t["cu_seqlens"].cuda() if s["layout"] == "thd" else None, eps=s["eps"],
-        query_scale=s.get("query_scale", 1.0), use_rope=s.get("use_rope", True), rope_base=s["rope_base"])
+        query_scale=s.get("query_scale", 1.0), use_rope=s.get("use_rope", True), rope_base=s["rope_base"],
+        upcast_rope=s.get("upcast_rope", True))
     torch.cuda.synchronize()
     rq, rk = oracle.qk_norm_rope_bwd(_np(q), _np(k), _np(gq), _np(gk), harness.all_positions(wl, ci),
                                      s["eps"], s.get("query_scale", 1.0), s.get("use_rope", True),
-                                     s["rope_base"])
+                                     s["rope_base"], upcast_rope=s.get("upcast_rope", True))
     what = f"{wl.name}/qk_norm_rope/{variant}"
     check(_np(dq.reshape(q.shape)), rq, what + "/dq", backward=True)
     check(_np(dk.reshape(k.shape)), rk, what + "/dk", backward=True)
