@@ -80,6 +80,11 @@ def _load():
             lib.muse_oracle_norm_residual_bwd.argtypes = [
                 P, c_int, P, P, i64, i64, P, f32, P, c_int, f32, c_int,
                 P, P, P, P, P, P, P, P, P, P, P, P, P, P]
+            lib.muse_oracle_vision_rope_frequencies.argtypes = [i32, i32, i32, f32, P]
+            lib.muse_oracle_vision_rope.argtypes = [c_int, P, P, i64, i32, i32, i32, P,
+                                                    P, P, P, P, P, P, P, P]
+            for name in ("muse_oracle_vision_rope_frequencies", "muse_oracle_vision_rope"):
+                getattr(lib, name).restype = c_int
             for name in ("muse_oracle_inv_freq", "muse_oracle_positions", "muse_oracle_rms_norm",
                          "muse_oracle_input_scale_norm", "muse_oracle_qk_norm_rope",
                          "muse_oracle_output_norm_gate", "muse_oracle_norm_residual",
@@ -348,3 +353,27 @@ def norm_residual_bwd(stream, branch, dstream_out, theta, gain=None, gain_offset
         _ptr(ghi), _ptr(gmag), _ptr(tlo), _ptr(thi), _ptr(tmag)), "norm_residual_bwd")
     return ((ds, sl, sh, sm), (db, bl, bh, bm), None if gain is None else (glo, ghi, gmag),
             (tlo, thi, tmag))
+
+
+def vision_rope_frequencies(head_dim, grid_h, grid_w, theta=10000.0) -> np.ndarray:
+    """Vision 2-D RoPE table of one row-major grid: float32 [grid_h*grid_w, head_dim/2, 2]."""
+    out = np.empty((grid_h * grid_w, head_dim // 2, 2), np.float32)
+    _check(_load().muse_oracle_vision_rope_frequencies(head_dim, grid_h, grid_w, theta, _ptr(out)),
+           "vision_rope_frequencies")
+    return out
+
+
+def vision_rope(q, k, freqs):
+    """Vision 2-D RoPE of q [T, hq, D], k [T, hk, D] with freqs [T, D/2, 2]: (q', k')."""
+    q, k = _c(q), _c(k)
+    freqs = np.ascontiguousarray(freqs, dtype=np.float32)
+    T, hq, d = q.shape
+    hk = k.shape[1]
+    assert k.shape[0] == T and k.shape[2] == d and freqs.shape == (T, d // 2, 2)
+    qo, ko = np.empty_like(q), np.empty_like(k)
+    ql, qh, qm = _checks(q.shape)
+    kl, kh, km = _checks(k.shape)
+    _check(_load().muse_oracle_vision_rope(_dt(q), _ptr(q), _ptr(k), T, hq, hk, d, _ptr(freqs),
+                                           _ptr(qo), _ptr(ql), _ptr(qh), _ptr(qm), _ptr(ko),
+                                           _ptr(kl), _ptr(kh), _ptr(km)), "vision_rope")
+    return (qo, ql, qh, qm), (ko, kl, kh, km)

@@ -908,3 +908,70 @@ int muse_oracle_qk_norm_rope_bwd(int dtype, const void* q, const void* k, const 
     free(gr);
     return 0;
 }
+
+/* ------------------------------------------------------- vision 2-D RoPE */
+
+/* _rope_frequencies (vision page): the table [grid_h * grid_w, D/2, 2] of one
+ * row-major patch grid, the (cos, sin) of each adjacent pair's angle.
+ * Reading (the page gives the shape only): the first D/4 pairs take the
+ * patch's row index h, the other D/4 its column index w, each with the
+ * frequencies theta^(-2j/(D/2)), j = 0 .. D/4 - 1 (the text model's inverse
+ * frequencies over half the head); the angle is f32(f32(coord) * freq) and
+ * its cosine and sine are rounded to FP32.  head_dim a multiple of 4. */
+int muse_oracle_vision_rope_frequencies(int32_t head_dim, int32_t grid_h, int32_t grid_w,
+                                        float theta, float* out) {
+    if (head_dim <= 0 || (head_dim & 3) || grid_h < 0 || grid_w < 0 || !(theta > 0.0f)) return -1;
+    if ((int64_t)grid_h * grid_w > 0 && !out) return -1;
+    const int32_t quarter = head_dim / 4;
+    float* f = (float*)malloc(sizeof(float) * (size_t)quarter);
+    if (!f) return -1;
+    if (muse_oracle_inv_freq(head_dim / 2, theta, f) != 0) { free(f); return -1; }
+    for (int32_t h = 0; h < grid_h; ++h)
+        for (int32_t w = 0; w < grid_w; ++w) {
+            float* row = out + ((int64_t)h * grid_w + w) * head_dim;
+            for (int32_t i = 0; i < head_dim / 2; ++i) {
+                const float coord = (float)(i < quarter ? h : w);
+                const float phi = coord * f[i < quarter ? i : i - quarter];
+                row[2 * i] = (float)cos((double)phi);
+                row[2 * i + 1] = (float)sin((double)phi);
+            }
+        }
+    free(f);
+    return 0;
+}
+
+/* _apply_vision_rope (vision page): adjacent-pair RoPE of q [tokens, hq, D]
+ * and k [tokens, hk, D] with the caller's table freqs [tokens, D/2, 2] of
+ * (cos, sin) per token and pair: y[2i] = a c - b s, y[2i+1] = a s + b c, in
+ * FP32 arithmetic on the Q/K values, cast once to their dtype (reading: the
+ * legacy precision of the text rotation). */
+static void vision_rope_rows(int dtype, const void* x, int64_t tokens, int32_t heads, int32_t d,
+                             const float* freqs, void* out, double* lo, double* hi, double* mag) {
+    for (int64_t t = 0; t < tokens; ++t)
+        for (int32_t h = 0; h < heads; ++h) {
+            const int64_t base = (t * heads + h) * (int64_t)d;
+            for (int32_t i = 0; i < d / 2; ++i) {
+                const double c = (double)freqs[(t * (d / 2) + i) * 2];
+                const double s = (double)freqs[(t * (d / 2) + i) * 2 + 1];
+                const double a = load_elem(dtype, x, base + 2 * i);
+                const double b = load_elem(dtype, x, base + 2 * i + 1);
+                const double y0 = a * c - b * s, y1 = a * s + b * c;
+                store_elem(dtype, out, base + 2 * i, y0);
+                store_elem(dtype, out, base + 2 * i + 1, y1);
+                put_check(lo, hi, mag, base + 2 * i, y0, y0, fabs(a * c) + fabs(b * s));
+                put_check(lo, hi, mag, base + 2 * i + 1, y1, y1, fabs(a * s) + fabs(b * c));
+            }
+        }
+}
+
+int muse_oracle_vision_rope(int dtype, const void* q, const void* k, int64_t tokens, int32_t hq,
+                            int32_t hk, int32_t head_dim, const float* freqs, void* q_out,
+                            double* q_lo, double* q_hi, double* q_mag, void* k_out, double* k_lo,
+                            double* k_hi, double* k_mag) {
+    if (!valid_dtype(dtype) || tokens < 0 || hq <= 0 || hk <= 0 || head_dim <= 0 || (head_dim & 1))
+        return -1;
+    if (tokens && (!q || !k || !freqs || !q_out || !k_out)) return -1;
+    vision_rope_rows(dtype, q, tokens, hq, head_dim, freqs, q_out, q_lo, q_hi, q_mag);
+    vision_rope_rows(dtype, k, tokens, hk, head_dim, freqs, k_out, k_lo, k_hi, k_mag);
+    return 0;
+}

@@ -189,6 +189,20 @@ int muse_oracle_norm_residual_bwd(const float* stream, int branch_dtype, const v
                                   double* dgain_lo, double* dgain_hi, double* dgain_mag,
                                   double* dtheta_lo, double* dtheta_hi, double* dtheta_mag);
 
+/* Vision 2-D RoPE (page "...muse_spark.vision": _rope_frequencies,
+ * _apply_vision_rope).  Frequencies of one row-major grid, out
+ * [grid_h * grid_w, head_dim / 2, 2] = (cos, sin) per pair: the first
+ * head_dim / 4 pairs from the patch row, the rest from the column, with
+ * frequencies theta^(-2j/(head_dim/2)) (a reading; the page gives the shape).
+ * The rotation: y[2i] = a c - b s, y[2i+1] = a s + b c per token and head
+ * with the token's (c, s) from freqs [tokens, head_dim / 2, 2], one cast. */
+int muse_oracle_vision_rope_frequencies(int32_t head_dim, int32_t grid_h, int32_t grid_w,
+                                        float theta, float* out);
+int muse_oracle_vision_rope(int dtype, const void* q, const void* k, int64_t tokens, int32_t hq,
+                            int32_t hk, int32_t head_dim, const float* freqs, void* q_out,
+                            double* q_lo, double* q_hi, double* q_mag, void* k_out, double* k_lo,
+                            double* k_hi, double* k_mag);
+
 #ifdef __cplusplus
 }
 #endif

@@ -490,3 +490,94 @@ def test_rms_norm_grouped_pins():
     assert np.array_equal(one, oracle.rms_norm(x, g, 0.0, 1e-6)[0])
     with pytest.raises(ValueError):
         oracle.rms_norm_grouped(x, gains, np.array([0, 3, 2, 9], np.int32))
+
+
+# ------------------------------------------------------- vision 2-D RoPE
+
+def _vision_inputs(seed, T=5, hq=3, hk=2, D=16, dtype="bf16"):
+    r = rng(seed)
+    q = r.standard_normal((T, hq, D)) * 2.0
+    k = r.standard_normal((T, hk, D)) * 2.0
+    if dtype == "bf16":
+        return bf16(q), bf16(k)
+    return q.astype(np.float32), k.astype(np.float32)
+
+
+def _table(T, D, angles):
+    f = np.empty((T, D // 2, 2), np.float32)
+    f[..., 0] = np.cos(angles)
+    f[..., 1] = np.sin(angles)
+    return f
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_vision_rope_identity_and_quarter_turn(dtype):
+    # (c, s) = (1, 0) leaves every element unchanged; (0, 1) maps (a, b) to (-b, a)
+    q, k = _vision_inputs(30, dtype=dtype)
+    T, D = q.shape[0], q.shape[2]
+    ident = np.zeros((T, D // 2, 2), np.float32)
+    ident[..., 0] = 1.0
+    (qo, lo, hi, _), (ko, *_) = oracle.vision_rope(q, k, ident)
+    assert np.array_equal(qo, q) and np.array_equal(ko, k) and np.array_equal(lo, hi)
+    quarter = np.zeros_like(ident)
+    quarter[..., 1] = 1.0
+    (qo, *_), _ = oracle.vision_rope(q, k, quarter)
+    val = from_bf16 if dtype == "bf16" else (lambda a: a.astype(np.float64))
+    assert np.array_equal(val(qo)[..., 0::2], -val(q)[..., 1::2])
+    assert np.array_equal(val(qo)[..., 1::2], val(q)[..., 0::2])
+
+
+def test_vision_rope_is_complex_multiplication():
+    # adjacent pairs (2i, 2i+1) as a + ib, the table's (c, s) as c + is:
+    # the exact rotated value is their complex product (numpy complex128)
+    q, k = _vision_inputs(31, T=7, D=24)
+    T, D = q.shape[0], q.shape[2]
+    ang = rng(32).uniform(-40.0, 40.0, (T, D // 2))
+    f = _table(T, D, ang)
+    (qo, lo, hi, mag), (ko, klo, _, _) = oracle.vision_rope(q, k, f)
+    for x, l in ((q, lo), (k, klo)):
+        xv = from_bf16(x)
+        z = (xv[..., 0::2] + 1j * xv[..., 1::2]) * (f[None, :, :, 0].astype(np.float64).transpose(1, 0, 2)
+                                                    + 1j * f[None, :, :, 1].astype(np.float64).transpose(1, 0, 2))
+        ref = np.stack([z.real, z.imag], -1).reshape(x.shape)
+        assert np.allclose(l, ref, rtol=1e-13, atol=1e-300)
+    assert np.array_equal(lo, hi)
+    assert np.all(mag >= np.abs(lo))
+
+
+def test_vision_rope_preserves_pair_norms_and_composes():
+    # a unit (c, s) keeps |(a, b)|; rotating by alpha then beta equals one
+    # rotation by alpha + beta (exact arithmetic on the oracle's pre-cast values)
+    q, k = _vision_inputs(33, dtype="f32")
+    T, D = q.shape[0], q.shape[2]
+    r = rng(34)
+    al, be = r.uniform(-3, 3, (T, D // 2)), r.uniform(-3, 3, (T, D // 2))
+    (_, lo1, _, _), _ = oracle.vision_rope(q, k, _table(T, D, al))
+    n0 = q.astype(np.float64)[..., 0::2] ** 2 + q.astype(np.float64)[..., 1::2] ** 2
+    n1 = lo1[..., 0::2] ** 2 + lo1[..., 1::2] ** 2
+    assert np.allclose(n1, n0, rtol=1e-6)
+    (q1, *_), _ = oracle.vision_rope(q, k, _table(T, D, al))
+    (_, lo2, _, _), _ = oracle.vision_rope(q1, k, _table(T, D, be))
+    (_, lo3, _, _), _ = oracle.vision_rope(q, k, _table(T, D, al + be))
+    assert np.allclose(lo2, lo3, rtol=1e-5, atol=1e-5)
+
+
+def test_vision_rope_frequencies_reading():
+    # patch (0, 0): every angle 0; the first D/4 pairs vary with the row only,
+    # the others with the column only; angles grow linearly with the index and
+    # fall geometrically over the pairs (ratio theta^(-2/(D/2)))
+    D, Hg, Wg, theta = 16, 3, 5, 100.0
+    f = oracle.vision_rope_frequencies(D, Hg, Wg, theta).reshape(Hg, Wg, D // 2, 2)
+    assert np.array_equal(f[0, 0, :, 0], np.ones(D // 2, np.float32))
+    assert np.array_equal(f[0, 0, :, 1], np.zeros(D // 2, np.float32))
+    assert np.allclose(f[..., 0] ** 2 + f[..., 1] ** 2, 1.0, atol=1e-6)
+    q4 = D // 4
+    assert np.all(f[:, :, :q4] == f[:, :1, :q4])   # row half: same along a row
+    assert np.all(f[:, :, q4:] == f[:1, :, q4:])   # column half: same down a column
+    ang = np.arctan2(f[..., 1].astype(np.float64), f[..., 0].astype(np.float64))
+    # row 1 / column 1 give the frequencies themselves (all below pi)
+    fr, fc = ang[1, 0, :q4], ang[0, 1, q4:]
+    assert np.allclose(fr, fc, rtol=1e-6)
+    assert np.allclose(fr[1:] / fr[:-1], theta ** (-2.0 / (D // 2)), rtol=1e-5)
+    assert abs(fr[0] - 1.0) < 1e-6
+    assert np.allclose(ang[2, 0, :q4], np.angle(np.exp(2j * fr)), rtol=1e-5, atol=1e-6)
