@@ -354,6 +354,48 @@ def grouped_call(st: "Step", experts: int = 64):
     return call
 
 
+def vision_call(name: str = "vision_i16_g32x32_h16x80"):
+    """Vision 2-D RoPE on a packed batch of patch grids: the table built by
+    muse_vision_rope_frequencies (one launch per image, written in patch
+    order), then a callable rotating Q and K into fresh outputs."""
+    vw = inputs.VISION_WORKLOADS[name]
+    q, k = (t.cuda() for t in inputs.vision_qk(vw, 0))
+    per = vw.grid_h * vw.grid_w
+    table = torch.empty((vw.tokens, vw.head_dim // 2, 2), dtype=torch.float32, device="cuda")
+    for i in range(vw.images):
+        cores.vision_rope_frequencies(vw.head_dim, vw.grid_h, vw.grid_w, vw.theta, out=table[i * per:(i + 1) * per])
+    qo, ko = torch.empty_like(q), torch.empty_like(k)
+
+    def call():
+        cores.vision_rope(q, k, table, q_out=qo, k_out=ko)
+
+    return vw, call
+
+
+def vision_rope_timing(peak: float, flush: torch.Tensor, warmup: int = 10, reps: int = 50):
+    """The vision rotation alone: median of `reps` launches, L2 read-flushed before each."""
+    vw, call = vision_call()
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    torch.cuda._sleep(20_000_000)
+    ev = []
+    for i in range(warmup + reps):
+        flush.amax()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        if i >= warmup:
+            ev.append((e0, e1))
+    torch.cuda.synchronize()
+    us = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+    nb = vw.tokens * (2 * 2 * 2 * vw.heads * vw.head_dim + 4 * vw.head_dim)  # Q, K in and out (bf16); table
+    return {"workload": vw.name, "tokens": vw.tokens, "us": round(us, 3),
+            "tokens_per_s": round(vw.tokens / (us * 1e-6), 1), "gbs": round(nb / (us * 1e-6) / 1e9, 1),
+            "frac": round(nb / (us * 1e-6) / 1e9 / peak, 4), "algo_bytes": nb,
+            "note": "muse_vision_rope: Q and K (16 heads x 80) of 16 images of 32x32 patches, bf16"}
+
+
 def grouped_norm(st: "Step", peak: float, flush: torch.Tensor, experts: int = 64, warmup: int = 10,
                  reps: int = 50):
     """Per-expert core 1 (MoE pre/post expert norm) on the batch's activations
@@ -639,6 +681,7 @@ def run_ours(args, world, rank, local):
     del bst
     fused = fused_vs_unfused(st, peak, flush)
     grouped = grouped_norm(st, peak, flush)
+    vision = vision_rope_timing(peak, flush)
     del flush
     torch.cuda.empty_cache()
 
@@ -666,6 +709,7 @@ def run_ours(args, world, rank, local):
             "backward": backward,
             "fused_residual_prenorm": fused,
             "per_expert_norm": grouped,
+            "vision_rope": vision,
             "roofline": roofline,
             "copy_kernel_gbs": None if copy_gbs is None else round(copy_gbs, 1),
             "e2e": e2e,
@@ -765,15 +809,17 @@ def run_reference(args, world, rank):
 
 
 def profile_pass(args):
-    """Each forward core, each backward core, then core 5 fused with the next
-    pre-norm and the per-expert core 1, the sequence launched twice on the
-    workload's batch: a short, fixed launch sequence for an ncu capture (16
-    kernel launches per pass; skip the first pass to capture warm ones)."""
+    """Each forward core, each backward core, core 5 fused with the next
+    pre-norm, the per-expert core 1 and the vision RoPE, the sequence launched
+    twice on the workload's batch: a short, fixed launch sequence for an ncu
+    capture (16 table launches first, then 17 kernel launches per pass; skip
+    the table and the first pass to capture warm ones)."""
     wl = WORKLOADS[args.workload]
     st = Step(wl, seed=0)
     bst = BwdStep(st, seed=0)
     fused, _ = fused_calls(st)
     grouped = grouped_call(st)
+    _, vision = vision_call()  # 16 table launches before the passes
     for _ in range(2):
         for c in CORE_ORDER:
             st.launch(c)
@@ -781,9 +827,10 @@ def profile_pass(args):
             bst.launch(c)
         fused()
         grouped()
+        vision()
     torch.cuda.synchronize()
-    print("profile pass: 2 x (5 forward + 5 backward calls, fused core 5 + pre-norm, per-expert core 1) on "
-          + wl.name, file=sys.stderr)
+    print("profile pass: 16 vision-table launches, then 2 x (5 forward + 5 backward calls, fused core 5 + "
+          "pre-norm, per-expert core 1, vision RoPE) on " + wl.name, file=sys.stderr)
 
 
 def main():

@@ -33,6 +33,7 @@ EXPORTS = (
     "muse_input_scale_norm_backward", "muse_norm_residual_backward",
     "muse_output_norm_gate_backward", "muse_qk_norm_rope_backward",
     "muse_rms_norm_backward_noalloc", "muse_norm_residual_rms_norm", "muse_rms_norm_grouped",
+    "muse_vision_rope", "muse_vision_rope_frequencies",
 )
 
 
@@ -93,6 +94,8 @@ def load() -> ctypes.CDLL:
         lib.muse_qk_norm_rope_backward.argtypes = [P, P, P, P, P, P, c_int, c_int, i64, i64, P,
                                                    i32, i64, P, i32, i32, i32, i64, i64, i64, i64,
                                                    i64, i64, f32, f32, c_int, c_int, f32, P]
+        lib.muse_vision_rope.argtypes = [P, P, P, P, c_int, i64, i32, i32, i32, i64, i64, i64, i64, P, P]
+        lib.muse_vision_rope_frequencies.argtypes = [P, i32, i32, i32, f32, P]
         for name in EXPORTS[3:]:
             getattr(lib, name).restype = c_int
         lib.muse_norm_backward_workspace_bytes.restype = sz
@@ -227,3 +230,13 @@ def muse_rms_norm_grouped(x, y, dtype, rows, hidden, x_row_stride, y_row_stride,
                           group_offsets, num_groups, eps, stream) -> None:
     _call("muse_rms_norm_grouped", x, y, dtype, rows, hidden, x_row_stride, y_row_stride, gains,
           gain_offset, group_offsets, num_groups, eps, stream)
+
+
+def muse_vision_rope(q, k, q_out, k_out, dtype, tokens, hq, hk, head_dim, q_tok_stride, k_tok_stride,
+                     q_out_tok_stride, k_out_tok_stride, freqs, stream) -> None:
+    _call("muse_vision_rope", q, k, q_out, k_out, dtype, tokens, hq, hk, head_dim, q_tok_stride,
+          k_tok_stride, q_out_tok_stride, k_out_tok_stride, freqs, stream)
+
+
+def muse_vision_rope_frequencies(out, head_dim, grid_h, grid_w, theta, stream) -> None:
+    _call("muse_vision_rope_frequencies", out, head_dim, grid_h, grid_w, theta, stream)

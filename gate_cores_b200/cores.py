@@ -208,6 +208,42 @@ def rms_norm_grouped(x: torch.Tensor, gains: torch.Tensor, group_offsets: torch.
     return y
 
 
+def vision_rope(q: torch.Tensor, k: torch.Tensor, freqs: torch.Tensor, q_out: torch.Tensor | None = None,
+                k_out: torch.Tensor | None = None, stream=None):
+    """Vision 2-D RoPE: q [T, hq, D], k [T, hk, D] rotated by freqs FP32
+    [T, D/2, 2] ((cos, sin) per token and pair); returns (q', k') in q's
+    dtype.  q_out / k_out may be q / k (in place)."""
+    _cuda(q, k, freqs, q_out, k_out)
+    if q.dim() != 3 or k.dim() != 3 or q.shape[0] != k.shape[0] or q.shape[-1] != k.shape[-1]:
+        raise ValueError("q, k must be [T, heads, head_dim] with the same T and head_dim")
+    if q.dtype != k.dtype:
+        raise TypeError("q and k must share a dtype")
+    T, hq, d = q.shape
+    hk = k.shape[1]
+    if freqs.dtype != torch.float32 or tuple(freqs.shape) != (T, d // 2, 2):
+        raise ValueError("freqs must be float32 [T, head_dim/2, 2]")
+    freqs = freqs.contiguous()
+    qo = torch.empty_like(q, memory_format=torch.contiguous_format) if q_out is None else q_out
+    ko = torch.empty_like(k, memory_format=torch.contiguous_format) if k_out is None else k_out
+    _lib.muse_vision_rope(q.data_ptr(), k.data_ptr(), qo.data_ptr(), ko.data_ptr(), _dtype(q), T, hq, hk, d,
+                          _tok_stride(q, hq, d), _tok_stride(k, hk, d), _tok_stride(qo, hq, d),
+                          _tok_stride(ko, hk, d), freqs.data_ptr(), _stream(stream))
+    return qo, ko
+
+
+def vision_rope_frequencies(head_dim: int, grid_h: int, grid_w: int, theta: float = 10000.0,
+                            out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The vision RoPE table of one row-major grid: FP32 [grid_h*grid_w, head_dim/2, 2]
+    on the current CUDA device (or written into `out`)."""
+    if out is None:
+        out = torch.empty((grid_h * grid_w, head_dim // 2, 2), dtype=torch.float32, device="cuda")
+    _cuda(out)
+    if out.dtype != torch.float32 or not out.is_contiguous() or out.numel() != grid_h * grid_w * head_dim:
+        raise ValueError("out must be contiguous float32 [grid_h*grid_w, head_dim/2, 2]")
+    _lib.muse_vision_rope_frequencies(out.data_ptr(), head_dim, grid_h, grid_w, theta, _stream(stream))
+    return out
+
+
 def norm_residual_rms_norm(stream_in: torch.Tensor, branch: torch.Tensor, theta: torch.Tensor,
                            gain: torch.Tensor | None = None, gain_offset: float = 0.0,
                            input_scale: bool = False, norm_eps: float = 1e-6,

@@ -813,4 +813,73 @@ muse_status muse_stream_copy(const void* src, void* dst, int64_t bytes, cudaStre
     return from_cuda(muse::launch_copy(src, dst, bytes, stream), name);
 }
 
+muse_status muse_vision_rope(const void* q, const void* k, void* q_out, void* k_out, muse_dtype dtype,
+                             int64_t tokens, int32_t hq, int32_t hk, int32_t head_dim,
+                             int64_t q_tok_stride, int64_t k_tok_stride, int64_t q_out_tok_stride,
+                             int64_t k_out_tok_stride, const float* freqs, cudaStream_t stream) {
+    const char* name = "muse_vision_rope";
+    if (!valid_dtype(dtype)) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, (int)dtype);
+    if (tokens < 0 || hq <= 0 || hk <= 0 || head_dim <= 0 || (head_dim & 1))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: tokens=%lld hq=%d hk=%d head_dim=%d", name,
+                    (long long)tokens, hq, hk, head_dim);
+    const int64_t qw = (int64_t)hq * head_dim, kw = (int64_t)hk * head_dim;
+    if (q_tok_stride < qw || q_out_tok_stride < qw || k_tok_stride < kw || k_out_tok_stride < kw)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: token strides must cover all heads", name);
+    if (tokens == 0) return MUSE_OK;
+    if (!q || !k || !q_out || !k_out || !freqs)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null q, k, q_out, k_out or freqs", name);
+    const int64_t es = elem_size(dtype);
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(q_out, 16) || !aligned(k_out, 16) || !aligned(freqs, 16) ||
+        (head_dim * es) % 16 || (q_tok_stride * es) % 16 || (k_tok_stride * es) % 16 ||
+        (q_out_tok_stride * es) % 16 || (k_out_tok_stride * es) % 16)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: pointers, head_dim and strides must be 16-byte multiples", name);
+    if ((qw + kw) / vec_elems(dtype) > (int64_t)1 << 30)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: token rows too wide", name);
+    const Span sq = span(q, tokens, qw, q_tok_stride, es), sk = span(k, tokens, kw, k_tok_stride, es);
+    const Span sqo = span(q_out, tokens, qw, q_out_tok_stride, es);
+    const Span sko = span(k_out, tokens, kw, k_out_tok_stride, es);
+    const Span sf = span(freqs, 1, tokens * head_dim, tokens * head_dim, 4);
+    if (bad_alias(sqo, sq, true) || bad_alias(sqo, sk, false) || bad_alias(sqo, sko, false) ||
+        bad_alias(sko, sk, true) || bad_alias(sko, sq, false) || bad_alias(sqo, sf, false) ||
+        bad_alias(sko, sf, false))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: output partially overlaps an input", name);
+    muse::VisionRopeArgs a{};
+    a.q = q;
+    a.k = k;
+    a.q_out = q_out;
+    a.k_out = k_out;
+    a.freqs = freqs;
+    a.tokens = tokens;
+    a.q_stride = q_tok_stride;
+    a.k_stride = k_tok_stride;
+    a.q_out_stride = q_out_tok_stride;
+    a.k_out_stride = k_out_tok_stride;
+    a.hq = hq;
+    a.hk = hk;
+    a.head_dim = head_dim;
+    return from_cuda(muse::launch_vision_rope(dtype, a, stream), name);
+}
+
+muse_status muse_vision_rope_frequencies(float* out, int32_t head_dim, int32_t grid_h, int32_t grid_w,
+                                         float theta, cudaStream_t stream) {
+    const char* name = "muse_vision_rope_frequencies";
+    if (head_dim <= 0 || (head_dim & 3) || grid_h < 0 || grid_w < 0 || !(finite(theta) && theta > 0.0f))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: head_dim=%d (a positive multiple of 4), grid %dx%d, theta > 0",
+                    name, head_dim, grid_h, grid_w);
+    if (head_dim / 4 > muse::kMaxHalfDim)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: head_dim=%d above %d", name, head_dim, 4 * muse::kMaxHalfDim);
+    if ((int64_t)grid_h * grid_w == 0) return MUSE_OK;
+    if (!out) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null out", name);
+    if (!aligned(out, 8)) return fail(MUSE_ERR_UNSUPPORTED, "%s: out not 8-byte aligned", name);
+    muse::VisionFreqArgs a{};
+    a.out = out;
+    a.head_dim = head_dim;
+    a.grid_h = grid_h;
+    a.grid_w = grid_w;
+    // frequencies over half the head: theta^(-2j/(head_dim/2)), rounded to FP32
+    for (int j = 0; j < head_dim / 4; ++j)
+        a.inv_freq[j] = (float)std::pow((double)theta, -(2.0 * j) / (double)(head_dim / 2));
+    return from_cuda(muse::launch_vision_rope_frequencies(a, stream), name);
+}
+
 }  // extern "C"

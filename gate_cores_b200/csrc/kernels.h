@@ -137,6 +137,29 @@ struct QkBwdArgs {
     int64_t gq_stride, gk_stride;
 };
 cudaError_t launch_qk_bwd(int dtype, int use_rope, int upcast_rope, const QkBwdArgs& a, cudaStream_t s);
+
+// Vision 2-D RoPE: Q [tokens, hq, head_dim] and K [tokens, hk, head_dim] with
+// per-token strides, rotated by the table freqs [tokens, head_dim/2, 2]
+// (cos, sin per pair, contiguous).
+struct VisionRopeArgs {
+    const void* q;
+    const void* k;
+    void* q_out;
+    void* k_out;
+    const float* freqs;
+    int64_t tokens;
+    int64_t q_stride, k_stride, q_out_stride, k_out_stride;  // elements per token
+    int32_t hq, hk, head_dim;
+};
+// The table of one row-major grid_h x grid_w patch grid: out
+// [grid_h * grid_w, head_dim/2, 2]; inv_freq[j], j < head_dim/4.
+struct VisionFreqArgs {
+    float* out;
+    int32_t head_dim, grid_h, grid_w;
+    float inv_freq[kMaxHalfDim];
+};
+cudaError_t launch_vision_rope(int dtype, const VisionRopeArgs& a, cudaStream_t s);
+cudaError_t launch_vision_rope_frequencies(const VisionFreqArgs& a, cudaStream_t s);
 cudaError_t read_qk_bwd_device_error(unsigned int* out, bool clear);
 
 // Returns cudaSuccess or the launch error.

@@ -165,6 +165,45 @@ def expert_gains(wl: Workload, seed: int, num_groups: int, zero_centered: bool) 
     return torch.stack(rows), off
 
 
+@dataclass(frozen=True)
+class VisionWorkload:
+    """Packed patches of the vision tower: `images` row-major grids of
+    grid_h x grid_w patches (448-pixel images at patch 14 give 32 x 32),
+    `heads` x `head_dim` per token for Q and K; the RoPE base."""
+    name: str
+    images: int
+    grid_h: int
+    grid_w: int
+    heads: int
+    head_dim: int
+    theta: float = 10000.0
+
+    @property
+    def tokens(self) -> int:
+        return self.images * self.grid_h * self.grid_w
+
+
+VISION_WORKLOADS = {
+    "vision_i16_g32x32_h16x80": VisionWorkload("vision_i16_g32x32_h16x80", 16, 32, 32, 16, 80),
+    "vision_i2_g5x7_h3x16": VisionWorkload("vision_i2_g5x7_h3x16", 2, 5, 7, 3, 16, 100.0),
+}
+
+
+def vision_qk(vw: VisionWorkload, seed: int, dtype=torch.bfloat16) -> tuple[torch.Tensor, torch.Tensor]:
+    """(q, k) [tokens, heads, head_dim]: N(0, 1) projections rounded to dtype."""
+    shape = (vw.tokens, vw.heads, vw.head_dim)
+    q = torch.randn(shape, generator=_gen(seed, vw.name, "vision_q"), dtype=torch.float32)
+    k = torch.randn(shape, generator=_gen(seed, vw.name, "vision_k"), dtype=torch.float32)
+    return q.to(dtype), k.to(dtype)
+
+
+def vision_angles(vw: VisionWorkload, seed: int) -> torch.Tensor:
+    """Arbitrary per-token pair angles U(-100, 100) rad [tokens, head_dim/2] for
+    tables not drawn from a grid."""
+    g = _gen(seed, vw.name, "vision_angles")
+    return torch.rand((vw.tokens, vw.head_dim // 2), generator=g, dtype=torch.float64) * 200.0 - 100.0
+
+
 def upstream_grad(wl: Workload, seed: int, tag: str, shape, dtype=torch.bfloat16) -> torch.Tensor:
     """Incoming gradient dL/d(output) for the backward calls: N(0, 1) drawn in
     FP32 and rounded to dtype (no outlier channels)."""

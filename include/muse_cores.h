@@ -178,6 +178,36 @@ muse_status muse_rms_norm_grouped(const void* x, void* y, muse_dtype dtype, int6
                                   float eps, cudaStream_t stream);
 
 /*
+ * Vision 2-D RoPE (page "nemo_automodel.components.models.muse_spark.vision":
+ * _apply_vision_rope, the adjacent-pair rotation of the NaViT tower's Q/K).
+ * Per token t, head and pair i, with (c, s) = freqs[t, i, 0..1]:
+ *   y[2i] = a c - b s,   y[2i+1] = a s + b c   (FP32, cast once to dtype),
+ * (a, b) = x[2i], x[2i+1].  q [tokens, hq, head_dim], k [tokens, hk,
+ * head_dim] (heads contiguous, per-token strides in elements, as the Q/K
+ * core), freqs FP32 [tokens, head_dim/2, 2] contiguous (the (cos, sin) of each
+ * pair's angle, e.g. from muse_vision_rope_frequencies per grid, concatenated
+ * in the packed patch order).  q_out may be the very memory of q, k_out of k;
+ * any other overlap is MUSE_ERR_INVALID_ARGUMENT.  Pointers, head rows and
+ * strides 16-byte multiples, else MUSE_ERR_UNSUPPORTED.
+ */
+muse_status muse_vision_rope(const void* q, const void* k, void* q_out, void* k_out, muse_dtype dtype,
+                             int64_t tokens, int32_t hq, int32_t hk, int32_t head_dim,
+                             int64_t q_tok_stride, int64_t k_tok_stride, int64_t q_out_tok_stride,
+                             int64_t k_out_tok_stride, const float* freqs, cudaStream_t stream);
+
+/*
+ * The vision RoPE table of one row-major grid_h x grid_w patch grid
+ * (_rope_frequencies): out [grid_h * grid_w, head_dim/2, 2] FP32, the (cos,
+ * sin) of each pair's angle.  The page gives the shape only; the reading
+ * here: pairs i < head_dim/4 take the patch row h, the others the column w,
+ * angle = f32(coord) * f32(theta^(-2j/(head_dim/2))), j the pair's index
+ * within its half.  head_dim a positive multiple of 4 (at most 512), theta
+ * > 0; out 8-byte aligned.
+ */
+muse_status muse_vision_rope_frequencies(float* out, int32_t head_dim, int32_t grid_h, int32_t grid_w,
+                                         float theta, cudaStream_t stream);
+
+/*
  * Core 5 fused with the next sublayer's pre-norm.  The decoder layer updates
  * the FP32 stream with core 5 and then normalises that stream for the next
  * sublayer (MuseSparkDecoderLayer: add_attn, then pre_ffn_norm; add_ffn, then
