@@ -138,3 +138,77 @@ def test_gate_and_residual_validation(lib):
     assert c(A, A + 4096, 0, None) == 0
     assert c(A, A + 4096, 8192, None) == INV            # overlapping ranges
     assert c(A, A + (1 << 20), 100, None) == UNS
+
+
+def test_grouped_and_fused_validation(lib):
+    gr = lib.muse_rms_norm_grouped
+    G, O = A + (1 << 26), A + (2 << 26)  # gains, offsets
+    assert gr(A, A + (1 << 24), BF16, 0, 256, 256, 256, G, 0.0, O, 4, 1e-6, None) == 0
+    assert gr(A, A + (1 << 24), BF16, 8, 256, 256, 256, G, 0.0, O, 0, 1e-6, None) == INV  # no groups
+    assert gr(A, A + (1 << 24), BF16, 8, 256, 256, 256, G, 0.0, None, 4, 1e-6, None) == INV
+    assert gr(A, A + (1 << 24), BF16, 8, 256, 256, 256, G, 0.0, O + 2, 4, 1e-6, None) == UNS
+    assert gr(A, A + (1 << 26), BF16, 8, 16384, 16384, 16384, G + (1 << 20), 0.0, O, 4, 1e-6,
+              None) == UNS                                   # above 1024 vectors per row
+    assert gr(A, G + 64, BF16, 8, 256, 256, 256, G, 0.0, O, 4, 1e-6, None) == INV  # y over the gains
+    fz = lib.muse_norm_residual_rms_norm
+    T = A + (3 << 26)
+    assert fz(A, A + (1 << 24), A + (2 << 24), A + (4 << 24), F32, BF16, 4, 256, None, 0.0, T, 0,
+              1e-6, None, 0.0, 1e-6, None) == UNS            # FP32 branch, bf16 y
+    assert fz(A, A + (1 << 24), A + (2 << 24), A + (4 << 24), BF16, F32, 0, 256, None, 0.0, T, 0,
+              1e-6, None, 0.0, 1e-6, None) == 0
+    assert fz(A, A + (1 << 24), A + (2 << 24), A + (2 << 24) + 512, BF16, F32, 4, 256, None, 0.0, T,
+              0, 1e-6, None, 0.0, 1e-6, None) == INV         # y inside stream_out
+
+
+def test_backward_validation(lib):
+    ws = lib.muse_norm_backward_workspace_bytes(64, 256)
+    assert ws >= 256 * 4
+    rb = lib.muse_rms_norm_backward
+    assert rb(A, A + (1 << 24), A + (2 << 24), BF16, 0, 256, 256, 256, 256, None, 0.0, 1e-6, None,
+              None, 0, None) == 0
+    assert rb(A, A + (1 << 24), A + (2 << 24), BF16, 64, 256, 256, 256, 256, A + (3 << 24), 0.0,
+              1e-6, A + (4 << 24), A + (5 << 24), 16, None) == INV  # workspace too small
+    qb = lib.muse_qk_norm_rope_backward
+    args = [A, A + (1 << 26), A + (2 << 26), A + (3 << 26), A + (4 << 26), A + (5 << 26), BF16, 0, 2,
+            8, None, 0, 0, None, 4, 2, 64, 256, 128, 256, 128, 256, 128, 1e-6, 1.0, 1, 0, 1e4, None]
+    # (args itself is valid and would launch: only its invalid variants are called)
+    bad = list(args)
+    bad[7] = 5                                               # unknown layout
+    assert qb(*bad) == INV
+    bad = list(args)
+    bad[16] = 63                                             # odd head_dim
+    assert qb(*bad) == INV
+    bad = list(args)
+    bad[4] = A + 64                                          # dq half a head into q
+    assert qb(*bad) == INV
+
+
+def test_vision_validation(lib):
+    v = lib.muse_vision_rope
+    F = A + (4 << 26)
+
+    def call(q=A, k=A + (1 << 26), qo=A + (2 << 26), ko=A + (3 << 26), dt=BF16, T=16, hq=4, hk=4,
+             d=64, qs=None, ks=None, qos=None, kos=None, f=F):
+        qs = hq * d if qs is None else qs
+        ks = hk * d if ks is None else ks
+        qos = hq * d if qos is None else qos
+        kos = hk * d if kos is None else kos
+        return v(q, k, qo, ko, dt, T, hq, hk, d, qs, ks, qos, kos, f, None)
+
+    assert call(T=0) == 0
+    assert call(hq=0) == INV
+    assert call(d=63) == INV
+    assert call(qs=100) == INV                               # stride below the heads
+    assert call(f=None) == INV
+    assert call(d=12) == UNS                                 # 24-byte bf16 heads
+    assert call(f=F + 8) == UNS                              # table not 16-byte aligned
+    assert call(qo=A + 64) == INV                            # q_out partially over q
+    assert call(ko=F + 256) == INV                           # k_out over the table
+    assert call(dt=7) == INV
+    fr = lib.muse_vision_rope_frequencies
+    assert fr(A, 64, 0, 32, 1e4, None) == 0
+    assert fr(A, 66, 4, 4, 1e4, None) == INV                 # head_dim not a multiple of 4
+    assert fr(A, 64, 4, 4, 0.0, None) == INV
+    assert fr(A, 1024, 4, 4, 1e4, None) == UNS
+    assert fr(A + 4, 64, 4, 4, 1e4, None) == UNS
+    assert fr(None, 64, 4, 4, 1e4, None) == INV
