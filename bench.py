@@ -676,7 +676,8 @@ def run_ours(args, world, rank, local):
                 "algo_bytes_per_step": bwd_bytes,
                 "gpu_launches_per_step": 9,
                 "per_core_isolated": bwd_iso,
-                "note": "gradients of the five cores (the Q/K call with the FP32 rotation); gain and "
+                "note": "gradients of the five cores (the Q/K call with the FP32 rotation; "
+                        "per_core_isolated.qk_norm_rope_v2 is the v2 rotation's backward alone); gain and "
                         "theta gradients reduced through the caller's workspace"}
     del bst
     fused = fused_vs_unfused(st, peak, flush)
