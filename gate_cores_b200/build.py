@@ -1,9 +1,11 @@
 """Build libmuse_cores.so in-tree with nvcc for sm_100a.
 
-    python -m gate_cores_b200.build [--force] [--verbose]
+    python -m gate_cores_b200.build [--force] [--verbose] [--jobs N]
 
-The library links the CUDA runtime statically, so it depends on the driver
-only; the .so sits next to this file, where the binding looks for it.
+Each .cu file compiles to its own object in parallel (the kernels share no
+device symbols across files), then nvcc links the shared library.  The
+library links the CUDA runtime statically, so it depends on the driver only;
+the .so sits next to this file, where the binding looks for it.
 """
 from __future__ import annotations
 
@@ -12,13 +14,16 @@ import glob
 import os
 import shutil
 import subprocess
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
+OBJ = os.path.join(ROOT, "_build", "muse_cores")
 LIB = os.path.join(PKG, "libmuse_cores.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC,-O2,-Wall"]
 
 
 def nvcc() -> str:
@@ -32,26 +37,45 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
+def _headers() -> list[str]:
+    return (glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) +
+            glob.glob(os.path.join(INCLUDE, "*.h")))
+
+
 def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-    deps += glob.glob(os.path.join(INCLUDE, "*.h"))
-    return any(os.path.getmtime(d) > t for d in deps)
+    return any(os.path.getmtime(d) > t for d in sources() + _headers())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
-           "-Xcompiler", "-fPIC,-O2,-Wall", "-shared", "-I", INCLUDE, "-I", CSRC,
-           "-o", tmp, *sources()]
+def _compile(src: str, verbose: bool) -> str:
+    obj = os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
+    newest_dep = max(os.path.getmtime(d) for d in [src] + _headers())
+    if os.path.exists(obj) and os.path.getmtime(obj) >= newest_dep:
+        return obj
+    tmp = obj + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", "-o", tmp, src]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
-        print(" ".join(cmd))
+        print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)
+    os.replace(tmp, obj)
+    return obj
+
+
+def build(force: bool = False, verbose: bool = False, jobs: int | None = None) -> str:
+    if not force and not _stale():
+        return LIB
+    os.makedirs(OBJ, exist_ok=True)
+    if force:
+        for o in glob.glob(os.path.join(OBJ, "*.o")):
+            os.remove(o)
+    srcs = sources()
+    with ThreadPoolExecutor(max_workers=jobs or min(len(srcs), os.cpu_count() or 1)) as ex:
+        objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
+    tmp = LIB + f".tmp{os.getpid()}"
+    subprocess.check_call([nvcc(), *ARCH, "-shared", "-o", tmp, *objs])
     os.replace(tmp, LIB)
     return LIB
 
@@ -60,5 +84,6 @@ if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--jobs", type=int, default=None)
     args = ap.parse_args()
-    print(build(force=args.force, verbose=args.verbose))
+    print(build(force=args.force, verbose=args.verbose, jobs=args.jobs))
