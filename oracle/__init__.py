@@ -80,6 +80,12 @@ def _load():
             lib.muse_oracle_norm_residual_bwd.argtypes = [
                 P, c_int, P, P, i64, i64, P, f32, P, c_int, f32, c_int,
                 P, P, P, P, P, P, P, P, P, P, P, P, P, P]
+            lib.muse_oracle_residual_blend.argtypes = [P, c_int, P, i64, i64, P, P, P, P, P]
+            lib.muse_oracle_residual_gate_coefficients.argtypes = [P, i64, f32, f32, P, P, P]
+            lib.muse_oracle_residual.argtypes = [P, c_int, P, i64, i64, P, f32, f32, P, P, P, P]
+            for name in ("muse_oracle_residual_blend", "muse_oracle_residual_gate_coefficients",
+                         "muse_oracle_residual"):
+                getattr(lib, name).restype = c_int
             lib.muse_oracle_vision_rope_frequencies.argtypes = [i32, i32, i32, f32, P]
             lib.muse_oracle_vision_rope.argtypes = [c_int, P, P, i64, i32, i32, i32, P,
                                                     P, P, P, P, P, P, P, P]
@@ -261,6 +267,50 @@ def norm_residual(stream, branch, theta, gain=None, gain_offset=0.0, input_scale
         _ptr(stream), _dt(branch), _ptr(branch), rows, hidden, _ptr(gain), gain_offset,
         _ptr(theta), int(input_scale), norm_eps, _ptr(out), _ptr(lo), _ptr(hi), _ptr(mag)),
         "norm_residual")
+    return out, lo, hi, mag
+
+
+def residual_blend(stream, branch, theta):
+    """_residual_core without a branch norm, core 5's declared blend:
+    cos(theta) h + sin(theta) branch per channel."""
+    stream = np.ascontiguousarray(stream, dtype=np.float32)
+    branch = _c(branch)
+    theta = np.ascontiguousarray(theta, dtype=np.float32)
+    assert stream.shape == branch.shape
+    hidden = stream.shape[-1]
+    rows = stream.size // hidden
+    out = np.empty_like(stream)
+    lo, hi, mag = _checks(stream.shape)
+    _check(_load().muse_oracle_residual_blend(_ptr(stream), _dt(branch), _ptr(branch), rows, hidden,
+                                              _ptr(theta), _ptr(out), _ptr(lo), _ptr(hi), _ptr(mag)),
+           "residual_blend")
+    return out, lo, hi, mag
+
+
+def residual_gate_coefficients(gate, temperature=0.3, eps=1e-3):
+    """Declared reading of the learned gate: (c, s, theta) in double, with
+    c^2 = max(sigmoid(gate/temperature), eps), s^2 = 1 - c^2, theta = atan2(s, c)."""
+    gate = np.ascontiguousarray(gate, dtype=np.float32)
+    c, s, th = (np.empty(gate.shape, np.float64) for _ in range(3))
+    _check(_load().muse_oracle_residual_gate_coefficients(_ptr(gate), gate.size, temperature, eps,
+                                                          _ptr(c), _ptr(s), _ptr(th)),
+           "residual_gate_coefficients")
+    return c, s, th
+
+
+def residual(stream, branch, gate, temperature=0.3, eps=1e-3):
+    """_residual_core(stream, branch, gate, temperature, eps): c h + s branch."""
+    stream = np.ascontiguousarray(stream, dtype=np.float32)
+    branch = _c(branch)
+    gate = np.ascontiguousarray(gate, dtype=np.float32)
+    assert stream.shape == branch.shape
+    hidden = stream.shape[-1]
+    rows = stream.size // hidden
+    out = np.empty_like(stream)
+    lo, hi, mag = _checks(stream.shape)
+    _check(_load().muse_oracle_residual(_ptr(stream), _dt(branch), _ptr(branch), rows, hidden,
+                                        _ptr(gate), temperature, eps, _ptr(out), _ptr(lo), _ptr(hi),
+                                        _ptr(mag)), "residual")
     return out, lo, hi, mag
 
 

@@ -469,6 +469,85 @@ int muse_oracle_norm_residual(const float* stream, int branch_dtype, const void*
     return 0;
 }
 
+/* -------------------------------------------------- _residual_core (blend) */
+
+/* _residual_core / MuseSparkResidual.forward: the residual stream blended
+ * with the branch as it arrives (no branch norm), under the declared blend of
+ * core 5: out = cos(theta) h + sin(theta) branch per channel, FP32 theta, the
+ * branch read exactly in double (bf16 -> f32 is exact), the stream dtype kept. */
+int muse_oracle_residual_blend(const float* stream, int branch_dtype, const void* branch,
+                               int64_t rows, int64_t hidden, const float* theta, float* out,
+                               double* lo, double* hi, double* mag) {
+    if (!valid_dtype(branch_dtype) || rows < 0 || hidden <= 0) return -1;
+    if (rows && (!stream || !branch || !out || !theta)) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t j = 0; j < hidden; ++j) {
+            const int64_t i = r * hidden + j;
+            const double c = cos((double)theta[j]), s = sin((double)theta[j]);
+            const double h = (double)stream[i], b = load_elem(branch_dtype, branch, i);
+            const double y = c * h + s * b;
+            out[i] = (float)y;
+            put_check(lo, hi, mag, i, y, y, fabs(c * h) + fabs(s * b));
+        }
+    }
+    return 0;
+}
+
+/* The learned gate of _residual_core / MuseSparkResidual (gate [hidden],
+ * temperature, eps) as the blend's two coefficients - the declared reading:
+ * the squared residual coefficient is the sigmoid of gate / temperature,
+ * bounded below by eps ("lower bound on the squared residual coefficient"),
+ * and the branch coefficient keeps the squares summing to one
+ * ("norm-preserving"):
+ *   c^2 = max(sigmoid(gate / temperature), eps),   s^2 = 1 - c^2,
+ * c, s >= 0, so that theta = atan2(s, c) lies in [0, pi/2] and the blend is
+ * core 5's cos(theta) h + sin(theta) b.  1 - max(sigmoid(x), eps) is written
+ * as min(sigmoid(-x), 1 - eps), the same number, so that s keeps its
+ * relative precision when sigmoid(x) is close to 1.  Any of c, s, theta may
+ * be NULL. */
+int muse_oracle_residual_gate_coefficients(const float* gate, int64_t hidden, float temperature,
+                                           float eps, double* c, double* s, double* theta) {
+    if (!gate || hidden <= 0 || !(temperature > 0.0f) || !(eps >= 0.0f && eps <= 1.0f)) return -1;
+    for (int64_t j = 0; j < hidden; ++j) {
+        const double x = (double)gate[j] / (double)temperature;
+        const double c2 = fmax(1.0 / (1.0 + exp(-x)), (double)eps);
+        const double s2 = fmin(1.0 / (1.0 + exp(x)), 1.0 - (double)eps);
+        const double cj = sqrt(c2), sj = sqrt(s2);
+        if (c) c[j] = cj;
+        if (s) s[j] = sj;
+        if (theta) theta[j] = atan2(sj, cj);
+    }
+    return 0;
+}
+
+/* _residual_core(stream, branch, gate, temperature, eps) under the reading
+ * above: out = c h + s branch per channel. */
+int muse_oracle_residual(const float* stream, int branch_dtype, const void* branch, int64_t rows,
+                         int64_t hidden, const float* gate, float temperature, float eps, float* out,
+                         double* lo, double* hi, double* mag) {
+    if (!valid_dtype(branch_dtype) || rows < 0 || hidden <= 0 || !gate) return -1;
+    if (rows && (!stream || !branch || !out)) return -1;
+    double* c = (double*)malloc(sizeof(double) * (size_t)hidden);
+    double* s = (double*)malloc(sizeof(double) * (size_t)hidden);
+    if (!c || !s || muse_oracle_residual_gate_coefficients(gate, hidden, temperature, eps, c, s, NULL)) {
+        free(c);
+        free(s);
+        return -1;
+    }
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t j = 0; j < hidden; ++j) {
+            const int64_t i = r * hidden + j;
+            const double h = (double)stream[i], b = load_elem(branch_dtype, branch, i);
+            const double y = c[j] * h + s[j] * b;
+            out[i] = (float)y;
+            put_check(lo, hi, mag, i, y, y, fabs(c[j] * h) + fabs(s[j] * b));
+        }
+    }
+    free(c);
+    free(s);
+    return 0;
+}
+
 /* ================================================================ backward
  *
  * The cores run under autograd (the page's _checkpoint_recomputed_math keeps

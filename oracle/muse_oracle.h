@@ -132,6 +132,22 @@ int muse_oracle_norm_residual(const float* stream, int branch_dtype, const void*
                               float norm_eps, float* out, double* lo, double* hi,
                               double* mag);
 
+/* _residual_core / MuseSparkResidual without a branch norm, with core 5's
+ * declared blend: h' = f32(cos(theta) h + sin(theta) branch), per channel. */
+int muse_oracle_residual_blend(const float* stream, int branch_dtype, const void* branch,
+                               int64_t rows, int64_t hidden, const float* theta, float* out,
+                               double* lo, double* hi, double* mag);
+
+/* The declared reading of the learned gate (gate, temperature, eps):
+ * c^2 = max(sigmoid(gate/temperature), eps), s^2 = 1 - c^2, theta = atan2(s, c). */
+int muse_oracle_residual_gate_coefficients(const float* gate, int64_t hidden, float temperature,
+                                           float eps, double* c, double* s, double* theta);
+
+/* _residual_core(stream, branch, gate, temperature, eps): h' = c h + s branch. */
+int muse_oracle_residual(const float* stream, int branch_dtype, const void* branch, int64_t rows,
+                         int64_t hidden, const float* gate, float temperature, float eps, float* out,
+                         double* lo, double* hi, double* mag);
+
 /* ---------------------------------------------------------------- backward
  *
  * Gradients of the five cores (the cores run under autograd): the derivative

@@ -112,6 +112,14 @@ def test_golden_closed_forms(case):
             _f32(case["stream"]), _f32(case["branch"]), _f32(case["theta"]), _f32(case["gain"]),
             case["gain_offset"], case["input_scale"], eps)
         got = {"expect": lo.ravel()}
+    elif core == "residual_blend":
+        out, lo, hi, mag = oracle.residual_blend(_f32(case["stream"]), _f32(case["branch"]),
+                                                 _f32(case["theta"]))
+        got = {"expect": lo.ravel()}
+    elif core == "residual":
+        out, lo, hi, mag = oracle.residual(_f32(case["stream"]), _f32(case["branch"]), _f32(case["gate"]),
+                                           case["temperature"], float(np.float32(case["eps"])))
+        got = {"expect": lo.ravel()}
     else:
         raise AssertionError(core)
     for key, vals in got.items():
