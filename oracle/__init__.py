@@ -83,8 +83,11 @@ def _load():
             lib.muse_oracle_residual_blend.argtypes = [P, c_int, P, i64, i64, P, P, P, P, P]
             lib.muse_oracle_residual_gate_coefficients.argtypes = [P, i64, f32, f32, P, P, P]
             lib.muse_oracle_residual.argtypes = [P, c_int, P, i64, i64, P, f32, f32, P, P, P, P]
+            lib.muse_oracle_residual_blend_bwd.argtypes = [P, c_int, P, P, i64, i64, P] + [P] * 11
+            lib.muse_oracle_residual_bwd.argtypes = [P, c_int, P, P, i64, i64, P, f32, f32] + [P] * 11
             for name in ("muse_oracle_residual_blend", "muse_oracle_residual_gate_coefficients",
-                         "muse_oracle_residual"):
+                         "muse_oracle_residual", "muse_oracle_residual_blend_bwd",
+                         "muse_oracle_residual_bwd"):
                 getattr(lib, name).restype = c_int
             lib.muse_oracle_vision_rope_frequencies.argtypes = [i32, i32, i32, f32, P]
             lib.muse_oracle_vision_rope.argtypes = [c_int, P, P, i64, i32, i32, i32, P,
@@ -312,6 +315,37 @@ def residual(stream, branch, gate, temperature=0.3, eps=1e-3):
                                         _ptr(gate), temperature, eps, _ptr(out), _ptr(lo), _ptr(hi),
                                         _ptr(mag)), "residual")
     return out, lo, hi, mag
+
+
+def _residual_bwd_call(fn, what, stream, branch, dy, *params):
+    stream = np.ascontiguousarray(stream, dtype=np.float32)
+    dy = np.ascontiguousarray(dy, dtype=np.float32)
+    branch = _c(branch)
+    assert stream.shape == branch.shape == dy.shape
+    hidden = stream.shape[-1]
+    rows = stream.size // hidden
+    ds = np.empty_like(stream)
+    db = np.empty_like(branch)
+    sl, sh, sm = _checks(stream.shape)
+    bl, bh, bm = _checks(stream.shape)
+    pl, ph, pm = _checks((hidden,))
+    _check(fn(_ptr(stream), _dt(branch), _ptr(branch), _ptr(dy), rows, hidden, *params, _ptr(ds), _ptr(sl),
+              _ptr(sh), _ptr(sm), _ptr(db), _ptr(bl), _ptr(bh), _ptr(bm), _ptr(pl), _ptr(ph), _ptr(pm)), what)
+    return (ds, sl, sh, sm), (db, bl, bh, bm), (pl, ph, pm)
+
+
+def residual_blend_bwd(stream, branch, dy, theta):
+    """Backward of the angle form: (dstream, dbranch, dtheta)."""
+    theta = np.ascontiguousarray(theta, dtype=np.float32)
+    return _residual_bwd_call(_load().muse_oracle_residual_blend_bwd, "residual_blend_bwd", stream, branch,
+                              dy, _ptr(theta))
+
+
+def residual_bwd(stream, branch, dy, gate, temperature=0.3, eps=1e-3):
+    """Backward of the gate form: (dstream, dbranch, dgate)."""
+    gate = np.ascontiguousarray(gate, dtype=np.float32)
+    return _residual_bwd_call(_load().muse_oracle_residual_bwd, "residual_bwd", stream, branch, dy,
+                              _ptr(gate), temperature, eps)
 
 
 # ------------------------------------------------------------------ backward

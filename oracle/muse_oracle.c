@@ -846,6 +846,96 @@ int muse_oracle_norm_residual_bwd(const float* stream, int branch_dtype, const v
     return 0;
 }
 
+/* Backward of _residual_core, both forms: out = c h + s b per channel (b the
+ * branch read in FP32).  Given dy = dL/dout (FP32):
+ *   dstream = c dy                          (FP32);
+ *   dbranch = cast_branch(s dy)             (the forward upcast the branch to
+ *                                            FP32; the gradient of that cast
+ *                                            is rounded back);
+ *   angle form: dtheta_j = sum over rows of dy (-s h + c b),
+ *               c = cos(theta_j), s = sin(theta_j);
+ *   gate form:  dgate_j  = sum over rows of dy (c' h + s' b), with
+ *               c' = dc/dgate = c s^2 / (2 temperature),
+ *               s' = ds/dgate = -s c^2 / (2 temperature)
+ *               where sigmoid(gate / temperature) >= eps (c^2 = sigmoid there),
+ *               and c' = s' = 0 where the bound holds c (clamp_min's rule: the
+ *               gradient passes at equality).
+ * Parameter gradients come as (lo, hi, mag): the exact sum twice and the sum
+ * of the magnitudes of its terms. */
+static int residual_bwd(const float* stream, int branch_dtype, const void* branch, const float* dy,
+                        int64_t rows, int64_t hidden, const double* c, const double* s,
+                        const double* dc, const double* ds, float* dstream, double* ds_lo,
+                        double* ds_hi, double* ds_mag, void* dbranch, double* db_lo, double* db_hi,
+                        double* db_mag, double* dp_lo, double* dp_hi, double* dp_mag) {
+    if (rows && (!stream || !branch || !dy || !dstream || !dbranch)) return -1;
+    zero_n(dp_lo, hidden);
+    zero_n(dp_hi, hidden);
+    zero_n(dp_mag, hidden);
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t j = 0; j < hidden; ++j) {
+            const int64_t i = r * hidden + j;
+            const double g = (double)dy[i], h = (double)stream[i];
+            const double b = load_elem(branch_dtype, branch, i);
+            dstream[i] = (float)(c[j] * g);
+            put_check(ds_lo, ds_hi, ds_mag, i, c[j] * g, c[j] * g, fabs(c[j] * g));
+            store_elem(branch_dtype, dbranch, i, s[j] * g);
+            put_check(db_lo, db_hi, db_mag, i, s[j] * g, s[j] * g, fabs(s[j] * g));
+            const double t = g * (dc[j] * h + ds[j] * b);
+            acc_param(dp_lo, dp_hi, dp_mag, j, iv_exact(t), fabs(g) * (fabs(dc[j] * h) + fabs(ds[j] * b)));
+        }
+    }
+    return 0;
+}
+
+int muse_oracle_residual_blend_bwd(const float* stream, int branch_dtype, const void* branch,
+                                   const float* dy, int64_t rows, int64_t hidden, const float* theta,
+                                   float* dstream, double* ds_lo, double* ds_hi, double* ds_mag,
+                                   void* dbranch, double* db_lo, double* db_hi, double* db_mag,
+                                   double* dtheta_lo, double* dtheta_hi, double* dtheta_mag) {
+    if (!valid_dtype(branch_dtype) || rows < 0 || hidden <= 0 || !theta) return -1;
+    double* cs = (double*)malloc(sizeof(double) * (size_t)hidden * 4);
+    if (!cs) return -1;
+    double *c = cs, *s = cs + hidden, *dc = cs + 2 * hidden, *ds = cs + 3 * hidden;
+    for (int64_t j = 0; j < hidden; ++j) {
+        c[j] = cos((double)theta[j]);
+        s[j] = sin((double)theta[j]);
+        dc[j] = -s[j]; /* d cos / d theta */
+        ds[j] = c[j];  /* d sin / d theta */
+    }
+    const int rc = residual_bwd(stream, branch_dtype, branch, dy, rows, hidden, c, s, dc, ds, dstream,
+                                ds_lo, ds_hi, ds_mag, dbranch, db_lo, db_hi, db_mag, dtheta_lo,
+                                dtheta_hi, dtheta_mag);
+    free(cs);
+    return rc;
+}
+
+int muse_oracle_residual_bwd(const float* stream, int branch_dtype, const void* branch,
+                             const float* dy, int64_t rows, int64_t hidden, const float* gate,
+                             float temperature, float eps, float* dstream, double* ds_lo,
+                             double* ds_hi, double* ds_mag, void* dbranch, double* db_lo,
+                             double* db_hi, double* db_mag, double* dgate_lo, double* dgate_hi,
+                             double* dgate_mag) {
+    if (!valid_dtype(branch_dtype) || rows < 0 || hidden <= 0 || !gate) return -1;
+    double* cs = (double*)malloc(sizeof(double) * (size_t)hidden * 4);
+    if (!cs) return -1;
+    double *c = cs, *s = cs + hidden, *dc = cs + 2 * hidden, *ds = cs + 3 * hidden;
+    if (muse_oracle_residual_gate_coefficients(gate, hidden, temperature, eps, c, s, NULL)) {
+        free(cs);
+        return -1;
+    }
+    for (int64_t j = 0; j < hidden; ++j) {
+        const double x = (double)gate[j] / (double)temperature;
+        const int free_ = 1.0 / (1.0 + exp(-x)) >= (double)eps;
+        dc[j] = free_ ? c[j] * s[j] * s[j] / (2.0 * (double)temperature) : 0.0;
+        ds[j] = free_ ? -s[j] * c[j] * c[j] / (2.0 * (double)temperature) : 0.0;
+    }
+    const int rc = residual_bwd(stream, branch_dtype, branch, dy, rows, hidden, c, s, dc, ds, dstream,
+                                ds_lo, ds_hi, ds_mag, dbranch, db_lo, db_hi, db_mag, dgate_lo,
+                                dgate_hi, dgate_mag);
+    free(cs);
+    return rc;
+}
+
 /* Gradient of one pair's rotated-in values under the v2 rotation (bf16):
  * the forward's y0 = cast(cast(a C) - cast(b S)), y1 = cast(cast(a S) +
  * cast(b C)) with C = cast(c), S = cast(s).  Backward through those bf16

@@ -205,6 +205,21 @@ int muse_oracle_norm_residual_bwd(const float* stream, int branch_dtype, const v
                                   double* dgain_lo, double* dgain_hi, double* dgain_mag,
                                   double* dtheta_lo, double* dtheta_hi, double* dtheta_mag);
 
+/* Backward of _residual_core: dstream = c dy (FP32), dbranch = cast_branch(s dy),
+ * and the angle (dtheta) or gate (dgate) gradient as a sum over rows, returned as
+ * (lo, hi, mag) double triples. */
+int muse_oracle_residual_blend_bwd(const float* stream, int branch_dtype, const void* branch,
+                                   const float* dy, int64_t rows, int64_t hidden, const float* theta,
+                                   float* dstream, double* ds_lo, double* ds_hi, double* ds_mag,
+                                   void* dbranch, double* db_lo, double* db_hi, double* db_mag,
+                                   double* dtheta_lo, double* dtheta_hi, double* dtheta_mag);
+int muse_oracle_residual_bwd(const float* stream, int branch_dtype, const void* branch,
+                             const float* dy, int64_t rows, int64_t hidden, const float* gate,
+                             float temperature, float eps, float* dstream, double* ds_lo,
+                             double* ds_hi, double* ds_mag, void* dbranch, double* db_lo,
+                             double* db_hi, double* db_mag, double* dgate_lo, double* dgate_hi,
+                             double* dgate_mag);
+
 /* Vision 2-D RoPE (page "...muse_spark.vision": _rope_frequencies,
  * _apply_vision_rope).  Frequencies of one row-major grid, out
  * [grid_h * grid_w, head_dim / 2, 2] = (cos, sin) per pair: the first
