@@ -13,9 +13,13 @@ from .cores import (  # noqa: F401
     norm_residual,
     output_norm_gate,
     qk_norm_rope,
+    residual,
+    residual_blend,
+    residual_gate_angles,
     rms_norm,
     stream_copy,
 )
 
 __all__ = ["rms_norm", "input_scale_norm", "qk_norm_rope", "output_norm_gate", "norm_residual",
-           "stream_copy", "MuseError", "load_library"]
+           "residual_blend", "residual", "residual_gate_angles", "stream_copy", "MuseError",
+           "load_library"]

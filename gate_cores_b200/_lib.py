@@ -33,7 +33,9 @@ EXPORTS = (
     "muse_input_scale_norm_backward", "muse_norm_residual_backward",
     "muse_output_norm_gate_backward", "muse_qk_norm_rope_backward",
     "muse_rms_norm_backward_noalloc", "muse_norm_residual_rms_norm", "muse_rms_norm_grouped",
-    "muse_vision_rope", "muse_vision_rope_frequencies",
+    "muse_vision_rope", "muse_vision_rope_frequencies", "muse_rms_norm_stall_probe",
+    "muse_residual_blend", "muse_residual", "muse_residual_gate_angles",
+    "muse_residual_backward_workspace_bytes", "muse_residual_blend_backward", "muse_residual_backward",
 )
 
 
@@ -70,6 +72,14 @@ def load() -> ctypes.CDLL:
         row = [P, P, c_int, i64, i64, i64, i64, P, f32, f32, P]
         lib.muse_rms_norm.argtypes = row
         lib.muse_input_scale_norm.argtypes = row
+        lib.muse_rms_norm_stall_probe.argtypes = row[:-1] + [ctypes.c_uint32, i64, P]
+        lib.muse_residual_blend.argtypes = [P, P, P, c_int, i64, i64, P, P]
+        lib.muse_residual.argtypes = [P, P, P, c_int, i64, i64, P, f32, f32, P]
+        lib.muse_residual_gate_angles.argtypes = [P, P, i64, f32, f32, P]
+        lib.muse_residual_backward_workspace_bytes.argtypes = [i64, i64]
+        lib.muse_residual_blend_backward.argtypes = [P, P, P, P, P, c_int, i64, i64, P, P, P, ctypes.c_size_t, P]
+        lib.muse_residual_backward.argtypes = [P, P, P, P, P, c_int, i64, i64, P, f32, f32, P, P,
+                                               ctypes.c_size_t, P]
         lib.muse_qk_norm_rope.argtypes = [P, P, P, P, c_int, c_int, i64, i64, P, i32, i64, P,
                                           i32, i32, i32, i64, i64, i64, i64, f32, f32, c_int,
                                           c_int, f32, P]
@@ -99,6 +109,7 @@ def load() -> ctypes.CDLL:
         for name in EXPORTS[3:]:
             getattr(lib, name).restype = c_int
         lib.muse_norm_backward_workspace_bytes.restype = sz
+        lib.muse_residual_backward_workspace_bytes.restype = sz
         _lib = lib
         return lib
 
@@ -236,6 +247,42 @@ def muse_vision_rope(q, k, q_out, k_out, dtype, tokens, hq, hk, head_dim, q_tok_
                      q_out_tok_stride, k_out_tok_stride, freqs, stream) -> None:
     _call("muse_vision_rope", q, k, q_out, k_out, dtype, tokens, hq, hk, head_dim, q_tok_stride,
           k_tok_stride, q_out_tok_stride, k_out_tok_stride, freqs, stream)
+
+
+def muse_rms_norm_stall_probe(x, y, dtype, rows, hidden, x_row_stride, y_row_stride, gain, gain_offset,
+                              eps, spin_limit, stall_row, stream) -> None:
+    _call("muse_rms_norm_stall_probe", x, y, dtype, rows, hidden, x_row_stride, y_row_stride, gain,
+          gain_offset, eps, spin_limit, stall_row, stream)
+
+
+def muse_residual_blend(stream_in, branch, stream_out, branch_dtype, rows, hidden, theta, stream) -> None:
+    _call("muse_residual_blend", stream_in, branch, stream_out, branch_dtype, rows, hidden, theta, stream)
+
+
+def muse_residual(stream_in, branch, stream_out, branch_dtype, rows, hidden, gate, temperature, eps,
+                  stream) -> None:
+    _call("muse_residual", stream_in, branch, stream_out, branch_dtype, rows, hidden, gate, temperature, eps,
+          stream)
+
+
+def muse_residual_backward_workspace_bytes(rows, hidden) -> int:
+    return load().muse_residual_backward_workspace_bytes(rows, hidden)
+
+
+def muse_residual_blend_backward(stream_in, branch, dstream_out, dstream_in, dbranch, branch_dtype, rows, hidden,
+                                 theta, dtheta, workspace, workspace_bytes, stream) -> None:
+    _call("muse_residual_blend_backward", stream_in, branch, dstream_out, dstream_in, dbranch, branch_dtype, rows,
+          hidden, theta, dtheta, workspace, workspace_bytes, stream)
+
+
+def muse_residual_backward(stream_in, branch, dstream_out, dstream_in, dbranch, branch_dtype, rows, hidden, gate,
+                           temperature, eps, dgate, workspace, workspace_bytes, stream) -> None:
+    _call("muse_residual_backward", stream_in, branch, dstream_out, dstream_in, dbranch, branch_dtype, rows, hidden,
+          gate, temperature, eps, dgate, workspace, workspace_bytes, stream)
+
+
+def muse_residual_gate_angles(gate, theta, hidden, temperature, eps, stream) -> None:
+    _call("muse_residual_gate_angles", gate, theta, hidden, temperature, eps, stream)
 
 
 def muse_vision_rope_frequencies(out, head_dim, grid_h, grid_w, theta, stream) -> None:

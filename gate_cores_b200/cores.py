@@ -187,6 +187,55 @@ def norm_residual(stream_in: torch.Tensor, branch: torch.Tensor, theta: torch.Te
     return h_out
 
 
+def _residual_args(stream_in, branch, p, what):
+    _cuda(stream_in, branch, p)
+    if stream_in.dtype != torch.float32 or p.dtype != torch.float32:
+        raise TypeError(f"stream and {what} must be float32")
+    if branch.shape != stream_in.shape:
+        raise ValueError("branch must match the stream's shape")
+    if not (stream_in.is_contiguous() and branch.is_contiguous()):
+        raise ValueError("stream and branch must be contiguous")
+    hidden = stream_in.shape[-1]
+    return hidden, stream_in.numel() // hidden
+
+
+def residual_blend(stream_in: torch.Tensor, branch: torch.Tensor, theta: torch.Tensor,
+                   out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """_residual_core without a branch norm, in core 5's angle form:
+    cos(theta) * stream + sin(theta) * branch per channel (theta FP32 [H])."""
+    hidden, rows = _residual_args(stream_in, branch, theta, "theta")
+    _cuda(out)
+    h_out = _out_like(stream_in, out)
+    _lib.muse_residual_blend(stream_in.data_ptr(), branch.data_ptr(), h_out.data_ptr(), _dtype(branch), rows,
+                             hidden, theta.contiguous().data_ptr(), _stream(stream))
+    return h_out
+
+
+def residual(stream_in: torch.Tensor, branch: torch.Tensor, gate: torch.Tensor, temperature: float = 0.3,
+             eps: float = 1e-3, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """_residual_core(stream, branch, gate, temperature, eps): c * stream +
+    s * branch per channel with c^2 = max(sigmoid(gate / temperature), eps),
+    s^2 = 1 - c^2 (gate FP32 [H])."""
+    hidden, rows = _residual_args(stream_in, branch, gate, "gate")
+    _cuda(out)
+    h_out = _out_like(stream_in, out)
+    _lib.muse_residual(stream_in.data_ptr(), branch.data_ptr(), h_out.data_ptr(), _dtype(branch), rows, hidden,
+                       gate.contiguous().data_ptr(), temperature, eps, _stream(stream))
+    return h_out
+
+
+def residual_gate_angles(gate: torch.Tensor, temperature: float = 0.3, eps: float = 1e-3,
+                         out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Blend angle per channel from the learned gate: atan2(s, c) (FP32 [H])."""
+    _cuda(gate, out)
+    if gate.dtype != torch.float32 or gate.dim() != 1:
+        raise TypeError("gate must be a float32 vector")
+    theta = _out_like(gate, out)
+    _lib.muse_residual_gate_angles(gate.contiguous().data_ptr(), theta.data_ptr(), gate.numel(), temperature,
+                                   eps, _stream(stream))
+    return theta
+
+
 def rms_norm_grouped(x: torch.Tensor, gains: torch.Tensor, group_offsets: torch.Tensor,
                      gain_offset: float = 0.0, eps: float = 1e-6, out: torch.Tensor | None = None,
                      stream=None) -> torch.Tensor:
@@ -352,6 +401,35 @@ def norm_residual_backward(stream_in, branch, dstream_out, theta, gain=None,
         theta.contiguous().data_ptr(), input_scale, norm_eps, _ptr(dgain), _ptr(dtheta), _ptr(ws),
         0 if ws is None else ws.numel(), _stream(stream))
     return dsi, db, dgain, dtheta
+
+
+def residual_backward(stream_in, branch, dstream_out, theta=None, gate=None, temperature: float = 0.3,
+                      eps: float = 1e-3, want_param: bool = True, workspace=None, stream=None):
+    """Backward of _residual_core: the angle form (theta given) or the gate form
+    (gate given).  Returns (dstream_in, dbranch, dtheta or dgate)."""
+    if (theta is None) == (gate is None):
+        raise ValueError("give exactly one of theta and gate")
+    p = theta if gate is None else gate
+    hidden, rows = _residual_args(stream_in, branch, p, "theta / gate")
+    _cuda(dstream_out)
+    if dstream_out.dtype != torch.float32 or dstream_out.shape != stream_in.shape or not dstream_out.is_contiguous():
+        raise ValueError("dstream_out must be float32, contiguous and shaped like the stream")
+    dsi = torch.empty_like(stream_in)
+    db = torch.empty_like(branch)
+    dp = ws = None
+    if want_param:
+        dp = torch.empty(hidden, dtype=torch.float32, device=stream_in.device)
+        need = _lib.muse_residual_backward_workspace_bytes(rows, hidden)
+        ws = workspace if workspace is not None else torch.empty(max(need, 16), dtype=torch.uint8,
+                                                                 device=stream_in.device)
+    args = (stream_in.data_ptr(), branch.data_ptr(), dstream_out.data_ptr(), dsi.data_ptr(), db.data_ptr(),
+            _dtype(branch), rows, hidden, p.contiguous().data_ptr())
+    tail = (_ptr(dp), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    if gate is None:
+        _lib.muse_residual_blend_backward(*args, *tail)
+    else:
+        _lib.muse_residual_backward(*args, temperature, eps, *tail)
+    return dsi, db, dp
 
 
 def output_norm_gate_backward(o, gate, dy, norm_group=None, eps: float = 1e-6, stream=None):

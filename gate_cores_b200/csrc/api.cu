@@ -84,9 +84,12 @@ bool bad_alias(const Span& out, const Span& other, bool may_coincide) {
     return overlap(out, other);
 }
 
+// probe: the bounded-wait probe of muse_rms_norm_stall_probe (spin_limit
+// polls per wait; the stage of row stall_row is never signalled).
 muse_status row_entry(muse::RowOp op, const void* x, void* y, muse_dtype dtype, int64_t rows,
                       int64_t hidden, int64_t xs, int64_t ys, const float* gain,
-                      float gain_offset, float eps, cudaStream_t stream, const char* name) {
+                      float gain_offset, float eps, cudaStream_t stream, const char* name,
+                      bool probe = false, uint32_t spin_limit = 0, int64_t stall_row = 0) {
     if (!valid_dtype(dtype)) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, (int)dtype);
     if (rows < 0 || hidden <= 0)
         return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: rows=%lld hidden=%lld", name, (long long)rows, (long long)hidden);
@@ -102,6 +105,14 @@ muse_status row_entry(muse::RowOp op, const void* x, void* y, muse_dtype dtype, 
     if (gain && !aligned(gain, 16)) return fail(MUSE_ERR_UNSUPPORTED, "%s: gain not 16-byte aligned", name);
     if (hidden * es > MUSE_MAX_ROW_BYTES)
         return fail(MUSE_ERR_UNSUPPORTED, "%s: row of %lld bytes exceeds %d", name, (long long)(hidden * es), MUSE_MAX_ROW_BYTES);
+    if (probe) {
+        // the probe needs the bulk-copy pipeline, which rows up to 1024 16-byte vectors take
+        if (hidden * es > 16384)
+            return fail(MUSE_ERR_UNSUPPORTED, "%s: probe rows are limited to 16384 bytes", name);
+        if (spin_limit < 1 || spin_limit > (1u << 24) || stall_row < 0 || stall_row >= rows)
+            return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: spin_limit in [1, 2^24] and stall_row in [0, rows) required",
+                        name);
+    }
     const Span sx = span(x, rows, hidden, xs, es), sy = span(y, rows, hidden, ys, es);
     if (bad_alias(sy, sx, true) || (gain && bad_alias(sy, span(gain, 1, hidden, hidden, 4), false)))
         return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: output partially overlaps an input", name);
@@ -115,6 +126,11 @@ muse_status row_entry(muse::RowOp op, const void* x, void* y, muse_dtype dtype, 
     a.width = (int32_t)hidden;
     a.gain_offset = gain_offset;
     a.eps = eps;
+    if (probe) {
+        a.spin_limit = spin_limit;
+        a.probe_stall = 1;
+        a.stall_row = stall_row;
+    }
     return from_cuda(muse::launch_row(dtype, op, a, stream), name);
 }
 
@@ -136,11 +152,15 @@ bool any_overlap(const Span& a, std::initializer_list<Span> others) {
     return false;
 }
 
+// noalloc: the gain partials go to the library's fixed device array instead
+// of the caller's workspace (ws / ws_bytes ignored); its size is checked
+// against the grid this launch will use, and its address is looked up only
+// after every argument check has passed.
 muse_status row_bwd_entry(bool input_scale, const void* x, const void* dy, void* dx,
                           muse_dtype dtype, int64_t rows, int64_t hidden, int64_t xs,
                           int64_t dys, int64_t dxs, const float* gain, float gain_offset,
                           float eps, float* dgain, void* ws, size_t ws_bytes, cudaStream_t stream,
-                          const char* name) {
+                          const char* name, bool noalloc = false) {
     if (!valid_dtype(dtype)) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, (int)dtype);
     if (rows < 0 || hidden <= 0)
         return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: rows=%lld hidden=%lld", name, (long long)rows, (long long)hidden);
@@ -162,14 +182,18 @@ muse_status row_bwd_entry(bool input_scale, const void* x, const void* dy, void*
         return fail(MUSE_ERR_UNSUPPORTED, "%s: gain / dgain not 16-byte aligned", name);
     if (hidden / vec_elems(dtype) > muse::kBwdMaxVectors)
         return fail(MUSE_ERR_UNSUPPORTED, "%s: rows of more than %d 16-byte vectors", name, muse::kBwdMaxVectors);
-    // cores 1 and 2 use the gain half of the workspace only
-    muse_status st = bwd_workspace_check(name, muse::row_bwd_gain_scratch_bytes(rows, (int32_t)hidden),
-                                         ws, ws_bytes, dgain != nullptr);
-    if (st != MUSE_OK) return st;
+    const muse::BwdOp op = input_scale ? muse::BwdOp::kInputScale : muse::BwdOp::kRms;
+    if (noalloc) ws = nullptr, ws_bytes = 0;
+    if (!noalloc) {
+        // cores 1 and 2 use the gain half of the workspace only
+        muse_status st = bwd_workspace_check(name, muse::row_bwd_gain_scratch_bytes(rows, (int32_t)hidden),
+                                             ws, ws_bytes, dgain != nullptr);
+        if (st != MUSE_OK) return st;
+    }
     const Span sx = span(x, rows, hidden, xs, es), sdy = span(dy, rows, hidden, dys, es);
     const Span sdx = span(dx, rows, hidden, dxs, es);
     const Span sg = span(gain, gain ? 1 : 0, hidden, hidden, 4), sdg = span(dgain, dgain ? 1 : 0, hidden, hidden, 4);
-    const Span sws = span(ws, dgain ? 1 : 0, (int64_t)ws_bytes, (int64_t)ws_bytes, 1);
+    const Span sws = span(ws, (dgain && ws) ? 1 : 0, (int64_t)ws_bytes, (int64_t)ws_bytes, 1);
     if (bad_alias(sdx, sx, true) || bad_alias(sdx, sdy, true) || any_overlap(sdx, {sg, sdg, sws}) ||
         any_overlap(sdg, {sx, sdy, sg, sws}) || any_overlap(sws, {sx, sdy, sg}))
         return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: an output or the workspace overlaps another tensor", name);
@@ -186,7 +210,21 @@ muse_status row_bwd_entry(bool input_scale, const void* x, const void* dy, void*
     a.width = (int32_t)hidden;
     a.gain_offset = gain_offset;
     a.eps = eps;
-    const muse::BwdOp op = input_scale ? muse::BwdOp::kInputScale : muse::BwdOp::kRms;
+    if (noalloc && dgain) {
+        // the partials of the grid this launch uses: one row of hidden floats per CTA
+        int64_t grid = 0;
+        muse_status st = from_cuda(muse::row_bwd_launch_grid(dtype, op, a, &grid), name);
+        if (st != MUSE_OK) return st;
+        const size_t need = (size_t)grid * (size_t)hidden * sizeof(float);
+        if (need > muse::kNoAllocScratchBytes)
+            return fail(MUSE_ERR_UNSUPPORTED, "%s: gain partials of %lld CTAs need %zu bytes, the fixed scratch holds %zu",
+                        name, (long long)grid, need, muse::kNoAllocScratchBytes);
+        void* scratch = nullptr;
+        st = from_cuda(muse::noalloc_scratch(&scratch), name);
+        if (st != MUSE_OK) return st;
+        // the library's own array cannot overlap the caller's tensors
+        a.part_gain = static_cast<float*>(scratch);
+    }
     return from_cuda(muse::launch_row_bwd(dtype, op, a, dgain, nullptr, stream), name);
 }
 
@@ -249,6 +287,15 @@ muse_status muse_rms_norm(const void* x, void* y, muse_dtype dtype, int64_t rows
                           float gain_offset, float eps, cudaStream_t stream) {
     return row_entry(muse::RowOp::kRms, x, y, dtype, rows, hidden, x_row_stride, y_row_stride,
                      gain, gain_offset, eps, stream, "muse_rms_norm");
+}
+
+muse_status muse_rms_norm_stall_probe(const void* x, void* y, muse_dtype dtype, int64_t rows,
+                                      int64_t hidden, int64_t x_row_stride, int64_t y_row_stride,
+                                      const float* gain, float gain_offset, float eps,
+                                      uint32_t spin_limit, int64_t stall_row, cudaStream_t stream) {
+    return row_entry(muse::RowOp::kRms, x, y, dtype, rows, hidden, x_row_stride, y_row_stride,
+                     gain, gain_offset, eps, stream, "muse_rms_norm_stall_probe", true, spin_limit,
+                     stall_row);
 }
 
 muse_status muse_input_scale_norm(const void* x, void* y, muse_dtype dtype, int64_t rows,
@@ -339,7 +386,6 @@ muse_status muse_qk_norm_rope(const void* q, const void* k, void* q_out, void* k
     a.hq = hq;
     a.hkv = hkv;
     a.head_dim = head_dim;
-    a.split = 1;
     a.pos_mode = positions ? 0 : (layout == MUSE_LAYOUT_BSHD ? 1 : 2);
     a.eps = eps;
     a.query_scale = query_scale;
@@ -435,6 +481,192 @@ muse_status muse_norm_residual(const float* stream_in, const void* branch, float
     return from_cuda(muse::launch_row(branch_dtype, op, a, stream), name);
 }
 
+}  // extern "C"
+
+namespace {
+
+// Shared checks of the two _residual_core entry points; p is theta or the gate.
+muse_status residual_entry(const float* stream_in, const void* branch, float* stream_out,
+                           muse_dtype branch_dtype, int64_t rows, int64_t hidden, const float* p,
+                           bool gate, float temperature, float eps, cudaStream_t stream, const char* name) {
+    if (!valid_dtype(branch_dtype)) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, (int)branch_dtype);
+    if (rows < 0 || hidden <= 0)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: rows=%lld hidden=%lld", name, (long long)rows, (long long)hidden);
+    if (gate && !(finite(temperature) && temperature > 0.0f && finite(eps) && eps >= 0.0f && eps <= 1.0f))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: temperature must be finite and > 0, eps in [0, 1]", name);
+    if (rows == 0) return MUSE_OK;
+    if (!stream_in || !branch || !stream_out || !p)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null stream_in/branch/stream_out/%s", name, gate ? "gate" : "theta");
+    const int64_t es = elem_size(branch_dtype);
+    if (!aligned(stream_in, 16) || !aligned(stream_out, 16) || !aligned(branch, 16) || !aligned(p, 16) ||
+        (hidden * es) % 16)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: pointers and row widths must be 16-byte multiples", name);
+    if (hidden / vec_elems(branch_dtype) > (int64_t)65535 * 256)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: rows of more than %d 16-byte vectors", name, 65535 * 256);
+    const Span sin_ = span(stream_in, rows, hidden, hidden, 4), sout = span(stream_out, rows, hidden, hidden, 4);
+    const Span sb = span(branch, rows, hidden, hidden, es), sp = span(p, 1, hidden, hidden, 4);
+    if (bad_alias(sout, sin_, true) || bad_alias(sout, sb, false) || bad_alias(sout, sp, false))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: output partially overlaps an input", name);
+    muse::ResidualArgs a{};
+    a.stream_in = stream_in;
+    a.branch = branch;
+    a.stream_out = stream_out;
+    a.theta = gate ? nullptr : p;
+    a.gate = gate ? p : nullptr;
+    a.rows = rows;
+    a.width = hidden;
+    a.temperature = temperature;
+    a.eps = eps;
+    return from_cuda(muse::launch_residual_blend(branch_dtype, gate, a, stream), name);
+}
+
+}  // namespace
+
+extern "C" {
+
+muse_status muse_residual_blend(const float* stream_in, const void* branch, float* stream_out,
+                                muse_dtype branch_dtype, int64_t rows, int64_t hidden, const float* theta,
+                                cudaStream_t stream) {
+    return residual_entry(stream_in, branch, stream_out, branch_dtype, rows, hidden, theta, false, 1.0f, 0.0f,
+                          stream, "muse_residual_blend");
+}
+
+muse_status muse_residual(const float* stream_in, const void* branch, float* stream_out, muse_dtype branch_dtype,
+                          int64_t rows, int64_t hidden, const float* gate, float temperature, float eps,
+                          cudaStream_t stream) {
+    return residual_entry(stream_in, branch, stream_out, branch_dtype, rows, hidden, gate, true, temperature, eps,
+                          stream, "muse_residual");
+}
+
+}  // extern "C"
+
+namespace {
+
+// The backward's row blocks at most, for either branch dtype: its CTAs are
+// min(256, vectors per row rounded up to 32) threads, so at most
+// min(32, 2048 / threads) of them reside on an SM; the row blocks are those
+// resident CTAs over the column blocks, and no more than the row tiles of 4.
+int64_t residual_bwd_parts_cap(int64_t rows, int64_t hidden) {
+    int64_t cap = 0;
+    for (int vec : {8, 4}) {
+        const int64_t nvec = hidden / vec;
+        if (nvec < 1) continue;
+        const int64_t threads = nvec >= 256 ? 256 : (nvec + 31) / 32 * 32;
+        const int64_t per_sm = 2048 / threads < 32 ? 2048 / threads : 32;
+        const int64_t gy = (nvec + threads - 1) / threads;
+        const int64_t gx = (per_sm * (int64_t)muse::sm_count() + gy - 1) / gy;
+        if (gx > cap) cap = gx;
+    }
+    const int64_t tiles = (rows + 3) / 4;
+    return tiles < cap ? tiles : cap;
+}
+
+muse_status residual_bwd_entry(const float* stream_in, const void* branch, const float* dstream_out,
+                               float* dstream_in, void* dbranch, muse_dtype branch_dtype, int64_t rows,
+                               int64_t hidden, const float* p, bool gate, float temperature, float eps,
+                               float* dparam, void* ws, size_t ws_bytes, cudaStream_t stream, const char* name) {
+    if (!valid_dtype(branch_dtype)) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype %d", name, (int)branch_dtype);
+    if (rows < 0 || hidden <= 0)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: rows=%lld hidden=%lld", name, (long long)rows, (long long)hidden);
+    if (gate && !(finite(temperature) && temperature > 0.0f && finite(eps) && eps >= 0.0f && eps <= 1.0f))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: temperature must be finite and > 0, eps in [0, 1]", name);
+    if (!p) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null %s", name, gate ? "gate" : "theta");
+    if (rows == 0) {
+        if (dparam) return from_cuda(cudaMemsetAsync(dparam, 0, sizeof(float) * (size_t)hidden, stream), name);
+        return MUSE_OK;
+    }
+    if (!stream_in || !branch || !dstream_out || !dstream_in || !dbranch)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null tensor", name);
+    const int64_t es = elem_size(branch_dtype);
+    if (!aligned(stream_in, 16) || !aligned(branch, 16) || !aligned(dstream_out, 16) || !aligned(dstream_in, 16) ||
+        !aligned(dbranch, 16) || !aligned(p, 16) || (dparam && !aligned(dparam, 16)) || (hidden * es) % 16)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: pointers and row widths must be 16-byte multiples", name);
+    if (hidden / vec_elems(branch_dtype) > (int64_t)65535 * 256)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: rows of more than %d 16-byte vectors", name, 65535 * 256);
+    const size_t need = (size_t)residual_bwd_parts_cap(rows, hidden) * (size_t)hidden * sizeof(float);
+    if (dparam) {
+        muse_status st = bwd_workspace_check(name, need, ws, ws_bytes, true);
+        if (st != MUSE_OK) return st;
+    }
+    const Span sh = span(stream_in, rows, hidden, hidden, 4), sdo = span(dstream_out, rows, hidden, hidden, 4);
+    const Span sb = span(branch, rows, hidden, hidden, es), sdb = span(dbranch, rows, hidden, hidden, es);
+    const Span sdi = span(dstream_in, rows, hidden, hidden, 4), sp = span(p, 1, hidden, hidden, 4);
+    const Span sdp = span(dparam, dparam ? 1 : 0, hidden, hidden, 4);
+    const Span sws = span(ws, dparam ? 1 : 0, (int64_t)ws_bytes, (int64_t)ws_bytes, 1);
+    bool bad = bad_alias(sdi, sdo, true) || any_overlap(sdi, {sh, sb, sdb, sp, sdp, sws});
+    bad = bad || bad_alias(sdb, sb, true) || any_overlap(sdb, {sh, sdo, sp, sdp, sws});
+    bad = bad || any_overlap(sdp, {sh, sdo, sb, sp, sws}) || any_overlap(sws, {sh, sdo, sb, sp});
+    if (bad) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: an output or the workspace overlaps another tensor", name);
+    muse::ResidualArgs a{};
+    a.stream_in = stream_in;
+    a.branch = branch;
+    a.stream_out = dstream_in;
+    a.theta = gate ? nullptr : p;
+    a.gate = gate ? p : nullptr;
+    a.rows = rows;
+    a.width = hidden;
+    a.temperature = temperature;
+    a.eps = eps;
+    a.dy = dstream_out;
+    a.dbranch = dbranch;
+    a.part = dparam ? static_cast<float*>(ws) : nullptr;
+    if (dparam) {
+        int64_t gx = 0;
+        muse_status st = from_cuda(muse::launch_residual_blend_bwd(branch_dtype, gate, a, dparam, stream, &gx), name);
+        if (st != MUSE_OK) return st;
+        if ((size_t)gx * (size_t)hidden * sizeof(float) > need)
+            return fail(MUSE_ERR_UNSUPPORTED, "%s: the grid's partial rows exceed the workspace bound", name);
+    }
+    return from_cuda(muse::launch_residual_blend_bwd(branch_dtype, gate, a, dparam, stream), name);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t muse_residual_backward_workspace_bytes(int64_t rows, int64_t hidden) {
+    if (rows <= 0 || hidden <= 0 || hidden > (int64_t)1 << 30) return 0;
+    return (size_t)residual_bwd_parts_cap(rows, hidden) * (size_t)hidden * sizeof(float);
+}
+
+muse_status muse_residual_blend_backward(const float* stream_in, const void* branch, const float* dstream_out,
+                                         float* dstream_in, void* dbranch, muse_dtype branch_dtype, int64_t rows,
+                                         int64_t hidden, const float* theta, float* dtheta, void* workspace,
+                                         size_t workspace_bytes, cudaStream_t stream) {
+    return residual_bwd_entry(stream_in, branch, dstream_out, dstream_in, dbranch, branch_dtype, rows, hidden,
+                              theta, false, 1.0f, 0.0f, dtheta, workspace, workspace_bytes, stream,
+                              "muse_residual_blend_backward");
+}
+
+muse_status muse_residual_backward(const float* stream_in, const void* branch, const float* dstream_out,
+                                   float* dstream_in, void* dbranch, muse_dtype branch_dtype, int64_t rows,
+                                   int64_t hidden, const float* gate, float temperature, float eps, float* dgate,
+                                   void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    return residual_bwd_entry(stream_in, branch, dstream_out, dstream_in, dbranch, branch_dtype, rows, hidden,
+                              gate, true, temperature, eps, dgate, workspace, workspace_bytes, stream,
+                              "muse_residual_backward");
+}
+
+muse_status muse_residual_gate_angles(const float* gate, float* theta, int64_t hidden, float temperature,
+                                      float eps, cudaStream_t stream) {
+    const char* name = "muse_residual_gate_angles";
+    if (hidden <= 0) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: hidden=%lld", name, (long long)hidden);
+    if (!(finite(temperature) && temperature > 0.0f && finite(eps) && eps >= 0.0f && eps <= 1.0f))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: temperature must be finite and > 0, eps in [0, 1]", name);
+    if (!gate || !theta) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null gate or theta", name);
+    if (!aligned(gate, 4) || !aligned(theta, 4))
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: gate / theta not 4-byte aligned", name);
+    if (overlap(span(theta, 1, hidden, hidden, 4), span(gate, 1, hidden, hidden, 4)) && theta != gate)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: theta partially overlaps gate", name);
+    if (hidden > ((int64_t)1 << 31) - 256) return fail(MUSE_ERR_UNSUPPORTED, "%s: hidden too large", name);
+    muse::ResidualArgs a{};
+    a.gate = gate;
+    a.width = hidden;
+    a.temperature = temperature;
+    a.eps = eps;
+    return from_cuda(muse::launch_residual_gate_angles(a, theta, stream), name);
+}
+
 size_t muse_norm_backward_workspace_bytes(int64_t rows, int64_t hidden) {
     if (rows <= 0 || hidden <= 0 || hidden > (int64_t)1 << 30) return 0;
     return muse::row_bwd_workspace_bytes(rows, (int32_t)hidden);
@@ -455,19 +687,9 @@ muse_status muse_rms_norm_backward_noalloc(const void* x, const void* dy, void* 
                                            int64_t dy_row_stride, int64_t dx_row_stride,
                                            const float* gain, float gain_offset, float eps,
                                            float* dgain, cudaStream_t stream) {
-    const char* name = "muse_rms_norm_backward_noalloc";
-    void* scratch = nullptr;
-    if (dgain && gain && rows > 0 && hidden > 0 && hidden <= ((int64_t)1 << 30)) {
-        const size_t need = muse::row_bwd_gain_scratch_bytes(rows, (int32_t)hidden);
-        if (need > muse::kNoAllocScratchBytes)
-            return fail(MUSE_ERR_UNSUPPORTED, "%s: gain partials need %zu bytes, the fixed scratch holds %zu",
-                        name, need, muse::kNoAllocScratchBytes);
-        const muse_status st = from_cuda(muse::noalloc_scratch(&scratch), name);
-        if (st != MUSE_OK) return st;
-    }
     return row_bwd_entry(false, x, dy, dx, dtype, rows, hidden, x_row_stride, dy_row_stride,
-                         dx_row_stride, gain, gain_offset, eps, dgain, scratch,
-                         scratch ? muse::kNoAllocScratchBytes : 0, stream, name);
+                         dx_row_stride, gain, gain_offset, eps, dgain, nullptr, 0, stream,
+                         "muse_rms_norm_backward_noalloc", true);
 }
 
 muse_status muse_input_scale_norm_backward(const void* x, const void* dy, void* dx,
@@ -674,7 +896,6 @@ muse_status muse_qk_norm_rope_backward(const void* q, const void* k, const void*
     a.hq = hq;
     a.hkv = hkv;
     a.head_dim = head_dim;
-    a.split = 1;
     a.pos_mode = positions ? 0 : (layout == MUSE_LAYOUT_BSHD ? 1 : 2);
     a.eps = eps;
     a.query_scale = query_scale;
@@ -835,6 +1056,8 @@ muse_status muse_vision_rope(const void* q, const void* k, void* q_out, void* k_
         return fail(MUSE_ERR_UNSUPPORTED, "%s: pointers, head_dim and strides must be 16-byte multiples", name);
     if ((qw + kw) / vec_elems(dtype) > (int64_t)1 << 30)
         return fail(MUSE_ERR_UNSUPPORTED, "%s: token rows too wide", name);
+    if (head_dim * es > 512)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: head_dim=%d exceeds 512 bytes per head", name, head_dim);
     const Span sq = span(q, tokens, qw, q_tok_stride, es), sk = span(k, tokens, kw, k_tok_stride, es);
     const Span sqo = span(q_out, tokens, qw, q_out_tok_stride, es);
     const Span sko = span(k_out, tokens, kw, k_out_tok_stride, es);

@@ -266,9 +266,13 @@ __global__ void __launch_bounds__(256, MINB) qk_norm_rope_kernel(const __grid_co
 
 constexpr int kThreads = 256;
 // Q/K kernel: 4 head steps per batch, a ring of 3 batches per warp (48 KB of
-// slots per CTA), registers for 4 resident CTAs (32 warps) per SM - measured
-// best on B200 at prefill sizes, where it runs at the speed of a plain copy of
-// the same bytes.
+// slots per CTA), registers for 4 resident CTAs (32 warps) per SM.  Measured
+// on B200 against persistent grids that balance (token, batch) units over all
+// warps: contiguous unit ranges per warp 8% slower at prefill and 20% slower
+// at 32k-80k tokens (the warps stream thousands of far-apart windows), units
+// dealt round-robin 35% slower (angles and positions recomputed per unit).
+// What this one-shot grid loses at prefill is the last wave (8192 tokens on
+// 4736 warp slots is 1.73 waves).
 constexpr int kQkBatch = 4;
 constexpr int kQkRing = 3;
 constexpr int kQkMinBlocks = 4;
@@ -323,10 +327,10 @@ cudaError_t launch_qk_l(const QkArgs& a0, cudaStream_t s) {
                        a.hkv % RW == 0 && nst_q % BATCH == 0 && nst_k % BATCH == 0;
     auto kern = exact ? qk_norm_rope_kernel<T, L, ROPE, UPCAST, false, BATCH, kQkRing, kQkMinBlocks>
                       : qk_norm_rope_kernel<T, L, ROPE, UPCAST, true, BATCH, kQkRing, kQkMinBlocks>;
-    if (smem > 48 * 1024) {
-        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
+    // the opt-in is needed whenever static + dynamic shared memory passes 48 KB
+    // (the mbarriers are static), so it is always set
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     return launch_pdl(kern, (unsigned)grid, kThreads, smem, s, a);
 }
 

@@ -43,6 +43,13 @@ struct RowArgs {
     // kRmsGrouped: gain is [num_groups, width]; rows [offsets[g], offsets[g+1]) use row g
     const int32_t* group_offsets;
     int32_t num_groups;
+    // Bounded-wait probe (0 / unset in every ordinary call): spin_limit > 0
+    // replaces the default poll limit of every mbarrier wait; with
+    // probe_stall != 0 the producer never signals the stage of row stall_row
+    // (and issues nothing after it), so that row's wait runs out.
+    uint32_t spin_limit;
+    int32_t probe_stall;
+    int64_t stall_row;
 };
 
 // Many short rows (one attention head each), contiguous: core 4 per head.
@@ -90,6 +97,9 @@ size_t row_bwd_workspace_bytes(int64_t rows, int32_t width);
 size_t row_bwd_gain_scratch_bytes(int64_t rows, int32_t width);
 constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;
 cudaError_t noalloc_scratch(void** ptr);
+// The grid a row backward launch of these arguments uses on the current
+// device (nothing is launched); its gain partials take grid * width floats.
+cudaError_t row_bwd_launch_grid(int dtype, BwdOp op, const RowBwdArgs& a, int64_t* grid);
 
 constexpr int kMaxHalfDim = 128;  // head_dim <= 256
 
@@ -105,7 +115,7 @@ struct QkArgs {
     int64_t q_stride, k_stride, q_out_stride, k_out_stride;  // elements per token
     int32_t num_seqs;
     int32_t hq, hkv, head_dim;
-    int32_t split;              // warps sharing one token's head steps (1, 2, 4, 8)
+    int32_t split;              // forward: warps sharing one token's head steps (1, 2, 4, 8; set by the launcher)
     int32_t pos_mode;           // 0 explicit, 1 BSHD derived, 2 THD derived
     float eps;
     float query_scale;
@@ -161,6 +171,35 @@ struct VisionFreqArgs {
 cudaError_t launch_vision_rope(int dtype, const VisionRopeArgs& a, cudaStream_t s);
 cudaError_t launch_vision_rope_frequencies(const VisionFreqArgs& a, cudaStream_t s);
 cudaError_t read_qk_bwd_device_error(unsigned int* out, bool clear);
+
+// _residual_core: stream_out = c * stream_in + s * f32(branch) per channel,
+// (c, s) = (cos, sin) of theta, or from the learned gate (gate != null):
+// c^2 = max(sigmoid(gate / temperature), eps), s^2 = 1 - c^2.  Rows contiguous.
+struct ResidualArgs {
+    const float* stream_in;
+    const void* branch;
+    float* stream_out;      // forward: the new stream; backward: dL/dstream_in
+    const float* theta;     // angle form
+    const float* gate;      // gate form
+    int64_t rows;
+    int64_t width;
+    float temperature;
+    float eps;
+    // backward only
+    const float* dy;        // dL/dstream_out, FP32 [rows, width]
+    void* dbranch;          // dL/dbranch, branch dtype
+    float* part;            // [row blocks][width] partial angle / gate gradients (workspace)
+};
+cudaError_t launch_residual_blend(int dtype, bool gate, const ResidualArgs& a, cudaStream_t s);
+// Backward; dparam (dtheta or dgate, [width]) may be null.  With plan_gx the
+// row-block count of the grid (the partial rows the workspace must hold) is
+// returned and nothing is launched.
+cudaError_t launch_residual_blend_bwd(int dtype, bool gate, const ResidualArgs& a, float* dparam,
+                                      cudaStream_t s, int64_t* plan_gx = nullptr);
+// Deterministic column sums of nparts partial rows of width floats (row_bwd.cu).
+cudaError_t launch_param_grad_reduce(const float* part, int nparts, int width, float* out, cudaStream_t s);
+// theta[j] = atan2(s_j, c_j) from a.gate (a.width channels).
+cudaError_t launch_residual_gate_angles(const ResidualArgs& a, float* theta, cudaStream_t s);
 
 // Returns cudaSuccess or the launch error.
 // launch_row: TMA-pipelined kernels (row_tma.cu), falling back to

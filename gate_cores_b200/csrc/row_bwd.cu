@@ -379,8 +379,13 @@ __global__ void __launch_bounds__(32 * kReduceGroups) param_grad_reduce_kernel(c
 
 int bwd_grid_cap() { return kBwdMaxCtasPerSm * sm_count(); }
 
+// Launch shape of one instance: threads, dynamic shared memory and the grid
+// (resident CTAs x SMs, at most kBwdMaxCtasPerSm per SM and one CTA per row).
+// With plan_only the kernel is not launched (the grid is what a launch of the
+// same arguments on the current device would use).
 template <typename T, BwdOp OP, int VPT, bool G, int S>
-cudaError_t launch_bwd_s(RowBwdArgs a, int nvec, float* dgain, float* dtheta, cudaStream_t s) {
+cudaError_t launch_bwd_s(RowBwdArgs a, int nvec, float* dgain, float* dtheta, cudaStream_t s,
+                         int64_t* plan_grid = nullptr) {
     const int ncons = ((nvec + VPT - 1) / VPT + 31) / 32 * 32;
     const int threads = ncons + 32;
     const BwdLayout L = bwd_layout<T, OP>(a.width);
@@ -392,6 +397,10 @@ cudaError_t launch_bwd_s(RowBwdArgs a, int nvec, float* dgain, float* dtheta, cu
     int64_t grid = (int64_t)per_sm * sm_count();
     if (grid > a.rows) grid = a.rows;
     if (grid < 1) grid = 1;
+    if (plan_grid) {
+        *plan_grid = grid;
+        return cudaSuccess;
+    }
     if (!(G && dgain)) a.part_gain = nullptr;
     if (!dtheta) a.part_theta = nullptr;
     e = launch_pdl(kern, (unsigned)grid, (unsigned)threads, smem, s, a);
@@ -409,37 +418,43 @@ cudaError_t launch_bwd_s(RowBwdArgs a, int nvec, float* dgain, float* dtheta, cu
 }
 
 template <typename T, BwdOp OP, int VPT>
-cudaError_t launch_bwd_v(const RowBwdArgs& a, int nvec, float* dgain, float* dtheta, cudaStream_t s) {
+cudaError_t launch_bwd_v(const RowBwdArgs& a, int nvec, float* dgain, float* dtheta, cudaStream_t s,
+                         int64_t* plan_grid) {
     const BwdLayout L = bwd_layout<T, OP>(a.width);
     const bool g = a.gain != nullptr;
-    if (L.stage_bytes < 16 * 1024)
-        return g ? launch_bwd_s<T, OP, VPT, true, 3>(a, nvec, dgain, dtheta, s)
-                 : launch_bwd_s<T, OP, VPT, false, 3>(a, nvec, dgain, dtheta, s);
-    return g ? launch_bwd_s<T, OP, VPT, true, 2>(a, nvec, dgain, dtheta, s)
-             : launch_bwd_s<T, OP, VPT, false, 2>(a, nvec, dgain, dtheta, s);
+    // three stages up to 16 KB (cores 1, 2 at 4096 bf16 columns: 3% faster
+    // than two); core 5's 40 KB stages stay at two (three measured slower)
+    if (L.stage_bytes <= 16 * 1024)
+        return g ? launch_bwd_s<T, OP, VPT, true, 3>(a, nvec, dgain, dtheta, s, plan_grid)
+                 : launch_bwd_s<T, OP, VPT, false, 3>(a, nvec, dgain, dtheta, s, plan_grid);
+    return g ? launch_bwd_s<T, OP, VPT, true, 2>(a, nvec, dgain, dtheta, s, plan_grid)
+             : launch_bwd_s<T, OP, VPT, false, 2>(a, nvec, dgain, dtheta, s, plan_grid);
 }
 
 // Slots per consumer thread: one up to 256 vectors (core 5: 512), then two,
 // then four (cores 1, 2).
 template <typename T, BwdOp OP>
-cudaError_t launch_bwd_op(const RowBwdArgs& a, float* dgain, float* dtheta, cudaStream_t s) {
+cudaError_t launch_bwd_op(const RowBwdArgs& a, float* dgain, float* dtheta, cudaStream_t s,
+                          int64_t* plan_grid) {
     const int nvec = a.width / Vec<T>::N;
-    if (nvec <= 256 || (b_is_res(OP) && nvec <= 512)) return launch_bwd_v<T, OP, 1>(a, nvec, dgain, dtheta, s);
+    if (nvec <= 256 || (b_is_res(OP) && nvec <= 512))
+        return launch_bwd_v<T, OP, 1>(a, nvec, dgain, dtheta, s, plan_grid);
     if constexpr (b_is_res(OP)) {
-        return launch_bwd_v<T, OP, 2>(a, nvec, dgain, dtheta, s);
+        return launch_bwd_v<T, OP, 2>(a, nvec, dgain, dtheta, s, plan_grid);
     } else {
-        if (nvec <= 512) return launch_bwd_v<T, OP, 2>(a, nvec, dgain, dtheta, s);
-        return launch_bwd_v<T, OP, 4>(a, nvec, dgain, dtheta, s);
+        if (nvec <= 512) return launch_bwd_v<T, OP, 2>(a, nvec, dgain, dtheta, s, plan_grid);
+        return launch_bwd_v<T, OP, 4>(a, nvec, dgain, dtheta, s, plan_grid);
     }
 }
 
 template <typename T>
-cudaError_t launch_bwd_t(BwdOp op, const RowBwdArgs& a, float* dgain, float* dtheta, cudaStream_t s) {
+cudaError_t launch_bwd_t(BwdOp op, const RowBwdArgs& a, float* dgain, float* dtheta, cudaStream_t s,
+                         int64_t* plan_grid = nullptr) {
     switch (op) {
-        case BwdOp::kRms: return launch_bwd_op<T, BwdOp::kRms>(a, dgain, dtheta, s);
-        case BwdOp::kInputScale: return launch_bwd_op<T, BwdOp::kInputScale>(a, dgain, dtheta, s);
-        case BwdOp::kResidual: return launch_bwd_op<T, BwdOp::kResidual>(a, dgain, dtheta, s);
-        case BwdOp::kResidualIS: return launch_bwd_op<T, BwdOp::kResidualIS>(a, dgain, dtheta, s);
+        case BwdOp::kRms: return launch_bwd_op<T, BwdOp::kRms>(a, dgain, dtheta, s, plan_grid);
+        case BwdOp::kInputScale: return launch_bwd_op<T, BwdOp::kInputScale>(a, dgain, dtheta, s, plan_grid);
+        case BwdOp::kResidual: return launch_bwd_op<T, BwdOp::kResidual>(a, dgain, dtheta, s, plan_grid);
+        case BwdOp::kResidualIS: return launch_bwd_op<T, BwdOp::kResidualIS>(a, dgain, dtheta, s, plan_grid);
     }
     return cudaErrorInvalidValue;
 }
@@ -474,9 +489,19 @@ size_t row_bwd_gain_scratch_bytes(int64_t rows, int32_t width) {
     return (size_t)(grid < 1 ? 1 : grid) * (size_t)width * sizeof(float);
 }
 
+cudaError_t row_bwd_launch_grid(int dtype, BwdOp op, const RowBwdArgs& a, int64_t* grid) {
+    return dtype == 0 ? launch_bwd_t<__nv_bfloat16>(op, a, nullptr, nullptr, nullptr, grid)
+                      : launch_bwd_t<float>(op, a, nullptr, nullptr, nullptr, grid);
+}
+
 size_t row_bwd_workspace_bytes(int64_t rows, int32_t width) {
     const int64_t grid = min(rows, (int64_t)bwd_grid_cap());
     return (size_t)(grid < 1 ? 1 : grid) * (size_t)width * sizeof(float) * 2;
+}
+
+cudaError_t launch_param_grad_reduce(const float* part, int nparts, int width, float* out, cudaStream_t s) {
+    const unsigned rgrid = (unsigned)((width + 31) / 32);
+    return launch_pdl(param_grad_reduce_kernel, rgrid, 32u * kReduceGroups, 0, s, part, nparts, width, out);
 }
 
 cudaError_t launch_row_bwd(int dtype, BwdOp op, RowBwdArgs a, float* dgain, float* dtheta, cudaStream_t s) {

@@ -110,6 +110,7 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
     const int warp = tid >> 5, lane = tid & 31;
     const int nvec = a.width / V;
     const StageLayout L = stage_layout<T, OP>(a.width);
+    const uint32_t lim = a.spin_limit ? a.spin_limit : kSpinLimit;  // polls per mbarrier wait
 
     // This CTA's rows: r0, r0 + step, ... - rows interleaved across the grid,
     // so at any time the CTAs stream one compact window of the tensors
@@ -170,10 +171,12 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
             int grp = -1, runs = 0;  // per-expert core 1: current group, runs started
             for (int k = 0; k < n && ok; ++k) {
                 const int s = k % S;
-                if (k >= S) ok = mbar_wait(&empty_bar[s], (uint32_t)((k / S - 1) & 1));
+                const int64_t row = r0 + k * step;
+                // bounded-wait probe: this row's stage is never signalled
+                if (a.probe_stall && row == a.stall_row) break;
+                if (k >= S) ok = mbar_wait(&empty_bar[s], (uint32_t)((k / S - 1) & 1), lim);
                 if (!ok) break;
                 unsigned char* st = smem + (size_t)s * L.stage_bytes;
-                const int64_t row = r0 + k * step;
                 if constexpr (t_grouped(OP)) {
                     // the activation copy first; the stage's run index is written
                     // before the producer's arrival, which completes the phase
@@ -189,7 +192,7 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
                     if (g != grp) {
                         // a new run: its slot's previous run must be released first
                         const int j = runs % nslots;
-                        if (runs >= nslots) ok = mbar_wait(&gain_free[j], (uint32_t)((runs / nslots - 1) & 1));
+                        if (runs >= nslots) ok = mbar_wait(&gain_free[j], (uint32_t)((runs / nslots - 1) & 1), lim);
                         if (ok) {
                             mbar_arrive_expect_tx(&gain_full[j], (uint32_t)a.width * 4u);
                             bulk_g2s(gslots + (size_t)j * gslot_bytes, a.gain + (int64_t)g * a.width,
@@ -219,10 +222,10 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
             // the normal path the consumers already waited on them, so these
             // waits return at once.
             for (int k = max(0, issued - S); k < issued; ++k)
-                if (!mbar_wait(&full_bar[k % S], (uint32_t)((k / S) & 1))) break;
+                if (!mbar_wait(&full_bar[k % S], (uint32_t)((k / S) & 1), lim)) break;
             if constexpr (t_grouped(OP)) {
                 for (int r = max(0, runs - nslots); r < runs; ++r)
-                    if (!mbar_wait(&gain_full[r % nslots], (uint32_t)((r / nslots) & 1))) break;
+                    if (!mbar_wait(&gain_full[r % nslots], (uint32_t)((r / nslots) & 1), lim)) break;
             }
         }
         return;
@@ -300,7 +303,7 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
     uint32_t phase = 0;
     int run = -1;  // per-expert core 1: the expert run whose gain slot this warp holds
     for (int k = 0; k < n; ++k) {
-        if (alive) alive = mbar_wait(&full_bar[s], phase);
+        if (alive) alive = mbar_wait(&full_bar[s], phase, lim);
         alive = __all_sync(0xffffffffu, alive);
         const unsigned char* st = smem + s * L.stage_bytes;
         if constexpr (t_grouped(OP)) {
@@ -309,7 +312,7 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
                 // the first row of the next expert run: wait for its gain row,
                 // copy it (plus the offset, an FP32 sum) to registers, release the slot
                 run = r;
-                alive = mbar_wait(&gain_full[run % nslots], (uint32_t)((run / nslots) & 1));
+                alive = mbar_wait(&gain_full[run % nslots], (uint32_t)((run / nslots) & 1), lim);
                 alive = __all_sync(0xffffffffu, alive);
                 if (alive) {
                     if constexpr (HAS_GAIN) {
@@ -446,43 +449,46 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
 }
 
 // One entry symbol per core, so launch lists and profiles name the core.
+// One-slot instances keep a register budget for two resident CTAs of up to
+// 544 threads (core 5 at 4096 columns: 2 x 544 threads; one CTA per SM
+// measured 20% slower).
 template <typename T, int VPT, bool G, int S>
-__global__ void __launch_bounds__(512 + 32) rms_norm_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(512 + 32, VPT == 1 ? 2 : 1) rms_norm_kernel(const __grid_constant__ RowArgs a) {
     pdl_begin();
     row_tma_body<T, RowOp::kRms, VPT, G, S>(a);
 }
 template <typename T, int VPT, bool G, int S>
-__global__ void __launch_bounds__(512 + 32) input_scale_norm_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(512 + 32, VPT == 1 ? 2 : 1) input_scale_norm_kernel(const __grid_constant__ RowArgs a) {
     pdl_begin();
     row_tma_body<T, RowOp::kInputScale, VPT, G, S>(a);
 }
 template <typename T, int VPT, bool G, int S>
-__global__ void __launch_bounds__(512 + 32) output_norm_gate_row_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(512 + 32, VPT == 1 ? 2 : 1) output_norm_gate_row_kernel(const __grid_constant__ RowArgs a) {
     pdl_begin();
     row_tma_body<T, RowOp::kNormGate, VPT, G, S>(a);
 }
 template <typename T, int VPT, bool G, int S>
-__global__ void __launch_bounds__(512 + 32) norm_residual_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(512 + 32, VPT == 1 ? 2 : 1) norm_residual_kernel(const __grid_constant__ RowArgs a) {
     pdl_begin();
     row_tma_body<T, RowOp::kResidual, VPT, G, S>(a);
 }
 template <typename T, int VPT, bool G, int S>
-__global__ void __launch_bounds__(512 + 32) norm_residual_input_scale_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(512 + 32, VPT == 1 ? 2 : 1) norm_residual_input_scale_kernel(const __grid_constant__ RowArgs a) {
     pdl_begin();
     row_tma_body<T, RowOp::kResidualIS, VPT, G, S>(a);
 }
 template <typename T, int VPT, bool G, int S>
-__global__ void __launch_bounds__(512 + 32) rms_norm_grouped_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(512 + 32, VPT == 1 ? 2 : 1) rms_norm_grouped_kernel(const __grid_constant__ RowArgs a) {
     pdl_begin();
     row_tma_body<T, RowOp::kRmsGrouped, VPT, G, S>(a);
 }
 template <typename T, int VPT, bool G, int S>
-__global__ void __launch_bounds__(512 + 32) norm_residual_prenorm_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(512 + 32, VPT == 1 ? 2 : 1) norm_residual_prenorm_kernel(const __grid_constant__ RowArgs a) {
     pdl_begin();
     row_tma_body<T, RowOp::kResidualPre, VPT, G, S>(a);
 }
 template <typename T, int VPT, bool G, int S>
-__global__ void __launch_bounds__(512 + 32) norm_residual_input_scale_prenorm_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(512 + 32, VPT == 1 ? 2 : 1) norm_residual_input_scale_prenorm_kernel(const __grid_constant__ RowArgs a) {
     pdl_begin();
     row_tma_body<T, RowOp::kResidualISPre, VPT, G, S>(a);
 }

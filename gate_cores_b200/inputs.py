@@ -139,6 +139,13 @@ def theta(wl: Workload, seed: int, tag: str = "theta") -> torch.Tensor:
     return u * float(math.pi / 2)
 
 
+def residual_gate(wl: Workload, seed: int, tag: str = "residual_gate") -> torch.Tensor:
+    """Learned residual gate [H] FP32 for _residual_core: N(0, 1) (the pages
+    give no distribution; at temperature 0.3 this spans the sigmoid from its
+    lower bound to saturation)."""
+    return torch.randn(wl.hidden, generator=_gen(seed, wl.name, tag), dtype=torch.float32)
+
+
 def expert_groups(wl: Workload, seed: int, num_groups: int, tokens: int | None = None) -> torch.Tensor:
     """Routed-token group boundaries for per-expert norms: int32 [num_groups + 1],
     0 .. tokens, group sizes drawn from a seeded Dirichlet-like split (some
@@ -222,7 +229,7 @@ class CoreInputs:
 def make_inputs(wl: Workload | str, core: str, seed: int = 0, act_dtype=torch.bfloat16,
                 zero_centered: bool = True) -> CoreInputs:
     """Inputs of one core.  core in {rms_norm, input_scale_norm, qk_norm_rope,
-    output_norm_gate, norm_residual}."""
+    output_norm_gate, norm_residual, residual_blend, residual}."""
     if isinstance(wl, str):
         wl = WORKLOADS[wl]
     T = num_tokens(wl, seed)
@@ -256,6 +263,14 @@ def make_inputs(wl: Workload | str, core: str, seed: int = 0, act_dtype=torch.bf
         ci.tensors["gain"] = g
         ci.tensors["theta"] = theta(wl, seed)
         ci.scalars.update(gain_offset=off, norm_eps=1e-6)
+    elif core in ("residual_blend", "residual"):
+        ci.tensors["stream"] = activation(wl, seed, "stream", (T, H), torch.float32)
+        ci.tensors["branch"] = activation(wl, seed, "branch", (T, H), act_dtype)
+        if core == "residual_blend":
+            ci.tensors["theta"] = theta(wl, seed)
+        else:
+            ci.tensors["gate"] = residual_gate(wl, seed)
+            ci.scalars.update(temperature=0.3, eps=1e-3)
     else:
         raise ValueError(f"unknown core {core!r}")
     return ci

@@ -161,6 +161,74 @@ muse_status muse_norm_residual(const float* stream_in, const void* branch, float
                                int input_scale, float norm_eps, cudaStream_t stream);
 
 /*
+ * _residual_core / MuseSparkResidual.forward (layers page: "blend the
+ * residual and branch using the checkpoint's learned gate"; a learned
+ * norm-preserving residual connection) - the blend without a branch norm.
+ * The page gives no formula; two forms are offered:
+ *
+ * muse_residual_blend - the blend core 5 uses, per channel j:
+ *   stream_out[r, j] = cos(theta[j]) * stream_in[r, j] + sin(theta[j]) * f32(branch[r, j])
+ *   (FP32 arithmetic; the branch is read as it is, no cast).
+ * muse_residual - the page's signature (gate, temperature, eps), read as
+ *   c^2 = max(sigmoid(gate[j] / temperature), eps)   (eps: the lower bound on
+ *         the squared residual coefficient),  s^2 = 1 - c^2,  c, s >= 0,
+ *   stream_out[r, j] = c * stream_in[r, j] + s * f32(branch[r, j]),
+ *   i.e. muse_residual_blend with theta = atan2(s, c).  temperature finite
+ *   and > 0, eps in [0, 1], else MUSE_ERR_INVALID_ARGUMENT.  The page's
+ *   defaults are temperature 0.3 and eps 0.001.
+ * stream_in, stream_out: FP32 [rows, hidden] contiguous (stream_out ==
+ * stream_in is allowed); branch: [rows, hidden] contiguous in branch_dtype;
+ * theta / gate: FP32 [hidden].  Pointers 16-byte aligned and hidden a
+ * multiple of 16 bytes of the branch dtype, else MUSE_ERR_UNSUPPORTED.
+ */
+muse_status muse_residual_blend(const float* stream_in, const void* branch, float* stream_out,
+                                muse_dtype branch_dtype, int64_t rows, int64_t hidden, const float* theta,
+                                cudaStream_t stream);
+muse_status muse_residual(const float* stream_in, const void* branch, float* stream_out, muse_dtype branch_dtype,
+                          int64_t rows, int64_t hidden, const float* gate, float temperature, float eps,
+                          cudaStream_t stream);
+
+/*
+ * Backward of _residual_core (both forms), in the convention of the other
+ * backward calls (the gradient of every cast the forward materialises is the
+ * incoming gradient rounded to that tensor's dtype).  Given the forward's
+ * stream_in, branch and theta or gate, and dstream_out = dL/dstream_out (FP32):
+ *   dstream_in = c * dstream_out                              (FP32);
+ *   dbranch    = cast_branch(s * dstream_out);
+ *   dtheta[j]  = sum over rows of dstream_out (c b - s h)     (angle form),
+ *   dgate[j]   = sum over rows of dstream_out (dc/dgate h + ds/dgate b)
+ *              = c s / (2 temperature) * sum of dstream_out (s h - c b)
+ *                where sigmoid(gate / temperature) >= eps, else 0 (gate form).
+ * dtheta / dgate may be NULL (then the workspace may be NULL too); otherwise a
+ * caller-owned device workspace of muse_residual_backward_workspace_bytes(rows,
+ * hidden) bytes (16-byte aligned; contents ignored on entry, undefined on
+ * return) holds one partial row per row block, summed in a fixed order.
+ * dstream_in may be the very memory of dstream_out, dbranch of branch; nothing
+ * else may overlap.  Limits and errors as muse_residual; rows == 0 zeroes
+ * dtheta / dgate.
+ */
+size_t muse_residual_backward_workspace_bytes(int64_t rows, int64_t hidden);
+muse_status muse_residual_blend_backward(const float* stream_in, const void* branch, const float* dstream_out,
+                                         float* dstream_in, void* dbranch, muse_dtype branch_dtype, int64_t rows,
+                                         int64_t hidden, const float* theta, float* dtheta, void* workspace,
+                                         size_t workspace_bytes, cudaStream_t stream);
+muse_status muse_residual_backward(const float* stream_in, const void* branch, const float* dstream_out,
+                                   float* dstream_in, void* dbranch, muse_dtype branch_dtype, int64_t rows,
+                                   int64_t hidden, const float* gate, float temperature, float eps, float* dgate,
+                                   void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * The blend angle of each channel from the learned gate under the reading of
+ * muse_residual: theta[j] = atan2(s_j, c_j) in [0, pi/2].  It turns the
+ * page's (gate, temperature, residual_eps) of _norm_residual_core into the
+ * theta argument of muse_norm_residual / muse_norm_residual_rms_norm.
+ * gate, theta: FP32 [hidden], 4-byte aligned; theta may be the very memory
+ * of gate; temperature and eps as muse_residual.
+ */
+muse_status muse_residual_gate_angles(const float* gate, float* theta, int64_t hidden, float temperature,
+                                      float eps, cudaStream_t stream);
+
+/*
  * Per-expert form of core 1 (MuseSparkMoE pre_expert_norm / post_expert_norm:
  * per-expert norms over the tokens routed to each expert).  The rows arrive
  * grouped by expert, as a grouped-GEMM dispatch lays them out: rows
@@ -188,7 +256,8 @@ muse_status muse_rms_norm_grouped(const void* x, void* y, muse_dtype dtype, int6
  * pair's angle, e.g. from muse_vision_rope_frequencies per grid, concatenated
  * in the packed patch order).  q_out may be the very memory of q, k_out of k;
  * any other overlap is MUSE_ERR_INVALID_ARGUMENT.  Pointers, head rows and
- * strides 16-byte multiples, else MUSE_ERR_UNSUPPORTED.
+ * strides 16-byte multiples, heads of at most 512 bytes (256 bf16 or 128 f32
+ * elements), else MUSE_ERR_UNSUPPORTED.
  */
 muse_status muse_vision_rope(const void* q, const void* k, void* q_out, void* k_out, muse_dtype dtype,
                              int64_t tokens, int32_t hq, int32_t hk, int32_t head_dim,
@@ -278,15 +347,20 @@ muse_status muse_rms_norm_backward(const void* x, const void* dy, void* dx, muse
  * values per CTA) go to a fixed 16 MiB device array of the library, whose
  * address is looked up once per device on the first call that needs it.
  *   - Allocates nothing and never calls cudaMalloc / cudaFree.
- *   - Rejects with MUSE_ERR_UNSUPPORTED a call whose partials exceed the
- *     fixed array (with hidden = 4096, up to 1024 partial rows: any row
- *     count on a GPU whose backward grid stays at or below 1024 CTAs).
+ *   - Every argument is checked first; then a call whose partials exceed the
+ *     fixed array is rejected with MUSE_ERR_UNSUPPORTED.  The partials take
+ *     one row of hidden floats per CTA of the grid this launch uses
+ *     (resident CTAs x SMs, at most 4 per SM, at most one per row): on a
+ *     148-SM B200, hidden = 4096 fits at any row count.
  *   - The array is shared by every call on a device: two calls with dgain
  *     must not run concurrently (issue them on one stream, or order their
  *     streams); calls without dgain do not touch it.
  *   - The first call with dgain on each device performs the address lookup,
  *     which must not happen inside a stream capture: make that first call
- *     outside any capture; later calls are capture-safe.
+ *     outside any capture.
+ *   - The looked-up address is kept for the life of the process: do not use
+ *     this entry point after cudaDeviceReset on that device (the array's
+ *     address may change with the new context).
  */
 muse_status muse_rms_norm_backward_noalloc(const void* x, const void* dy, void* dx, muse_dtype dtype,
                                            int64_t rows, int64_t hidden, int64_t x_row_stride,
@@ -381,6 +455,31 @@ muse_status muse_qk_norm_rope_backward(const void* q, const void* k, const void*
  * pointer, MUSE_ERR_CUDA if the copy fails.
  */
 muse_status muse_device_error(unsigned int* flags, int clear);
+
+/*
+ * Bounded-wait probe (diagnostics; an addition of this library, the API
+ * reference pages have no counterpart).  It runs muse_rms_norm's kernel with
+ * one planted wait that cannot complete, so that a test can drive the
+ * failure handling of the bulk-copy pipeline without faulting or hanging the
+ * GPU.  Arguments as muse_rms_norm, plus:
+ *   spin_limit: polls per mbarrier wait before it gives up, 1 .. 2^24 (the
+ *     ordinary calls use 2^24);
+ *   stall_row: a row in [0, rows).  The producer warp of the CTA that owns
+ *     this row never signals the row's pipeline stage and issues no copy for
+ *     it or for that CTA's later rows.
+ * Expected outcome: every other CTA's rows are normalised as by
+ * muse_rms_norm; in the stalled CTA, the rows before stall_row are too, the
+ * consumer warps give up on stall_row after spin_limit polls, set bit 0 of
+ * muse_device_error, and write nothing from stall_row on; the producer waits
+ * (bounded) for the copies it did issue before the CTA exits, so no copy is
+ * left in flight.  Rows must be at most 16384 bytes (else
+ * MUSE_ERR_UNSUPPORTED); spin_limit or stall_row out of range is
+ * MUSE_ERR_INVALID_ARGUMENT.  Not for production use.
+ */
+muse_status muse_rms_norm_stall_probe(const void* x, void* y, muse_dtype dtype, int64_t rows,
+                                      int64_t hidden, int64_t x_row_stride, int64_t y_row_stride,
+                                      const float* gain, float gain_offset, float eps,
+                                      uint32_t spin_limit, int64_t stall_row, cudaStream_t stream);
 
 /*
  * Bandwidth reference (not a core): copy `bytes` bytes from src to dst with

@@ -43,11 +43,23 @@ VARIANTS = {
         "no_gain": dict(no_gain=True),
         "f32_branch": dict(act_dtype=torch.float32),
     },
+    "residual_blend": {
+        "bf16_branch": dict(),
+        "f32_branch": dict(act_dtype=torch.float32),
+    },
+    "residual": {
+        "bf16_branch": dict(),
+        "f32_branch": dict(act_dtype=torch.float32),
+        "sharp_gate": dict(temperature=0.05, eps=0.01),
+    },
 }
+# _residual_core forms (not among the five cores of the benchmark step)
+RESIDUAL_CORES = ("residual_blend", "residual")
 
 DEFAULT_VARIANT = {"rms_norm": "zc_gain", "input_scale_norm": "plain_gain",
                    "qk_norm_rope": "upcast", "output_norm_gate": "per_head",
-                   "norm_residual": "gain_after"}
+                   "norm_residual": "gain_after", "residual_blend": "bf16_branch",
+                   "residual": "bf16_branch"}
 
 
 def make(wl, core, variant, seed=0):
@@ -107,6 +119,11 @@ def run_gpu(wl, core, ci, stream=None):
         return (cores.norm_residual(_d(t["stream"]), _d(t["branch"]), _d(t["theta"]), _d(t["gain"]),
                                     s["gain_offset"], s.get("input_scale", False), s["norm_eps"],
                                     stream=stream),)
+    if core == "residual_blend":
+        return (cores.residual_blend(_d(t["stream"]), _d(t["branch"]), _d(t["theta"]), stream=stream),)
+    if core == "residual":
+        return (cores.residual(_d(t["stream"]), _d(t["branch"]), _d(t["gate"]), s["temperature"], s["eps"],
+                               stream=stream),)
     raise ValueError(core)
 
 
@@ -133,7 +150,53 @@ def run_oracle(wl, core, ci, rows=None):
         return [oracle.norm_residual(sel(np_(t["stream"])), sel(np_(t["branch"])), np_(t["theta"]),
                                      np_(t["gain"]), s["gain_offset"], s.get("input_scale", False),
                                      s["norm_eps"])]
+    if core == "residual_blend":
+        return [oracle.residual_blend(sel(np_(t["stream"])), sel(np_(t["branch"])), np_(t["theta"]))]
+    if core == "residual":
+        return [oracle.residual(sel(np_(t["stream"])), sel(np_(t["branch"])), np_(t["gate"]),
+                                s["temperature"], float(np.float32(s["eps"])))]
     raise ValueError(core)
+
+
+def compare_full(wl, core, ci, outs, what="", chunk_elems=1 << 21, threads=None):
+    """Every output element of the GPU against the oracle on the same inputs.
+
+    The oracle runs over consecutive row (token) chunks of about chunk_elems
+    output elements on all host threads (its C routines release the
+    interpreter lock); each chunk is checked element by element with
+    parity.check.  Returns per output the combined statistics (n, ambiguous,
+    and max_ulp_vs_oracle_out or max_rel_vs_mag).  Raises AssertionError with
+    the first failing chunk."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    from .parity import check
+
+    host = [to_host(o) for o in outs]
+    T = host[0].shape[0]
+    width = max(int(np.prod(h.shape[1:])) for h in host)
+    step = max(1, chunk_elems // max(1, width))
+    spans = [(lo, min(T, lo + step)) for lo in range(0, T, step)]
+
+    def one(span):
+        lo, hi = span
+        refs = run_oracle(wl, core, ci, slice(lo, hi))
+        return [check(h[lo:hi], r, f"{what} rows {lo}..{hi - 1}") for h, r in zip(host, refs)]
+
+    n = threads or min(32, os.cpu_count() or 1)
+    with ThreadPoolExecutor(max_workers=n) as ex:
+        parts = list(ex.map(one, spans))
+    total = []
+    for k in range(len(host)):
+        st = [p[k] for p in parts]
+        agg = {"n": sum(s["n"] for s in st), "ambiguous": sum(s["ambiguous"] for s in st)}
+        if "max_ulp_vs_oracle_out" in st[0]:
+            agg["max_ulp_vs_oracle_out"] = max(s["max_ulp_vs_oracle_out"] for s in st)
+            agg["exact_frac"] = sum(s["exact_frac"] * s["n"] for s in st) / max(1, agg["n"])
+        else:
+            agg["max_rel_vs_mag"] = max(s["max_rel_vs_mag"] for s in st)
+        total.append(agg)
+    return total
 
 
 def to_host(x: torch.Tensor, rows=None) -> np.ndarray:
@@ -150,4 +213,4 @@ def sample_rows(T: int, n: int = 48, seed: int = 0) -> np.ndarray:
 
 
 __all__ = ["VARIANTS", "DEFAULT_VARIANT", "make", "run_gpu", "run_oracle", "to_host",
-           "sample_rows", "all_positions"]
+           "sample_rows", "all_positions", "compare_full"]

@@ -201,6 +201,8 @@ def test_vision_validation(lib):
     assert call(qs=100) == INV                               # stride below the heads
     assert call(f=None) == INV
     assert call(d=12) == UNS                                 # 24-byte bf16 heads
+    assert call(d=264) == UNS                                # 528-byte heads: above 32 vectors
+    assert call(d=136, dt=F32) == UNS
     assert call(f=F + 8) == UNS                              # table not 16-byte aligned
     assert call(qo=A + 64) == INV                            # q_out partially over q
     assert call(ko=F + 256) == INV                           # k_out over the table
@@ -212,3 +214,30 @@ def test_vision_validation(lib):
     assert fr(A, 1024, 4, 4, 1e4, None) == UNS
     assert fr(A + 4, 64, 4, 4, 1e4, None) == UNS
     assert fr(None, 64, 4, 4, 1e4, None) == INV
+
+
+def test_residual_validation(lib):
+    S, B, O, P = A, A + (1 << 24), A + (2 << 24), A + (3 << 24)
+    blend = lambda **k: lib.muse_residual_blend(k.get("s", S), k.get("b", B), k.get("o", O), k.get("dt", BF16),  # noqa: E731
+                                                 k.get("rows", 4), k.get("hidden", 256), k.get("p", P), None)
+    gate = lambda **k: lib.muse_residual(k.get("s", S), k.get("b", B), k.get("o", O), k.get("dt", BF16),  # noqa: E731
+                                         k.get("rows", 4), k.get("hidden", 256), k.get("p", P),
+                                         k.get("t", 0.3), k.get("eps", 1e-3), None)
+    for fn in (blend, gate):
+        assert fn(rows=0) == 0
+        assert fn(dt=5) == INV
+        assert fn(rows=-1) == INV and fn(hidden=0) == INV
+        assert fn(p=None) == INV and fn(b=None) == INV
+        assert fn(s=S + 4) == UNS and fn(p=P + 4) == UNS
+        assert fn(hidden=260) == UNS                       # not a 16-byte branch row
+        assert fn(o=S + 16) == INV                         # partial overlap with the stream
+        assert fn(o=B) == INV                              # output over the branch
+    assert gate(t=0.0) == INV and gate(t=float("inf")) == INV and gate(t=-1.0) == INV
+    assert gate(eps=-0.1) == INV and gate(eps=1.5) == INV and gate(eps=float("nan")) == INV
+    ang = lambda **k: lib.muse_residual_gate_angles(k.get("g", P), k.get("th", O), k.get("hidden", 256),  # noqa: E731
+                                                    k.get("t", 0.3), k.get("eps", 1e-3), None)
+    assert ang(hidden=0) == INV and ang(g=None) == INV and ang(th=None) == INV
+    assert ang(t=0.0) == INV and ang(eps=2.0) == INV
+    assert ang(th=P + 8) == INV                            # partial overlap with the gate
+    assert ang(g=P + 2) == UNS
+    assert b"muse_residual_gate_angles" in lib.muse_last_error()
