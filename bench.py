@@ -119,7 +119,11 @@ def barrier(world: int):
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the GPU is under load."""
+    """nvidia-smi clock / throttle-reason samples while the GPU is under load.
+
+    The GPU is named by its UUID (the process may see it under another index
+    than nvidia-smi does); start() returns once the first sample has arrived,
+    so a short timed region is still covered."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -127,17 +131,32 @@ class ClockSampler:
 
     def __init__(self, index: int, period_ms: int = 20):
         self.proc = None
+        self.error = None
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        gid = str(index)
+        try:
+            u = str(torch.cuda.get_device_properties(index).uuid)
+            gid = u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:  # noqa: BLE001 - fall back to the index
+            pass
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 f"-lms={period_ms}"], stdout=self.f, stderr=subprocess.DEVNULL)
-        except (FileNotFoundError, OSError):
-            self.proc = None
+                ["nvidia-smi", f"--id={gid}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 f"-lms={period_ms}"], stdout=self.f, stderr=subprocess.PIPE)
+        except (FileNotFoundError, OSError) as e:
+            self.proc, self.error = None, str(e)
+            return
+        t0 = time.time()
+        while time.time() - t0 < 10.0 and self.proc.poll() is None:
+            if os.path.getsize(self.f.name) > 0:
+                break
+            time.sleep(0.05)
+        if self.proc.poll() is not None:
+            self.error = (self.proc.stderr.read() or b"").decode(errors="replace").strip()[:200]
 
     def stop(self):
         if self.proc is None:
-            return None
+            return {"error": self.error or "nvidia-smi not available", "samples": 0}
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -148,7 +167,7 @@ class ClockSampler:
         rows = [r for r in csv.reader(io.StringIO(self.f.read())) if len(r) >= 9]
         os.unlink(self.f.name)
         if not rows:
-            return None
+            return {"error": self.error or "no samples", "samples": 0}
         sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
         mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -455,6 +474,152 @@ def per_core_isolated(st, peak: float, flush: torch.Tensor | None, warmup: int =
     return out
 
 
+def per_core_steady(st, peak: float, reps: int, warmup: int = 3, nbytes=None, which=CORE_ORDER):
+    """Each core launched alone `reps` times back to back on the same batch,
+    with two CUDA events around the loop on the launching stream and no flush.
+    Every launch streams more than the 126 MB L2, so each one starts with its
+    predecessor's dirty output lines still to be written back and keeps the
+    programmatic-launch overlap with it, as inside the five-core step: a
+    steady-state per-core figure that neither credits writes left in L2 nor
+    charges the idle gap an event between two kernels adds."""
+    stream = torch.cuda.current_stream()
+    out = {}
+    for c in which:
+        for _ in range(warmup):
+            st.launch(c)
+        torch.cuda.synchronize()
+        torch.cuda._sleep(20_000_000)  # the host queues every launch ahead of the device
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            st.launch(c)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        nb = (nbytes or algo_bytes)(st.wl, c, st.T)
+        gbs = nb / (us * 1e-6) / 1e9
+        out[c] = {"us": round(us, 3), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+    return out
+
+
+class LaunchFloor:
+    """A 16-byte copy through the library's copy entry point: one CTA, launched
+    with programmatic dependent launch like every core, doing no real work -
+    the floor under the decode-batch latencies."""
+
+    def __init__(self):
+        self.src = torch.zeros(16, dtype=torch.uint8, device="cuda")
+        self.dst = torch.empty_like(self.src)
+        self.wl, self.T = None, 0
+
+    def launch(self, _core=None):
+        cores.stream_copy(self.src, self.dst)
+
+
+def per_config(args, peak: float, rank: int, world: int,
+               names=("thd16_h5120", "large_t32768_h8192")):
+    """The five cores on the other full-size workloads: per-core steady-state
+    figures (per_core_steady), the five-core step (K steps back to back, two
+    events), and the oracle on all host cores on a bounded sample of the same
+    batch (rank 0, one GPU)."""
+    stream = torch.cuda.current_stream()
+    reps = max(10, min(args.steps, 50))
+    out = {}
+    for name in names:
+        wl = WORKLOADS[name]
+        st = Step(wl, seed=rank)
+        steady = per_core_steady(st, peak, reps)
+        for _ in range(3):
+            for c in CORE_ORDER:
+                st.launch(c)
+        torch.cuda.synchronize()
+        torch.cuda._sleep(20_000_000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            for c in CORE_ORDER:
+                st.launch(c)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        el = allreduce_max(e0.elapsed_time(e1) / 1e3, world)
+        nb = sum(algo_bytes(wl, c, st.T) for c in CORE_ORDER)
+        rec = {"tokens": st.T, "hidden": wl.hidden, "q_heads": wl.hq, "kv_heads": wl.hkv,
+               "per_core_steady": steady,
+               "step": {"ms": round(el / reps * 1e3, 4), "tokens_per_s": round(world * st.T * reps / el, 1),
+                        "gbs": round(nb * reps / el / 1e9, 1), "frac": round(nb * reps / el / 1e9 / peak, 4),
+                        "algo_bytes": nb, "steps": reps}}
+        if rank == 0 and world == 1 and args.cpu_baseline:
+            rec["cpu_oracle_all_cores"] = cpu_baseline_threads(wl, seconds=4.0, host=st.host)
+        out[name] = rec
+        del st
+        torch.cuda.empty_cache()
+    return out
+
+
+class ResidualStep:
+    """_residual_core on the batch's shape: the FP32 stream blended with the
+    bf16 branch, in the gate form (muse_residual, temperature 0.3, eps 1e-3)
+    and the angle form (muse_residual_blend)."""
+
+    def __init__(self, wl, seed: int):
+        self.wl = wl
+        self.T = num_tokens(wl, seed)
+        dev = lambda ci: {k: v.cuda() for k, v in ci.tensors.items()}  # noqa: E731
+        self.g = dev(inputs.make_inputs(wl, "residual", seed=seed))
+        self.b = dev(inputs.make_inputs(wl, "residual_blend", seed=seed))
+        self.out = torch.empty_like(self.g["stream"])
+        self.dy = inputs.upstream_grad(wl, seed, "residual", tuple(self.out.shape), torch.float32).cuda()
+        self.dstream = torch.empty_like(self.out)
+        self.dbranch = torch.empty_like(self.g["branch"])
+        self.dparam = torch.empty(wl.hidden, dtype=torch.float32, device="cuda")
+        from gate_cores_b200 import _lib
+        self.lib = _lib
+        self.ws_bytes = _lib.muse_residual_backward_workspace_bytes(self.T, wl.hidden)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
+
+    def launch(self, core: str):
+        L, T, H = self.lib, self.T, self.wl.hidden
+        stream = torch.cuda.current_stream().cuda_stream
+        if core == "residual":
+            cores.residual(self.g["stream"], self.g["branch"], self.g["gate"], 0.3, 1e-3, out=self.out)
+        elif core == "residual_blend":
+            cores.residual_blend(self.b["stream"], self.b["branch"], self.b["theta"], out=self.out)
+        elif core == "residual_bwd":
+            L.muse_residual_backward(self.g["stream"].data_ptr(), self.g["branch"].data_ptr(), self.dy.data_ptr(),
+                                     self.dstream.data_ptr(), self.dbranch.data_ptr(), L.MUSE_DTYPE_BF16, T, H,
+                                     self.g["gate"].data_ptr(), 0.3, 1e-3, self.dparam.data_ptr(),
+                                     self.ws.data_ptr(), self.ws_bytes, stream)
+        else:
+            L.muse_residual_blend_backward(self.b["stream"].data_ptr(), self.b["branch"].data_ptr(),
+                                           self.dy.data_ptr(), self.dstream.data_ptr(), self.dbranch.data_ptr(),
+                                           L.MUSE_DTYPE_BF16, T, H, self.b["theta"].data_ptr(),
+                                           self.dparam.data_ptr(), self.ws.data_ptr(), self.ws_bytes, stream)
+
+
+def residual_bytes(wl, core: str, tokens: int) -> int:
+    """Forward: FP32 stream in and out, bf16 branch in; the gate or the angles
+    once.  Backward: the stream, the bf16 branch and dL/dout (FP32) in, the
+    stream and branch gradients out; the gate or angles and their gradient once."""
+    if core.endswith("_bwd"):
+        return 16 * wl.hidden * tokens + 8 * wl.hidden
+    return 10 * wl.hidden * tokens + 4 * wl.hidden
+
+
+def residual_timing(st, peak: float, flush: torch.Tensor, reps: int, rank: int):
+    rs = ResidualStep(st.wl, seed=rank)
+    which = ("residual", "residual_blend", "residual_bwd", "residual_blend_bwd")
+    out = {"steady": per_core_steady(rs, peak, reps, nbytes=residual_bytes, which=which),
+           "isolated": per_core_isolated(rs, peak, flush, nbytes=residual_bytes, which=which),
+           "algo_bytes": residual_bytes(st.wl, "residual", st.T),
+           "algo_bytes_bwd": residual_bytes(st.wl, "residual_bwd", st.T),
+           "kernel": "residual_blend_kernel",
+           "note": "_residual_core: FP32 stream blended with the bf16 branch per channel; residual = the "
+                   "gate form (temperature 0.3, eps 1e-3), residual_blend = the angle form; *_bwd = their "
+                   "backward with the gate / angle gradient (the kernel and the fixed-order reduction)"}
+    del rs
+    return out
+
+
 def time_copy_kernel(gib: float = 1.0, reps: int = 10) -> float:
     n = int(gib * (1 << 30)) // 16 * 16
     src = torch.empty(n, dtype=torch.uint8, device="cuda")
@@ -477,25 +642,22 @@ def time_copy_kernel(gib: float = 1.0, reps: int = 10) -> float:
 
 
 def traffic_from_profile(wl_name: str):
-    """dram read+write bytes per launch of the dominant kernel, from the committed
-    ncu summary, when the kernel sources are unchanged since the capture."""
+    """dram read+write bytes per launch of the dominant kernel from the committed
+    ncu figure (profiles/<kernel>__<workload>.json), when the kernel sources are
+    unchanged since the capture (their sha256 is stored beside the figure)."""
     import hashlib
 
-    p = os.path.join(ROOT, "profiles", f"{DOMINANT}__{wl_name}.md")
+    p = os.path.join(ROOT, "profiles", f"{DOMINANT}__{wl_name}.json")
     if not os.path.exists(p):
         return None
-    fields = {}
-    for line in open(p):
-        if line.startswith("traffic_bytes_per_launch:") or line.startswith("csrc_sha256:"):
-            k, v = line.split(":", 1)
-            fields[k.strip()] = v.strip()
+    rec = json.load(open(p))
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gate_cores_b200", "csrc")
     for f in DOMINANT_SOURCES:
         h.update(open(os.path.join(csrc, f), "rb").read())
-    if fields.get("csrc_sha256") != h.hexdigest() or "traffic_bytes_per_launch" not in fields:
+    if rec.get("csrc_sha256") != h.hexdigest() or "traffic_bytes_per_launch" not in rec:
         return None
-    return float(fields["traffic_bytes_per_launch"])
+    return float(rec["traffic_bytes_per_launch"])
 
 
 def cpu_baseline(wl, seconds: float = 12.0, chunk: int = 256):
@@ -529,7 +691,8 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def cpu_baseline_threads(wl, seconds: float = 8.0, chunk: int = 64, threads: int | None = None):
+def cpu_baseline_threads(wl, seconds: float = 8.0, chunk: int = 64, threads: int | None = None,
+                         host=None):
     """The same oracle over row chunks on all host cores: threads pull chunks
     of `chunk` tokens from a shared counter (the oracle's C routines run
     without the interpreter lock), all five cores per chunk, until `seconds`
@@ -541,7 +704,8 @@ def cpu_baseline_threads(wl, seconds: float = 8.0, chunk: int = 64, threads: int
     from tests import harness
 
     n = threads or min(os.cpu_count() or 1, 128)
-    host = {c: harness.make(wl.name, c, harness.DEFAULT_VARIANT[c]) for c in CORE_ORDER}
+    if host is None:
+        host = {c: harness.make(wl.name, c, harness.DEFAULT_VARIANT[c]) for c in CORE_ORDER}
     T = num_tokens(wl)
     lock = threading.Lock()
     state = {"next": 0, "done": 0}
@@ -579,9 +743,9 @@ def run_ours(args, world, rank, local):
     T = st.T
     stream = torch.cuda.current_stream()
     peak, peak_kind = measured_peaks()
+    sampler = ClockSampler(local) if rank == 0 else None
     copy_gbs = time_copy_kernel() if args.copy_ref else None
 
-    sampler = ClockSampler(local) if rank == 0 else None
     for _ in range(args.warmup):
         for c in CORE_ORDER:
             st.launch(c)
@@ -618,7 +782,6 @@ def run_ours(args, world, rank, local):
             ev[c][i][1].record(stream)
     torch.cuda.synchronize()
     barrier(world)
-    clocks = sampler.stop() if sampler else None
 
     per_core = {}
     for c in CORE_ORDER:
@@ -639,13 +802,20 @@ def run_ours(args, world, rank, local):
     # Each core alone on the same batch, L2 read-flushed before every launch;
     # and the decode batch (128 tokens), whose launches are latency-bound.
     flush = torch.empty(64 << 20, dtype=torch.int64, device="cuda").fill_(1)  # 512 MiB
+    steady = per_core_steady(st, peak, max(10, min(args.steps, 100)))
     isolated = per_core_isolated(st, peak, flush)
     dec = Step(WORKLOADS["decode_t128_h4096"], seed=rank)
     decode_cold = per_core_isolated(dec, peak, flush)
     decode_warm = per_core_isolated(dec, peak, None)
     decode = {c: {"us_cold_l2": decode_cold[c]["us"], "us_warm_l2": decode_warm[c]["us"]}
               for c in CORE_ORDER}
-    del dec
+    fl = LaunchFloor()
+    one = lambda wl, c, T: 32  # noqa: E731 - 16 bytes read, 16 written
+    decode["launch_floor"] = {"us_cold_l2": per_core_isolated(fl, peak, flush, nbytes=one, which=("floor",))["floor"]["us"],
+                              "us_warm_l2": per_core_isolated(fl, peak, None, nbytes=one, which=("floor",))["floor"]["us"],
+                              "note": "one-CTA 16-byte copy launched like the cores (programmatic "
+                                      "dependent launch), timed the same way"}
+    del dec, fl
     # Backward of the five cores on the same batch: each call alone (L2
     # read-flushed, median of 50) and the five back to back (K steps timed
     # with two events, as the forward step).
@@ -683,8 +853,11 @@ def run_ours(args, world, rank, local):
     fused = fused_vs_unfused(st, peak, flush)
     grouped = grouped_norm(st, peak, flush)
     vision = vision_rope_timing(peak, flush)
+    residual_core = residual_timing(st, peak, flush, max(10, min(args.steps, 100)), rank)
     del flush
     torch.cuda.empty_cache()
+    configs = per_config(args, peak, rank, world) if args.per_config else None
+    clocks = sampler.stop() if sampler else None
 
     e2e = run_e2e(st, args, world) if args.e2e else None
 
@@ -705,12 +878,15 @@ def run_ours(args, world, rank, local):
                        "l2": "no flush: each step streams %.2f GB, > 126 MB L2"
                              % (sum(algo_bytes(wl, c, T) for c in CORE_ORDER) / 1e9)},
             "per_core": per_core,
+            "per_core_steady": steady,
             "per_core_isolated": isolated,
             "decode_t128_h4096_latency": decode,
             "backward": backward,
             "fused_residual_prenorm": fused,
             "per_expert_norm": grouped,
             "vision_rope": vision,
+            "residual_core": residual_core,
+            "per_config": configs,
             "roofline": roofline,
             "copy_kernel_gbs": None if copy_gbs is None else round(copy_gbs, 1),
             "e2e": e2e,
@@ -719,9 +895,14 @@ def run_ours(args, world, rank, local):
             "gpu_launches": len(CORE_ORDER) * args.steps,
             "kernel_timing": "per_core and roofline: a second pass of the same K steps with "
                              "CUDA events around each launch (the timed region has none); "
+                             "per_core_steady: each core alone, launched back to back with two "
+                             "events around the loop, no flush (each launch drains its "
+                             "predecessor's dirty L2 lines, as in the step); "
                              "per_core_isolated: each core alone, median of 50 launches, "
-                             "a 512 MiB read pass (clean L2) before each; decode latency: "
-                             "median of 50, cold (read-flushed) and warm L2",
+                             "a 512 MiB read pass before each (a clean, cold L2 - credits the "
+                             "output lines still dirty in L2 when the kernel ends); decode "
+                             "latency: median of 50, cold (read-flushed) and warm L2, beside a "
+                             "launch floor",
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -730,36 +911,61 @@ def run_ours(args, world, rank, local):
 def run_e2e(st: Step, args, world):
     """Same metric through the public API with host buffers: every step copies
     its inputs from pinned host memory, runs the five cores and reads every
-    output back to pinned host memory."""
-    pinned_in = [(dev, torch.empty(dev.shape, dtype=dev.dtype, pin_memory=True).copy_(dev.cpu()))
-                 for _, dev in st.input_tensors()]
-    pinned_out = [(dev, torch.empty(dev.shape, dtype=dev.dtype, pin_memory=True))
-                  for dev in st.output_tensors()]
-    h2d = sum(h.numel() * h.element_size() for _, h in pinned_in)
-    d2h = sum(h.numel() * h.element_size() for _, h in pinned_out)
+    output back to pinned host memory.  Two sets of device and host buffers
+    and three streams (upload, compute, download) let one step's download
+    overlap the next step's upload and compute - PCIe carries both directions
+    at once - with events ordering each set's reuse."""
+    rank = int(os.environ.get("RANK", "0"))
+    sets = [st, Step(st.wl, seed=rank)]
+    pin_in = [[(dev, torch.empty(dev.shape, dtype=dev.dtype, pin_memory=True).copy_(dev.cpu()))
+               for _, dev in s_.input_tensors()] for s_ in sets]
+    pin_out = [[(dev, torch.empty(dev.shape, dtype=dev.dtype, pin_memory=True)) for dev in s_.output_tensors()]
+               for s_ in sets]
+    h2d = sum(h.numel() * h.element_size() for _, h in pin_in[0])
+    d2h = sum(h.numel() * h.element_size() for _, h in pin_out[0])
     steps = max(3, min(args.steps, 20))
+    up, comp, down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    up_done, comp_done, down_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    for k in range(2):  # every event recorded once before its first wait
+        for e in (up_done[k], comp_done[k], down_done[k]):
+            e.record(comp)
 
-    def one():
-        for dev, h in pinned_in:
-            dev.copy_(h, non_blocking=True)
-        for c in CORE_ORDER:
-            st.launch(c)
-        for dev, h in pinned_out:
-            h.copy_(dev, non_blocking=True)
+    def one(k):
+        j = k % 2
+        with torch.cuda.stream(up):
+            up.wait_event(comp_done[j])          # the set's previous inputs are consumed
+            for dev, h in pin_in[j]:
+                dev.copy_(h, non_blocking=True)
+            up_done[j].record(up)
+        with torch.cuda.stream(comp):
+            comp.wait_event(up_done[j])
+            comp.wait_event(down_done[j])        # the set's previous outputs are read back
+            for c in CORE_ORDER:
+                sets[j].launch(c)
+            comp_done[j].record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(comp_done[j])
+            for dev, h in pin_out[j]:
+                h.copy_(dev, non_blocking=True)
+            down_done[j].record(down)
 
-    for _ in range(2):
-        one()
+    for k in range(2):
+        one(k)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        one()
-    e1.record()
+    e0.record(up)
+    for k in range(steps):
+        one(k)
+    up.wait_stream(down)
+    e1.record(up)
     torch.cuda.synchronize()
     el = allreduce_max(e0.elapsed_time(e1) / 1e3, world)
+    del sets[1]
     return {"value": round(world * st.T * steps / el, 1), "unit": "tokens/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "overlap": "two buffer sets; upload, compute and download on three streams"}
 
 
 # ------------------------------------------------------------------ reference arm
@@ -811,15 +1017,17 @@ def run_reference(args, world, rank):
 
 def profile_pass(args):
     """Each forward core, each backward core, core 5 fused with the next
-    pre-norm, the per-expert core 1 and the vision RoPE, the sequence launched
-    twice on the workload's batch: a short, fixed launch sequence for an ncu
-    capture (16 table launches first, then 17 kernel launches per pass; skip
-    the table and the first pass to capture warm ones)."""
+    pre-norm, the per-expert core 1, the vision RoPE and the two _residual_core
+    forms with their backward, the sequence launched twice on the workload's
+    batch: a short, fixed launch sequence for an ncu capture (16 table launches
+    first, then 23 kernel launches per pass; skip the table and the first pass
+    to capture warm ones)."""
     wl = WORKLOADS[args.workload]
     st = Step(wl, seed=0)
     bst = BwdStep(st, seed=0)
     fused, _ = fused_calls(st)
     grouped = grouped_call(st)
+    rs = ResidualStep(wl, seed=0)
     _, vision = vision_call()  # 16 table launches before the passes
     for _ in range(2):
         for c in CORE_ORDER:
@@ -829,9 +1037,12 @@ def profile_pass(args):
         fused()
         grouped()
         vision()
+        for c in ("residual", "residual_blend", "residual_bwd", "residual_blend_bwd"):
+            rs.launch(c)
     torch.cuda.synchronize()
     print("profile pass: 16 vision-table launches, then 2 x (5 forward + 5 backward calls, fused core 5 + "
-          "pre-norm, per-expert core 1, vision RoPE) on " + wl.name, file=sys.stderr)
+          "pre-norm, per-expert core 1, vision RoPE, residual gate and angle forms and their backward) on "
+          + wl.name, file=sys.stderr)
 
 
 def main():
@@ -844,6 +1055,8 @@ def main():
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-copy-ref", dest="copy_ref", action="store_false")
+    ap.add_argument("--no-per-config", dest="per_config", action="store_false",
+                    help="skip the packed-THD and large-hidden workloads")
     ap.add_argument("--profile-pass", action="store_true",
                     help="for profilers: launch every forward and backward core twice on the batch "
                          "(no timing, no JSON line) and exit")
