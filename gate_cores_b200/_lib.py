@@ -36,6 +36,7 @@ EXPORTS = (
     "muse_vision_rope", "muse_vision_rope_frequencies", "muse_rms_norm_stall_probe",
     "muse_residual_blend", "muse_residual", "muse_residual_gate_angles",
     "muse_residual_backward_workspace_bytes", "muse_residual_blend_backward", "muse_residual_backward",
+    "muse_residual_blend_rms_norm",
 )
 
 
@@ -77,6 +78,7 @@ def load() -> ctypes.CDLL:
         lib.muse_residual.argtypes = [P, P, P, c_int, i64, i64, P, f32, f32, P]
         lib.muse_residual_gate_angles.argtypes = [P, P, i64, f32, f32, P]
         lib.muse_residual_backward_workspace_bytes.argtypes = [i64, i64]
+        lib.muse_residual_blend_rms_norm.argtypes = [P, P, P, P, c_int, c_int, i64, i64, P, P, f32, f32, P]
         lib.muse_residual_blend_backward.argtypes = [P, P, P, P, P, c_int, i64, i64, P, P, P, ctypes.c_size_t, P]
         lib.muse_residual_backward.argtypes = [P, P, P, P, P, c_int, i64, i64, P, f32, f32, P, P,
                                                ctypes.c_size_t, P]
@@ -279,6 +281,12 @@ def muse_residual_backward(stream_in, branch, dstream_out, dstream_in, dbranch, 
                            temperature, eps, dgate, workspace, workspace_bytes, stream) -> None:
     _call("muse_residual_backward", stream_in, branch, dstream_out, dstream_in, dbranch, branch_dtype, rows, hidden,
           gate, temperature, eps, dgate, workspace, workspace_bytes, stream)
+
+
+def muse_residual_blend_rms_norm(stream_in, branch, stream_out, y, branch_dtype, y_dtype, rows, hidden, theta,
+                                 next_gain, next_gain_offset, next_eps, stream) -> None:
+    _call("muse_residual_blend_rms_norm", stream_in, branch, stream_out, y, branch_dtype, y_dtype, rows, hidden,
+          theta, next_gain, next_gain_offset, next_eps, stream)
 
 
 def muse_residual_gate_angles(gate, theta, hidden, temperature, eps, stream) -> None:

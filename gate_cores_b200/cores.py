@@ -224,6 +224,26 @@ def residual(stream_in: torch.Tensor, branch: torch.Tensor, gate: torch.Tensor, 
     return h_out
 
 
+def residual_blend_rms_norm(stream_in: torch.Tensor, branch: torch.Tensor, theta: torch.Tensor,
+                            next_gain: torch.Tensor | None = None, next_gain_offset: float = 0.0,
+                            next_eps: float = 1e-6, y_dtype=torch.float32, out: torch.Tensor | None = None,
+                            y: torch.Tensor | None = None, stream=None):
+    """_residual_core (angle form) and the next sublayer's RMS pre-norm of the
+    new stream in one pass.  Returns (stream_out, y)."""
+    hidden, rows = _residual_args(stream_in, branch, theta, "theta")
+    _cuda(next_gain, out, y)
+    h_out = _out_like(stream_in, out)
+    if y is None:
+        y = torch.empty(stream_in.shape, dtype=y_dtype, device=stream_in.device)
+    elif y.shape != stream_in.shape or y.dtype != y_dtype or not y.is_contiguous():
+        raise ValueError("y must be contiguous, shaped like the stream, in y_dtype")
+    g2 = _gain(next_gain)
+    _lib.muse_residual_blend_rms_norm(stream_in.data_ptr(), branch.data_ptr(), h_out.data_ptr(), y.data_ptr(),
+                                      _dtype(branch), _dtype(y), rows, hidden, theta.contiguous().data_ptr(),
+                                      _ptr(g2), next_gain_offset, next_eps, _stream(stream))
+    return h_out, y
+
+
 def residual_gate_angles(gate: torch.Tensor, temperature: float = 0.3, eps: float = 1e-3,
                          out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Blend angle per channel from the learned gate: atan2(s, c) (FP32 [H])."""

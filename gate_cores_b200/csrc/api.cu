@@ -545,7 +545,8 @@ namespace {
 // The backward's row blocks at most, for either branch dtype: its CTAs are
 // min(256, vectors per row rounded up to 32) threads, so at most
 // min(32, 2048 / threads) of them reside on an SM; the row blocks are those
-// resident CTAs over the column blocks, and no more than the row tiles of 4.
+// resident CTAs over the column blocks, and no more than the row tiles of 4
+// (an upper bound: the kernel takes tiles of 8 rows).
 int64_t residual_bwd_parts_cap(int64_t rows, int64_t hidden) {
     int64_t cap = 0;
     for (int vec : {8, 4}) {
@@ -1007,6 +1008,55 @@ muse_status muse_norm_residual_rms_norm(const float* stream_in, const void* bran
     a.y_f32 = y_dtype == MUSE_DTYPE_F32 ? 1 : 0;
     const muse::RowOp op = input_scale ? muse::RowOp::kResidualISPre : muse::RowOp::kResidualPre;
     return from_cuda(muse::launch_row(branch_dtype, op, a, stream), name);
+}
+
+muse_status muse_residual_blend_rms_norm(const float* stream_in, const void* branch, float* stream_out, void* y,
+                                         muse_dtype branch_dtype, muse_dtype y_dtype, int64_t rows, int64_t hidden,
+                                         const float* theta, const float* next_gain, float next_gain_offset,
+                                         float next_eps, cudaStream_t stream) {
+    const char* name = "muse_residual_blend_rms_norm";
+    if (!valid_dtype(branch_dtype) || !valid_dtype(y_dtype))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: unknown dtype", name);
+    if (rows < 0 || hidden <= 0)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: rows=%lld hidden=%lld", name, (long long)rows, (long long)hidden);
+    if (!finite(next_eps) || next_eps < 0.0f || !finite(next_gain_offset))
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: next_eps must be finite and >= 0, next_gain_offset finite", name);
+    if (rows == 0) return MUSE_OK;
+    if (!stream_in || !branch || !stream_out || !theta || !y)
+        return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: null stream_in/branch/stream_out/theta/y", name);
+    const int64_t es = elem_size(branch_dtype), ys = elem_size(y_dtype);
+    if (!aligned(stream_in, 16) || !aligned(stream_out, 16) || !aligned(branch, 16) || !aligned(y, 16) ||
+        (hidden * es) % 16 || (hidden * ys) % 16)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: pointers and row widths must be 16-byte multiples", name);
+    if (!aligned(theta, 16) || (next_gain && !aligned(next_gain, 16)))
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: theta / next_gain not 16-byte aligned", name);
+    if (hidden / vec_elems(branch_dtype) > 1024)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: rows of more than 1024 16-byte branch vectors", name);
+    if (y_dtype != MUSE_DTYPE_F32 && y_dtype != branch_dtype)
+        return fail(MUSE_ERR_UNSUPPORTED, "%s: y must be FP32 or in the branch dtype", name);
+    const Span sin_ = span(stream_in, rows, hidden, hidden, 4), sout = span(stream_out, rows, hidden, hidden, 4);
+    const Span sb = span(branch, rows, hidden, hidden, es), st = span(theta, 1, hidden, hidden, 4);
+    const Span sy = span(y, rows, hidden, hidden, ys);
+    const Span sg2 = span(next_gain, next_gain ? 1 : 0, hidden, hidden, 4);
+    bool bad = bad_alias(sout, sin_, true) || any_overlap(sout, {sb, st, sg2, sy});
+    bad = bad || (!same_span(sy, sb) && overlap(sy, sb)) || any_overlap(sy, {sin_, st, sg2});
+    if (bad) return fail(MUSE_ERR_INVALID_ARGUMENT, "%s: an output partially overlaps an input", name);
+    muse::RowArgs a{};
+    a.x = branch;
+    a.y = y;
+    a.stream_in = stream_in;
+    a.stream_out = stream_out;
+    a.theta = theta;
+    a.rows = rows;
+    a.x_stride = hidden;
+    a.y_stride = hidden;
+    a.s_in_stride = a.s_out_stride = hidden;
+    a.width = (int32_t)hidden;
+    a.gain2 = next_gain;
+    a.gain2_offset = next_gain_offset;
+    a.eps2 = next_eps;
+    a.y_f32 = y_dtype == MUSE_DTYPE_F32 ? 1 : 0;
+    return from_cuda(muse::launch_row(branch_dtype, muse::RowOp::kBlendPre, a, stream), name);
 }
 
 muse_status muse_device_error(unsigned int* flags, int clear) {

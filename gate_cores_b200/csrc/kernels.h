@@ -16,6 +16,7 @@ enum class RowOp : int {
     kResidualPre = 5,    // core 5 (gain after) + the next sublayer's RMS pre-norm of the new stream
     kResidualISPre = 6,  // core 5 (gain before) + the next sublayer's RMS pre-norm
     kRmsGrouped = 7,     // core 1 with per-expert gains: rows of group g use gain row g
+    kBlendPre = 8,       // _residual_core (angle form, no branch norm) + the next sublayer's RMS pre-norm
 };
 
 // One row = one token's `width` elements.  Strides in elements.
@@ -34,7 +35,7 @@ struct RowArgs {
     int32_t rows_per_cta;   // set by the launcher (register-staged row kernels)
     float gain_offset;
     float eps;
-    // kResidualPre / kResidualISPre: y = cast((h' r(h')) (gain2 + gain2_offset))
+    // kResidualPre / kResidualISPre / kBlendPre: y = cast((h' r(h')) (gain2 + gain2_offset))
     // into `y` (row stride y_stride), FP32 when y_f32 else the branch dtype
     const float* gain2;     // may be null
     float gain2_offset;

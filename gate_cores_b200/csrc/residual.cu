@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(256) residual_gate_angles_kernel(const __grid_
 // accumulated over the thread's rows in registers and written as one partial
 // row per CTA row-block into the caller's workspace (a fixed-order reduction
 // follows).
-constexpr int kBlendBwdRows = 4;
+constexpr int kBlendBwdRows = 8;  // rows in flight per thread (4: 14% slower, 2: 16% slower)
 
 template <typename T, bool GATE>
 __global__ void __launch_bounds__(256) residual_blend_bwd_kernel(const __grid_constant__ ResidualArgs a) {

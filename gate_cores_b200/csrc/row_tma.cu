@@ -40,12 +40,18 @@ namespace {
 using namespace pipe;
 
 __host__ __device__ constexpr bool t_is_residual(RowOp op) {
-    return op == RowOp::kResidual || op == RowOp::kResidualIS || op == RowOp::kResidualPre || op == RowOp::kResidualISPre;
+    return op == RowOp::kResidual || op == RowOp::kResidualIS || op == RowOp::kResidualPre ||
+           op == RowOp::kResidualISPre || op == RowOp::kBlendPre;
 }
+// _residual_core fused with the next pre-norm: core 5's fused pipeline with
+// the branch entering the blend as it is (no branch norm, no cast).
+__host__ __device__ constexpr bool t_blend(RowOp op) { return op == RowOp::kBlendPre; }
 __host__ __device__ constexpr bool t_scales_first(RowOp op) {
     return op == RowOp::kInputScale || op == RowOp::kResidualIS || op == RowOp::kResidualISPre;
 }
-__host__ __device__ constexpr bool t_prenorm(RowOp op) { return op == RowOp::kResidualPre || op == RowOp::kResidualISPre; }
+__host__ __device__ constexpr bool t_prenorm(RowOp op) {
+    return op == RowOp::kResidualPre || op == RowOp::kResidualISPre || op == RowOp::kBlendPre;
+}
 // Ops whose stage carries the FP32 stream row besides the activation row (core 5).
 __host__ __device__ constexpr bool t_f32_row(RowOp op) { return t_is_residual(op); }
 // Per-expert core 1: each CTA takes a contiguous run of rows, so consecutive
@@ -367,8 +373,11 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
                 acc[q & 1] = f2_fma(x[i][q], x[i][q], acc[q & 1]);
             }
         }
-        const float part = f2_sum(acc[0]) + f2_sum(acc[1]);
-        const float r = inv_rms_fast(consumer_sum(part, red, bank, ncons), inv_width, a.eps);
+        float r = 1.0f;
+        if constexpr (!t_blend(OP)) {  // the branch norm (the blend alone has none)
+            const float part = f2_sum(acc[0]) + f2_sum(acc[1]);
+            r = inv_rms_fast(consumer_sum(part, red, bank, ncons), inv_width, a.eps);
+        }
         const f32x2 r2 = f2_make(r, r);
 
         if constexpr (OP == RowOp::kRms || OP == RowOp::kInputScale || OP == RowOp::kNormGate ||
@@ -406,7 +415,8 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
                 for (int q = 0; q < P; ++q) {
                     f32x2 t = f2_mul(x[i][q], r2);  // z r when the gain came first
                     if constexpr (!t_scales_first(OP) && HAS_GAIN) t = f2_mul(t, w[i][q]);
-                    const f32x2 nb = round_pair<T>(t);  // cast back to the branch dtype
+                    // cast back to the branch dtype; the blend alone takes the branch as read
+                    const f32x2 nb = t_blend(OP) ? x[i][q] : round_pair<T>(t);
                     o[q] = f2_fma(cth[i][q], h[q], f2_mul(sth[i][q], nb));
                     if constexpr (t_prenorm(OP)) {
                         hs[i][q] = o[q];
@@ -449,21 +459,23 @@ __device__ __forceinline__ void row_tma_body(const RowArgs& a) {
 }
 
 // One entry symbol per core, so launch lists and profiles name the core.
-// One-slot instances keep a register budget for two resident CTAs of up to
-// 544 threads (core 5 at 4096 columns: 2 x 544 threads; one CTA per SM
-// measured 20% slower).
+// Cores 1, 2, 4 and per-expert core 1 use at most 256 consumers (288 threads)
+// and keep a register budget for four resident CTAs up to two slots per
+// thread (two at four slots); core 5's one-slot instances (up to 544 threads)
+// keep one for two resident CTAs.  One CTA fewer per SM measured 8-20% slower.
+constexpr int kRowThreads = 256 + 32;
 template <typename T, int VPT, bool G, int S>
-__global__ void __launch_bounds__(512 + 32, VPT == 1 ? 2 : 1) rms_norm_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(kRowThreads, VPT <= 2 ? 4 : 2) rms_norm_kernel(const __grid_constant__ RowArgs a) {
     pdl_begin();
     row_tma_body<T, RowOp::kRms, VPT, G, S>(a);
 }
 template <typename T, int VPT, bool G, int S>
-__global__ void __launch_bounds__(512 + 32, VPT == 1 ? 2 : 1) input_scale_norm_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(kRowThreads, VPT <= 2 ? 4 : 2) input_scale_norm_kernel(const __grid_constant__ RowArgs a) {
     pdl_begin();
     row_tma_body<T, RowOp::kInputScale, VPT, G, S>(a);
 }
 template <typename T, int VPT, bool G, int S>
-__global__ void __launch_bounds__(512 + 32, VPT == 1 ? 2 : 1) output_norm_gate_row_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(kRowThreads, VPT <= 2 ? 4 : 2) output_norm_gate_row_kernel(const __grid_constant__ RowArgs a) {
     pdl_begin();
     row_tma_body<T, RowOp::kNormGate, VPT, G, S>(a);
 }
@@ -478,7 +490,7 @@ __global__ void __launch_bounds__(512 + 32, VPT == 1 ? 2 : 1) norm_residual_inpu
     row_tma_body<T, RowOp::kResidualIS, VPT, G, S>(a);
 }
 template <typename T, int VPT, bool G, int S>
-__global__ void __launch_bounds__(512 + 32, VPT == 1 ? 2 : 1) rms_norm_grouped_kernel(const __grid_constant__ RowArgs a) {
+__global__ void __launch_bounds__(kRowThreads, VPT <= 2 ? 4 : 2) rms_norm_grouped_kernel(const __grid_constant__ RowArgs a) {
     pdl_begin();
     row_tma_body<T, RowOp::kRmsGrouped, VPT, G, S>(a);
 }
@@ -493,6 +505,12 @@ __global__ void __launch_bounds__(512 + 32, VPT == 1 ? 2 : 1) norm_residual_inpu
     row_tma_body<T, RowOp::kResidualISPre, VPT, G, S>(a);
 }
 
+template <typename T, int VPT, bool G, int S>
+__global__ void __launch_bounds__(512 + 32, VPT == 1 ? 2 : 1) residual_blend_prenorm_kernel(const __grid_constant__ RowArgs a) {
+    pdl_begin();
+    row_tma_body<T, RowOp::kBlendPre, VPT, G, S>(a);
+}
+
 template <typename T, RowOp OP, int VPT, bool G, int S>
 constexpr auto row_tma_kernel() {
     if constexpr (OP == RowOp::kRms) return rms_norm_kernel<T, VPT, G, S>;
@@ -502,6 +520,7 @@ constexpr auto row_tma_kernel() {
     else if constexpr (OP == RowOp::kResidualIS) return norm_residual_input_scale_kernel<T, VPT, G, S>;
     else if constexpr (OP == RowOp::kResidualPre) return norm_residual_prenorm_kernel<T, VPT, G, S>;
     else if constexpr (OP == RowOp::kRmsGrouped) return rms_norm_grouped_kernel<T, VPT, G, S>;
+    else if constexpr (OP == RowOp::kBlendPre) return residual_blend_prenorm_kernel<T, VPT, G, S>;
     else return norm_residual_input_scale_prenorm_kernel<T, VPT, G, S>;
 }
 
@@ -541,6 +560,7 @@ cudaError_t launch_row_tma_v(const RowArgs& a, int nvec, int stages, cudaStream_
 // constants live in registers).
 constexpr uint32_t kRingMaxBytes = 200 * 1024;
 constexpr int kConsumers = 256;
+static_assert(kRowThreads == kConsumers + 32, "launch bounds of the non-residual row kernels");
 
 template <typename T, RowOp OP>
 cudaError_t launch_row_op(const RowArgs& a, cudaStream_t s) {
@@ -578,6 +598,7 @@ cudaError_t launch_row_t2(RowOp op, const RowArgs& a, cudaStream_t s) {
         case RowOp::kResidualPre: return launch_row_op<T, RowOp::kResidualPre>(a, s);
         case RowOp::kResidualISPre: return launch_row_op<T, RowOp::kResidualISPre>(a, s);
         case RowOp::kRmsGrouped: return launch_row_op<T, RowOp::kRmsGrouped>(a, s);
+        case RowOp::kBlendPre: return launch_row_op<T, RowOp::kBlendPre>(a, s);
     }
     return cudaErrorInvalidValue;
 }

@@ -218,6 +218,24 @@ muse_status muse_residual_backward(const float* stream_in, const void* branch, c
                                    void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * _residual_core (angle form) fused with the next sublayer's pre-norm, as
+ * muse_norm_residual_rms_norm is for core 5: in one pass,
+ *   stream_out = muse_residual_blend(stream_in, branch, theta)  (the same values),
+ *   y = cast_y((stream_out r(stream_out)) w2),  w2 = next_gain + next_gain_offset
+ *       (no multiply when next_gain is NULL), r with next_eps, FP32 arithmetic on
+ *       the FP32 values written to stream_out,
+ * so the new stream is not read back.  y [rows, hidden] contiguous, FP32 or
+ * the branch dtype; y may be the very memory of branch when the dtypes match;
+ * stream_out may be stream_in.  Rows up to 1024 16-byte branch vectors, else
+ * MUSE_ERR_UNSUPPORTED.  A gate-form caller converts its gate with
+ * muse_residual_gate_angles first.
+ */
+muse_status muse_residual_blend_rms_norm(const float* stream_in, const void* branch, float* stream_out, void* y,
+                                         muse_dtype branch_dtype, muse_dtype y_dtype, int64_t rows, int64_t hidden,
+                                         const float* theta, const float* next_gain, float next_gain_offset,
+                                         float next_eps, cudaStream_t stream);
+
+/*
  * The blend angle of each channel from the learned gate under the reading of
  * muse_residual: theta[j] = atan2(s_j, c_j) in [0, pi/2].  It turns the
  * page's (gate, temperature, residual_eps) of _norm_residual_core into the
