@@ -325,12 +325,34 @@ def fused_calls(st: "Step"):
     return fused, unfused
 
 
-def fused_vs_unfused(st: "Step", peak: float, flush: torch.Tensor, warmup: int = 10, reps: int = 50):
+def blend_fused_calls(st: "Step", seed: int = 0):
+    """(fused, unfused): _residual_core (angle form) with the next sublayer's
+    pre-norm in one call, and the blend then core 1 on its output."""
+    wl = st.wl
+    ci = inputs.make_inputs(wl, "residual_blend", seed=seed)
+    h_in, b, th = (ci.tensors[k].cuda() for k in ("stream", "branch", "theta"))
+    g2, off2 = inputs.gain(wl, 0, "gain_next", True)
+    g2 = g2.cuda()
+    h, y = torch.empty_like(h_in), torch.empty_like(h_in)
+
+    def fused():
+        cores.residual_blend_rms_norm(h_in, b, th, next_gain=g2, next_gain_offset=off2, next_eps=1e-6,
+                                      out=h, y=y)
+
+    def unfused():
+        cores.residual_blend(h_in, b, th, out=h)
+        cores.rms_norm(h, g2, off2, 1e-6, out=y)
+
+    return fused, unfused
+
+
+def fused_vs_unfused(st: "Step", peak: float, flush: torch.Tensor, warmup: int = 10, reps: int = 50,
+                     calls=None, note=None):
     """Core 5 fused with the next sublayer's pre-norm (FP32 y) against core 5
     followed by core 1 on the new FP32 stream: median of `reps`, each call
     pair timed with events around both launches, L2 read-flushed before each."""
     T, H = st.T, st.wl.hidden
-    fused, unfused = fused_calls(st)
+    fused, unfused = calls if calls is not None else fused_calls(st)
     stream = torch.cuda.current_stream()
     out = {}
     for name, fn in (("fused", fused), ("unfused", unfused)):
@@ -352,8 +374,8 @@ def fused_vs_unfused(st: "Step", peak: float, flush: torch.Tensor, warmup: int =
     out["fused_frac"] = round(out["fused_gbs"] / peak, 4)
     out["algo_bytes_fused"] = nb
     out["algo_bytes_unfused"] = 18 * H * T + 16 * H
-    out["note"] = ("core 5 + the next sublayer's RMS pre-norm of the new FP32 stream (FP32 y) in one "
-                   "pass, against muse_norm_residual then muse_rms_norm on its output")
+    out["note"] = note or ("core 5 + the next sublayer's RMS pre-norm of the new FP32 stream (FP32 y) in one "
+                           "pass, against muse_norm_residual then muse_rms_norm on its output")
     return out
 
 
@@ -437,9 +459,24 @@ def grouped_norm(st: "Step", peak: float, flush: torch.Tensor, experts: int = 64
     torch.cuda.synchronize()
     us = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
     nb = 4 * H * T + 4 * H * experts + 4 * (experts + 1)
+    # launched back to back (steady state), as per_core_steady
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    torch.cuda._sleep(20_000_000)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us_st = e0.elapsed_time(e1) * 1e3 / reps
     return {"us": round(us, 3), "gbs": round(nb / (us * 1e-6) / 1e9, 1),
-            "frac": round(nb / (us * 1e-6) / 1e9 / peak, 4), "experts": experts, "algo_bytes": nb,
-            "note": "muse_rms_norm_grouped: rows grouped by expert, each group with its own FP32 gain row"}
+            "frac": round(nb / (us * 1e-6) / 1e9 / peak, 4),
+            "steady_us": round(us_st, 3), "steady_frac": round(nb / (us_st * 1e-6) / 1e9 / peak, 4),
+            "experts": experts, "algo_bytes": nb,
+            "note": "muse_rms_norm_grouped: rows grouped by expert, each group with its own FP32 gain row; "
+                    "us alone with a read-flushed L2, steady_us launched back to back"}
 
 
 def per_core_isolated(st, peak: float, flush: torch.Tensor | None, warmup: int = 10,
@@ -851,6 +888,9 @@ def run_ours(args, world, rank, local):
                         "theta gradients reduced through the caller's workspace"}
     del bst
     fused = fused_vs_unfused(st, peak, flush)
+    fused_blend = fused_vs_unfused(st, peak, flush, calls=blend_fused_calls(st, rank),
+                                   note="_residual_core (angle form) + the next sublayer's RMS pre-norm (FP32 y) in "
+                                        "one pass, against muse_residual_blend then muse_rms_norm on its output")
     grouped = grouped_norm(st, peak, flush)
     vision = vision_rope_timing(peak, flush)
     residual_core = residual_timing(st, peak, flush, max(10, min(args.steps, 100)), rank)
@@ -883,6 +923,7 @@ def run_ours(args, world, rank, local):
             "decode_t128_h4096_latency": decode,
             "backward": backward,
             "fused_residual_prenorm": fused,
+            "fused_residual_blend_prenorm": fused_blend,
             "per_expert_norm": grouped,
             "vision_rope": vision,
             "residual_core": residual_core,
@@ -1018,14 +1059,16 @@ def run_reference(args, world, rank):
 def profile_pass(args):
     """Each forward core, each backward core, core 5 fused with the next
     pre-norm, the per-expert core 1, the vision RoPE and the two _residual_core
-    forms with their backward, the sequence launched twice on the workload's
-    batch: a short, fixed launch sequence for an ncu capture (16 table launches
-    first, then 23 kernel launches per pass; skip the table and the first pass
-    to capture warm ones)."""
+    forms with their backward and the blend fused with the next pre-norm, the
+    sequence launched twice on the workload's batch: a short, fixed launch
+    sequence for an ncu capture (16 table launches first, then 24 kernel
+    launches per pass; skip the table and the first pass to capture warm
+    ones)."""
     wl = WORKLOADS[args.workload]
     st = Step(wl, seed=0)
     bst = BwdStep(st, seed=0)
     fused, _ = fused_calls(st)
+    fused_blend, _ = blend_fused_calls(st)
     grouped = grouped_call(st)
     rs = ResidualStep(wl, seed=0)
     _, vision = vision_call()  # 16 table launches before the passes
@@ -1039,9 +1082,11 @@ def profile_pass(args):
         vision()
         for c in ("residual", "residual_blend", "residual_bwd", "residual_blend_bwd"):
             rs.launch(c)
+        fused_blend()
     torch.cuda.synchronize()
     print("profile pass: 16 vision-table launches, then 2 x (5 forward + 5 backward calls, fused core 5 + "
-          "pre-norm, per-expert core 1, vision RoPE, residual gate and angle forms and their backward) on "
+          "pre-norm, per-expert core 1, vision RoPE, residual gate and angle forms, their backward and the "
+          "fused blend + pre-norm) on "
           + wl.name, file=sys.stderr)
 
 
