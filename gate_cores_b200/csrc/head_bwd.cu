@@ -282,7 +282,10 @@ __global__ void __launch_bounds__(256, 3) qk_norm_rope_bwd_kernel(const __grid_c
 
     const bool vok = !TAIL || sub < nvec;
     const uint32_t voff = (uint32_t)sub * 16u;
+    // v2 with bf16 Q/K: the rounded cos / sin also as bf16 pairs
+    constexpr bool BF2 = ROPE && V2 && std::is_same<T, __nv_bfloat16>::value;
     f32x2 c2[H], s2[H], n2[H];
+    uint32_t cb[BF2 ? H : 1], sb[BF2 ? H : 1], nb2[BF2 ? H : 1];
     auto set_angles = [&](int64_t t) {
         if constexpr (ROPE) {
             const float pos = (float)token_position(a, t);
@@ -301,6 +304,11 @@ __global__ void __launch_bounds__(256, 3) qk_norm_rope_bwd_kernel(const __grid_c
                 c2[j] = f2_make(c0, c1);
                 s2[j] = f2_make(s0, s1);
                 n2[j] = f2_make(-s0, -s1);
+                if constexpr (BF2) {  // exact: the values are bf16 already
+                    cb[j] = pack_bf16x2(c0, c1);
+                    sb[j] = pack_bf16x2(s0, s1);
+                    nb2[j] = pack_bf16x2(-s0, -s1);
+                }
             }
         }
     };
@@ -313,20 +321,35 @@ __global__ void __launch_bounds__(256, 3) qk_norm_rope_bwd_kernel(const __grid_c
         for (int b = 0; b < BATCH; ++b) {
             f32x2 xe[H], xo[H], de[H], dd[H];
             qk::to_eo<T>(xv[b], xe, xo);
-            qk::to_eo<T>(gv[b], de, dd);
+            if constexpr (!BF2) qk::to_eo<T>(gv[b], de, dd);
             f32x2 ss = f2_make(0.0f, 0.0f), cd = f2_make(0.0f, 0.0f);
 #pragma unroll
             for (int j = 0; j < H; ++j) {
-                f32x2 me = de[j], mo = dd[j];
-                if constexpr (ROPE && V2) {  // bf16 products, their sums rounded below
-                    me = f2_add(round_pair<T>(f2_mul(de[j], c2[j])), round_pair<T>(f2_mul(dd[j], s2[j])));
-                    mo = f2_add(round_pair<T>(f2_mul(dd[j], c2[j])), round_pair<T>(f2_mul(de[j], n2[j])));
-                } else if constexpr (ROPE) {  // R^T: (c dy0 + s dy1, -s dy0 + c dy1)
-                    me = f2_fma(dd[j], s2[j], f2_mul(de[j], c2[j]));
-                    mo = f2_fma(de[j], n2[j], f2_mul(dd[j], c2[j]));
+                f32x2 me, mo;
+                if constexpr (BF2) {
+                    // v2, bf16 Q/K: the same bf16 products and sums as below on
+                    // bf16 pairs (first and second members of rotation pairs
+                    // 2j, 2j + 1 of the incoming gradient), already bf16
+                    static_assert(H == 2, "a 16-byte vector holds 4 rotation pairs of bf16");
+                    const uint32_t w0 = j == 0 ? gv[b].x : gv[b].z, w1 = j == 0 ? gv[b].y : gv[b].w;
+                    const uint32_t e = qk::lo_halves(w0, w1), o = qk::hi_halves(w0, w1);
+                    const uint32_t me_b = qk::bf2_add(qk::bf2_mul(e, cb[j]), qk::bf2_mul(o, sb[j]));
+                    const uint32_t mo_b = qk::bf2_add(qk::bf2_mul(o, cb[j]), qk::bf2_mul(e, nb2[j]));
+                    me = f2_make(bf16_lo(me_b), bf16_hi(me_b));
+                    mo = f2_make(bf16_lo(mo_b), bf16_hi(mo_b));
+                } else {
+                    me = de[j];
+                    mo = dd[j];
+                    if constexpr (ROPE && V2) {  // bf16 products, their sums rounded below
+                        me = f2_add(round_pair<T>(f2_mul(de[j], c2[j])), round_pair<T>(f2_mul(dd[j], s2[j])));
+                        mo = f2_add(round_pair<T>(f2_mul(dd[j], c2[j])), round_pair<T>(f2_mul(de[j], n2[j])));
+                    } else if constexpr (ROPE) {  // R^T: (c dy0 + s dy1, -s dy0 + c dy1)
+                        me = f2_fma(dd[j], s2[j], f2_mul(de[j], c2[j]));
+                        mo = f2_fma(de[j], n2[j], f2_mul(dd[j], c2[j]));
+                    }
+                    me = round_pair<T>(me);  // gradient of the rotated-in value, Q/K dtype
+                    mo = round_pair<T>(mo);
                 }
-                me = round_pair<T>(me);  // gradient of the rotated-in value, Q/K dtype
-                mo = round_pair<T>(mo);
                 if constexpr (SCALE) {   // through the query_scale cast
                     me = round_pair<T>(f2_mul(me, qs2));
                     mo = round_pair<T>(f2_mul(mo, qs2));

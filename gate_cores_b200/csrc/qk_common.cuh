@@ -87,5 +87,26 @@ __device__ __forceinline__ void rope_eo(f32x2& e, f32x2& o, f32x2 c, f32x2 s, f3
     }
 }
 
+// ---- bf16 pairs in one 32-bit word (low half = first element).
+// Word of the low halves of w0 and w1, and of their high halves.
+__device__ __forceinline__ uint32_t lo_halves(uint32_t w0, uint32_t w1) { return __byte_perm(w0, w1, 0x5410); }
+__device__ __forceinline__ uint32_t hi_halves(uint32_t w0, uint32_t w1) { return __byte_perm(w0, w1, 0x7632); }
+// Products and sums of bf16 pairs, each rounded once to bf16 (round to
+// nearest even).  For bf16 operands they equal the FP32 operation followed
+// by a cast to bf16: a product of two 8-bit significands is exact in FP32
+// (for results above FP32's normal minimum), and when a sum of two bf16
+// values rounds in FP32 the smaller term is below 2^-15 of the result, so
+// the FP32 rounding cannot move it onto a bf16 rounding midpoint.
+__device__ __forceinline__ uint32_t bf2_mul(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ uint32_t bf2_add(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 }  // namespace qk
 }  // namespace muse
