@@ -183,7 +183,11 @@ __global__ void __launch_bounds__(256, MINB) qk_norm_rope_kernel(const __grid_co
 
     const bool vok = !TAIL || sub < nvec;
     const uint32_t voff = (uint32_t)sub * 16u;
+    // v2 rotation with bf16 Q/K: the rotation on bf16 pairs (qk::bf2_mul /
+    // bf2_add give the bf16 products and their rounded sums)
+    constexpr bool BF2 = ROPE && !UPCAST && std::is_same<T, __nv_bfloat16>::value;
     f32x2 c2[H], s2[H], n2[H];
+    uint32_t cb[BF2 ? H : 1], sb[BF2 ? H : 1], nb2[BF2 ? H : 1];
     if constexpr (ROPE) {
         const int tb = tok * half + (vok ? sub * (V / 2) : 0);
 #pragma unroll
@@ -191,6 +195,14 @@ __global__ void __launch_bounds__(256, MINB) qk_norm_rope_kernel(const __grid_co
             c2[j] = *reinterpret_cast<const f32x2*>(cs + tb + 2 * j);
             s2[j] = *reinterpret_cast<const f32x2*>(sn + tb + 2 * j);
             n2[j] = f2_mul(s2[j], f2_make(-1.0f, -1.0f));
+            if constexpr (BF2) {  // exact: the table holds bf16 values
+                float lo, hi;
+                f2_split(c2[j], lo, hi);
+                cb[j] = pack_bf16x2(lo, hi);
+                f2_split(s2[j], lo, hi);
+                sb[j] = pack_bf16x2(lo, hi);
+                nb2[j] = pack_bf16x2(-lo, -hi);
+            }
         }
     }
     const f32x2 qs2 = f2_make(a.query_scale, a.query_scale);
@@ -212,6 +224,29 @@ __global__ void __launch_bounds__(256, MINB) qk_norm_rope_kernel(const __grid_co
             }
             const float r = inv_rms_fast(group_sum<L>(f2_sum(acc)), inv_width, a.eps);
             const f32x2 r2 = f2_make(r, r);
+            if constexpr (BF2) {
+                static_assert(H == 2, "a 16-byte vector holds 4 rotation pairs of bf16");
+                uint32_t w[4];
+#pragma unroll
+                for (int j = 0; j < H; ++j) {
+                    f32x2 ev = f2_mul(e[j], r2), ov = f2_mul(o[j], r2);
+                    if constexpr (SCALE) {  // cast, query_scale, cast again (the last cast below)
+                        ev = f2_mul(round_pair<T>(ev), qs2);
+                        ov = f2_mul(round_pair<T>(ov), qs2);
+                    }
+                    float lo, hi;
+                    f2_split(ev, lo, hi);
+                    const uint32_t eb = pack_bf16x2(lo, hi);  // cast to bf16
+                    f2_split(ov, lo, hi);
+                    const uint32_t ob = pack_bf16x2(lo, hi);
+                    const uint32_t er = qk::bf2_add(qk::bf2_mul(eb, cb[j]), qk::bf2_mul(ob, nb2[j]));
+                    const uint32_t orr = qk::bf2_add(qk::bf2_mul(eb, sb[j]), qk::bf2_mul(ob, cb[j]));
+                    w[2 * j] = qk::lo_halves(er, orr);  // rotation pair 2j: (first, second)
+                    w[2 * j + 1] = qk::hi_halves(er, orr);
+                }
+                if (hv[b]) st_vec(dst + (uint32_t)(b * RW) * head_bytes + voff, make_uint4(w[0], w[1], w[2], w[3]));
+                continue;
+            }
 #pragma unroll
             for (int j = 0; j < H; ++j) {
                 f32x2 ev = round_pair<T>(f2_mul(e[j], r2));  // cast to the Q/K dtype
@@ -276,6 +311,13 @@ constexpr int kThreads = 256;
 constexpr int kQkBatch = 4;
 constexpr int kQkRing = 3;
 constexpr int kQkMinBlocks = 4;
+// Warps (= tokens) per CTA when every warp takes whole tokens.  Seven: four
+// CTAs per SM still (64 registers), and 8192 tokens make 1.98 waves of the
+// 592 CTA slots instead of 1.73 with eight; measured on B200 at prefill, the
+// five-core step 166.6 -> 162.4 us (Q/K alone 29.3 -> 29.0 us back to back),
+// 1% faster on the 80k-token packed batch, unchanged at 32k tokens x 8192;
+// six, five or four warps per CTA gained nothing.
+constexpr int kQkWarpsWhole = 7;
 
 template <typename T, int L, int VPL, int CH>
 cudaError_t launch_head_gate_l(const HeadGateArgs& a, cudaStream_t s) {
@@ -317,11 +359,12 @@ cudaError_t launch_qk_l(const QkArgs& a0, cudaStream_t s) {
            (a.tokens * split + nwarps - 1) / nwarps < 2 * sm_count())
         split *= 2;
     a.split = split;
-    const int tt = nwarps / split;
+    const int threads = split == 1 ? 32 * kQkWarpsWhole : kThreads;
+    const int tt = split == 1 ? kQkWarpsWhole : nwarps / split;
     const uint32_t head_bytes = (uint32_t)a.head_dim * (uint32_t)sizeof(T);
     const size_t table = ((size_t)2 * tt * (a.head_dim / 2) * 4 + 127) & ~(size_t)127;
     const size_t slot = ((size_t)BATCH * RW * head_bytes + 127) & ~(size_t)127;
-    const size_t smem = table + (size_t)nwarps * kQkRing * slot;
+    const size_t smem = table + (size_t)(threads / 32) * kQkRing * slot;
     const int64_t grid = (a.tokens + tt - 1) / tt;
     const bool exact = split == 1 && a.head_dim / Vec<T>::N == L && a.hq % RW == 0 &&
                        a.hkv % RW == 0 && nst_q % BATCH == 0 && nst_k % BATCH == 0;
@@ -331,7 +374,7 @@ cudaError_t launch_qk_l(const QkArgs& a0, cudaStream_t s) {
     // (the mbarriers are static), so it is always set
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(kern, (unsigned)grid, kThreads, smem, s, a);
+    return launch_pdl(kern, (unsigned)grid, (unsigned)threads, smem, s, a);
 }
 
 template <typename T, int L>
