@@ -25,6 +25,13 @@ WLS = [
     Workload("ragged_t1_h4096", hidden=4096, hq=32, hkv=8, head_dim=128, rope_base=5.0e5, batch=1, seqlen=1),
     Workload("ragged_t300_h8192", hidden=8192, hq=64, hkv=8, head_dim=128, rope_base=5.0e5, batch=3,
              seqlen=100, outlier_frac=0.01),
+    # core 5 rows of 514 / 640 / 1024 vectors run on CTA pairs (idle consumers
+    # in each half at 514); 513 vectors (odd) on one CTA with two slots
+    Workload("ragged_t97_h4112", hidden=4112, hq=32, hkv=8, head_dim=128, rope_base=5.0e5, batch=1, seqlen=97),
+    Workload("ragged_t61_h4104", hidden=4104, hq=32, hkv=8, head_dim=128, rope_base=5.0e5, batch=1, seqlen=61),
+    Workload("ragged_t203_h5120", hidden=5120, hq=40, hkv=8, head_dim=128, rope_base=5.0e5, batch=1, seqlen=203),
+    Workload("mid_t2048_h8192", hidden=8192, hq=64, hkv=8, head_dim=128, rope_base=5.0e5, batch=1,
+             seqlen=2048, outlier_frac=0.01),
     inputs.WORKLOADS["prefill_t8192_h4096"],
 ]
 ROW_CASES = [("rms_norm", v) for v in ("zc_gain", "plain_gain", "no_gain", "f32_io")] + \
