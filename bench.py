@@ -284,10 +284,15 @@ class BwdStep:
         elif core == "qk_norm_rope":
             qw, kw = wl.hq * wl.head_dim, wl.hkv * wl.head_dim
             pos = d["positions"]
+            if self.st.thd:
+                cu = d["cu_seqlens"]
+                layout, bsz, sl, cup, nseq = L.MUSE_LAYOUT_THD, 0, 0, cu.data_ptr(), cu.numel() - 1
+            else:
+                layout, bsz, sl, cup, nseq = L.MUSE_LAYOUT_BSHD, wl.batch, wl.seqlen, None, 0
             L.muse_qk_norm_rope_backward(
                 d["q"].data_ptr(), d["k"].data_ptr(), self.dy["qk_q"].data_ptr(), self.dy["qk_k"].data_ptr(),
-                self.out["dq"].data_ptr(), self.out["dk"].data_ptr(), bf, L.MUSE_LAYOUT_BSHD, wl.batch,
-                wl.seqlen, None, 0, T, None if pos is None else pos.data_ptr(), wl.hq, wl.hkv,
+                self.out["dq"].data_ptr(), self.out["dk"].data_ptr(), bf, layout, bsz, sl, cup, nseq, T,
+                None if pos is None else pos.data_ptr(), wl.hq, wl.hkv,
                 wl.head_dim, qw, kw, qw, kw, qw, kw, sc["eps"], 1.0, True, self.qk_upcast, sc["rope_base"],
                 stream)
         elif core == "output_norm_gate":
@@ -556,9 +561,9 @@ class LaunchFloor:
 def per_config(args, peak: float, rank: int, world: int,
                names=("thd16_h5120", "large_t32768_h8192")):
     """The five cores on the other full-size workloads: per-core steady-state
-    figures (per_core_steady), the five-core step (K steps back to back, two
-    events), and the oracle on all host cores on a bounded sample of the same
-    batch (rank 0, one GPU)."""
+    figures (per_core_steady) of the forward and of the backward calls, the
+    five-core step (K steps back to back, two events), and the oracle on all
+    host cores on a bounded sample of the same batch (rank 0, one GPU)."""
     stream = torch.cuda.current_stream()
     reps = max(10, min(args.steps, 50))
     out = {}
@@ -585,6 +590,9 @@ def per_config(args, peak: float, rank: int, world: int,
                "step": {"ms": round(el / reps * 1e3, 4), "tokens_per_s": round(world * st.T * reps / el, 1),
                         "gbs": round(nb * reps / el / 1e9, 1), "frac": round(nb * reps / el / 1e9 / peak, 4),
                         "algo_bytes": nb, "steps": reps}}
+        bst = BwdStep(st, seed=rank)
+        rec["backward_steady"] = per_core_steady(bst, peak, reps, nbytes=algo_bytes_bwd)
+        del bst
         if rank == 0 and world == 1 and args.cpu_baseline:
             rec["cpu_oracle_all_cores"] = cpu_baseline_threads(wl, seconds=4.0, host=st.host)
         out[name] = rec
