@@ -920,11 +920,7 @@ def run_ours(args, world, rank, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16 activations, FP32 residual stream)",
-            "config": {"workload": wl.name, "tokens_per_gpu": T, "batch": wl.batch, "seq_len": wl.seqlen,
-                       "hidden": wl.hidden, "q_heads": wl.hq, "kv_heads": wl.hkv,
-                       "head_dim": wl.head_dim, "parallelism": f"token shards x{world} (no collective)",
-                       "l2": "no flush: each step streams %.2f GB, > 126 MB L2"
-                             % (sum(algo_bytes(wl, c, T) for c in CORE_ORDER) / 1e9)},
+            "config": run_config(wl, T, world),
             "per_core": per_core,
             "per_core_steady": steady,
             "per_core_isolated": isolated,
@@ -1019,6 +1015,15 @@ def run_e2e(st: Step, args, world):
 
 # ------------------------------------------------------------------ reference arm
 
+def run_config(wl, tokens: int, world: int) -> dict:
+    """The `config` of the JSON line (both arms)."""
+    return {"workload": wl.name, "tokens_per_gpu": tokens, "batch": wl.batch, "seq_len": wl.seqlen,
+            "hidden": wl.hidden, "q_heads": wl.hq, "kv_heads": wl.hkv, "head_dim": wl.head_dim,
+            "parallelism": f"token shards x{world} (no collective)",
+            "l2": "no flush: each step streams %.2f GB, > 126 MB L2"
+                  % (sum(algo_bytes(wl, c, tokens) for c in CORE_ORDER) / 1e9)}
+
+
 def run_reference(args, world, rank):
     """The oracle (plain double-precision C, single-threaded) on the host cores:
     each step is a bounded sample (64 consecutive tokens, rotating through the
@@ -1053,10 +1058,10 @@ def run_reference(args, world, rank):
         "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded, same generator as the GPU arm)",
-        "config": {"workload": wl.name, "tokens_per_step": per_step, "hidden": wl.hidden,
-                   "q_heads": wl.hq, "kv_heads": wl.hkv, "head_dim": wl.head_dim},
+        "config": run_config(wl, T, world),
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{per_step} consecutive tokens per step of {wl.name}, all five cores"},
+                         "sample": f"{per_step} consecutive tokens per step of the {T}-token batch of {wl.name} "
+                                   f"(rotating through it), all five cores; value = tokens of the samples / time"},
         "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
