@@ -245,21 +245,21 @@ __global__ void __launch_bounds__(256, MINB) qk_norm_rope_kernel(const __grid_co
                     w[2 * j + 1] = qk::hi_halves(er, orr);
                 }
                 if (hv[b]) st_vec(dst + (uint32_t)(b * RW) * head_bytes + voff, make_uint4(w[0], w[1], w[2], w[3]));
-                continue;
-            }
+            } else {
 #pragma unroll
-            for (int j = 0; j < H; ++j) {
-                f32x2 ev = round_pair<T>(f2_mul(e[j], r2));  // cast to the Q/K dtype
-                f32x2 ov = round_pair<T>(f2_mul(o[j], r2));
-                if constexpr (SCALE) {                      // query_scale, cast again
-                    ev = round_pair<T>(f2_mul(ev, qs2));
-                    ov = round_pair<T>(f2_mul(ov, qs2));
+                for (int j = 0; j < H; ++j) {
+                    f32x2 ev = round_pair<T>(f2_mul(e[j], r2));  // cast to the Q/K dtype
+                    f32x2 ov = round_pair<T>(f2_mul(o[j], r2));
+                    if constexpr (SCALE) {                      // query_scale, cast again
+                        ev = round_pair<T>(f2_mul(ev, qs2));
+                        ov = round_pair<T>(f2_mul(ov, qs2));
+                    }
+                    if constexpr (ROPE) qk::rope_eo<T, UPCAST>(ev, ov, c2[j], s2[j], n2[j]);
+                    e[j] = ev;
+                    o[j] = ov;
                 }
-                if constexpr (ROPE) qk::rope_eo<T, UPCAST>(ev, ov, c2[j], s2[j], n2[j]);
-                e[j] = ev;
-                o[j] = ov;
+                if (hv[b]) st_vec(dst + (uint32_t)(b * RW) * head_bytes + voff, qk::from_eo<T>(e, o));
             }
-            if (hv[b]) st_vec(dst + (uint32_t)(b * RW) * head_bytes + voff, qk::from_eo<T>(e, o));
         }
     };
 
