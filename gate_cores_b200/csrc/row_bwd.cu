@@ -373,8 +373,10 @@ __device__ __forceinline__ void row_bwd_body(const RowBwdArgs& a) {
 #pragma unroll
             for (int q = 0; q < P; ++q) {
                 if constexpr (FIRST) {
-                    const f32x2 u = f2_mul(x[i][q], w[i][q]);
-                    const f32x2 dz = f2_fma(u, ncr2, f2_mul(r2, g[i][q]));
+                    // dz = r g - cr x w as x (-cr w) + r g: the first pass's x w
+                    // then dies at the barrier instead of staying live across it
+                    // (that held 16 more registers; at 8192 columns it spilled)
+                    const f32x2 dz = f2_fma(x[i][q], f2_mul(ncr2, w[i][q]), f2_mul(r2, g[i][q]));
                     d[q] = f2_mul(dz, w[i][q]);
                     if constexpr (G) acc_g[i][q] = f2_fma(dz, x[i][q], acc_g[i][q]);
                 } else {
