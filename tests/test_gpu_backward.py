@@ -195,3 +195,46 @@ def test_qk_norm_rope_backward(cuda_ok, wl, variant):
 
 def test_no_device_error_after_backward_runs(cuda_ok):
     assert _lib.muse_device_error() == 0
+
+
+def test_backward_graph_replay_matches_eager(cuda_ok):
+    # captured backward calls (the row kernel and its fixed-order reduction of
+    # the parameter partials, programmatic launches and, for core 5, both
+    # parameter gradients) replay to the eager calls' bits
+    wl = inputs.WORKLOADS["prefill_t8192_h4096"]
+    ci = harness.make(wl, "rms_norm", "zc_gain")
+    x, g = ci.tensors["x"].cuda(), ci.tensors["gain"].cuda()
+    dy = inputs.upstream_grad(wl, 0, "rms_norm", tuple(x.shape), x.dtype).cuda()
+    ws = torch.empty(_lib.muse_norm_backward_workspace_bytes(x.shape[0], x.shape[1]), dtype=torch.uint8,
+                     device="cuda")
+    ref_dx, ref_dg = cores.rms_norm_backward(x, dy, g, 1.0, 1e-6, workspace=ws)
+    cr = harness.make(wl, "norm_residual", "gain_after")
+    t, s = cr.tensors, cr.scalars
+    h, b, th, gr = (t[k].cuda() for k in ("stream", "branch", "theta", "gain"))
+    dout = inputs.upstream_grad(wl, 0, "norm_residual", tuple(h.shape), torch.float32).cuda()
+    ws5 = torch.empty(_lib.muse_norm_backward_workspace_bytes(h.shape[0], h.shape[1]), dtype=torch.uint8,
+                      device="cuda")
+    res = (h, b, dout, th, gr, s["gain_offset"], False, s["norm_eps"])
+    ref5 = cores.norm_residual_backward(*res, workspace=ws5)
+    dx = torch.empty_like(x)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm-up outside the capture
+        cores.rms_norm_backward(x, dy, g, 1.0, 1e-6, dx=dx, workspace=ws)
+        cores.norm_residual_backward(*res, workspace=ws5)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        out = cores.rms_norm_backward(x, dy, g, 1.0, 1e-6, dx=dx, workspace=ws)
+        out5 = cores.norm_residual_backward(*res, workspace=ws5)
+    for _ in range(3):
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out[0].view(torch.int16), ref_dx.view(torch.int16))
+        assert torch.equal(out[1].view(torch.int32), ref_dg.view(torch.int32))
+        for u, v in zip(out5, ref5):
+            assert torch.equal(u.view(torch.int32) if u.dtype == torch.float32 else u.view(torch.int16),
+                               v.view(torch.int32) if v.dtype == torch.float32 else v.view(torch.int16))
+    del graph
+    assert _lib.muse_device_error() == 0
