@@ -57,11 +57,13 @@ __host__ __device__ constexpr bool b_gain_first(BwdOp op) { return op == BwdOp::
 
 // At most this many resident CTAs per SM (bounds the workspace).
 constexpr int kBwdMaxCtasPerSm = 4;
-// CTAs per cluster for core 5 rows of more than 512 vectors.  Measured on
-// B200 (32768 rows of 8192 / 80251 rows of 5120): two CTAs 785 / 1451 us
-// launched back to back and 765 / 1431 us alone; four CTAs 1272 / 1885 us
-// back to back although 693 / 1165 us alone.
-constexpr int kSplitCtas = 2;
+// CTAs per cluster for core 5 rows of more than 512 vectors (two when the
+// vector count does not divide by four).  Measured on B200 (32768 rows of
+// 8192 / 80251 rows of 5120), launched back to back / alone: four CTAs 716 /
+// 695 and 1204 / 1158 us, two CTAs 776 / 765 and 1453 / 1433 us.  Cluster
+// launches go without programmatic dependent launch: with it, four-CTA
+// clusters launched back to back took 1285 / 1815 us.
+constexpr int kSplitCtas = 4;
 
 __host__ __device__ inline uint32_t al128(uint32_t v) { return (v + 127u) & ~127u; }
 
@@ -514,24 +516,23 @@ int resident_clusters(const void* kernel, int threads, size_t smem, int cl) {
     return n;
 }
 
-// launch_pdl for clusters of `cl` CTAs along x.
+// Launch in clusters of `cl` CTAs along x (stream-ordered: no programmatic
+// dependent launch, which slowed four-CTA clusters launched back to back).
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), unsigned cl, unsigned grid, unsigned block, size_t smem,
-                               cudaStream_t stream, Args&&... args) {
+cudaError_t launch_cluster(void (*kernel)(KArgs...), unsigned cl, unsigned grid, unsigned block, size_t smem,
+                           cudaStream_t stream, Args&&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(block);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = cl;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
@@ -570,7 +571,7 @@ cudaError_t launch_bwd_s(RowBwdArgs a, int nvec, float* dgain, float* dtheta, cu
     if constexpr (CL == 1)
         e = launch_pdl(kern, (unsigned)grid, (unsigned)threads, smem, s, a);
     else
-        e = launch_pdl_cluster(kern, (unsigned)CL, (unsigned)grid, (unsigned)threads, smem, s, a);
+        e = launch_cluster(kern, (unsigned)CL, (unsigned)grid, (unsigned)threads, smem, s, a);
     if (e != cudaSuccess) return e;
     const unsigned rgrid = (unsigned)((a.width + 31) / 32);
     if (a.part_gain) {
