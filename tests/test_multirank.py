@@ -61,3 +61,10 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+    # the same workload description as the GPU arm prints at this rank count
+    sys.path.insert(0, ROOT)
+    import bench
+    from gate_cores_b200.inputs import WORKLOADS, num_tokens
+    wl = WORKLOADS["prefill_t8192_h4096"]
+    assert d["config"] == bench.run_config(wl, num_tokens(wl), 2)
+    assert d["metric"] == bench.METRIC and d["unit"] == "tokens/s" and d["higher_is_better"] is True
